@@ -1,0 +1,354 @@
+"""Throughput of the Inkling MoE feed-forward layer on B200 (one JSON line).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl reference]
+
+A step is one full forward pass of the layer (router, permutation, routed and
+shared expert GEMMs, recombination) over one batch of T tokens, through the
+library's C ABI, inputs resident in HBM.  The default workload is the layer
+at the pages' hidden size: T=8192, H=6144, E=128, k=8, S=1, I=2048, bf16.
+
+N > 1 (launched by torch.distributed.run): every rank runs an independent
+replica on its own GPU with its own token batch; the layer has no exchange
+step, so there is no collective on the data path (weak scaling).  Timing is
+taken on the device with CUDA events and reduced as the max over ranks.
+
+``--impl reference`` times the CPU fp64 oracle instead, on a bounded token
+sample per step, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import moe_workloads as mw  # noqa: E402
+
+METRIC = "Inkling MoE-layer tokens/s and TFLOP/s (% of B200 bf16 peak / % HBM BW), 1 GPU"
+DEFAULT_WORKLOAD = "bf16-T8192-H6144-E128k8S1-I2048"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes per launch of the expert GEMMs measured by ncu on this workload
+# (dram__bytes_read.sum + dram__bytes_write.sum); None until captured for the
+# current kernel build.
+NCU_TRAFFIC_BYTES = {}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        if self.path is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[4:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        seen = set()
+        for _, _, flags in rows:
+            for n, v in zip(names, flags[1:]):
+                if v.lower() == "active":
+                    seen.add(n)
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(seen), "samples": len(rows)}
+
+
+# ------------------------------------------------------------- distributed
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def finish(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------- CPU (oracle) arm
+def oracle_run(w, inputs, tokens_per_step: int, steps: int, warmup: int, threads: int):
+    import oracle
+    torch.set_num_threads(threads)
+    n_done = 0
+    t_total = 0.0
+    for i in range(warmup + steps):
+        tok = mw.token_sample(w, tokens_per_step, seed_offset=1000 + i)
+        t0 = time.perf_counter()
+        oracle.moe_forward_workload(inputs, w, tokens=tok, threads=threads)
+        dt = time.perf_counter() - t0
+        if i >= warmup:
+            n_done += tok.numel()
+            t_total += dt
+    return n_done / t_total, n_done, t_total
+
+
+def cpu_baseline(w, inputs, budget_s: float = 15.0):
+    """The oracle as it stands on the host cores, on a bounded token sample."""
+    threads = len(os.sched_getaffinity(0))
+    per_token_guess = max(1e-3, mw.flops(w, 1)["total"] / 60e9)   # rough fp64 rate
+    n = int(max(4, min(w.T, 256, budget_s / per_token_guess / 2)))
+    tps, done, secs = oracle_run(w, inputs, n, 1, 0, threads)
+    return {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} seeded tokens of {w.name} (oracle fp64, {secs:.1f} s)"}
+
+
+def reference_arm(args, world, rank):
+    """Rank 0 alone runs the oracle; other ranks exit at once (no process group)."""
+    w = mw.by_name(args.workload)
+    if rank != 0:
+        return
+    inputs = mw.generate(w)
+    threads = len(os.sched_getaffinity(0))
+    # bounded sample per step so that warmup + steps stay within a few minutes
+    tokens_per_step = int(max(1, min(64, 240 // max(1, args.steps + args.warmup))))
+    tps, done, secs = oracle_run(w, inputs, tokens_per_step, args.steps, args.warmup, threads)
+    fl = mw.flops(w, 1)["total"]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "H": w.H, "E": w.E, "k": w.k, "S": w.S, "I": w.I,
+                   "tokens_per_step": tokens_per_step},
+        "tflops": tps * fl / 1e12,
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{tokens_per_step} seeded tokens per step of {w.name}"},
+        "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- GPU arm
+def gpu_arm(args, world, rank, local):
+    import mixture_experts_feed_b200 as moe
+
+    w = mw.by_name(args.workload)
+    # every replica gets its own token batch (x seed differs per rank); same weights
+    wr = w.replace(seed=w.seed) if rank == 0 else w
+    inputs = mw.generate(wr)
+    if rank > 0:
+        g = torch.Generator().manual_seed(10_000 + rank)
+        inputs["x"] = torch.randn(w.T, w.H, generator=g).to(w.torch_dtype)
+    L = moe.Layer.from_workload(w)
+    dev = torch.device("cuda", local)
+    d = {k: v.to(dev).contiguous() for k, v in inputs.items()}
+    x_host = inputs["x"].pin_memory()
+    stream = torch.cuda.current_stream(dev)
+    ws = moe.new_workspace(L, device=dev)
+    T, k, S, H, E = L.T, L.k, L.S, L.H, L.E
+    tw = torch.empty(T, k, dtype=torch.float32, device=dev)
+    ti = torch.empty(T, k, dtype=torch.int32, device=dev)
+    sg = torch.empty(T, S, dtype=torch.float32, device=dev) if S else None
+    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    ps = torch.empty(T * k, dtype=torch.int32, device=dev)
+    ip = torch.empty(T * k, dtype=torch.int32, device=dev)
+    xp = torch.empty(T * k, H, dtype=L.dtype, device=dev)
+    yr = torch.empty(T * k, H, dtype=torch.float32, device=dev)
+    ys = torch.empty(S * T, H, dtype=torch.float32, device=dev) if S else None
+    out = torch.empty(T, H, dtype=L.dtype, device=dev)
+    out_host = torch.empty(T, H, dtype=L.dtype).pin_memory()
+    wsgu = d.get("ws_gate_up") if S else None
+    wsd = d.get("ws_down") if S else None
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        moe.moe_route(L, d["x"], d["w_router"], d["corr_bias"], tw, ti, sg, ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        moe.moe_permute(L, ti, None, d["x"], off, ps, ip, xp, ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        moe.moe_expert_ffn(L, d["x"], xp, off, ps, tw, sg, d["w_gate_up"], d["w_down"], wsgu, wsd,
+                           yr, ys, ws, stream)
+        if ev is not None:
+            ev[3].record(stream)
+        moe.moe_combine(L, yr, ys, ip, out, ws, stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    moe.read_device_status(ws, stream)
+
+    # ---- timed region: K steps, inputs (weights 9.7 GB at the default
+    # workload) far larger than the 126 MB L2, so no flush is needed between steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            step(evs[i])
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    clocks = clk.summary()
+    moe.read_device_status(ws, stream)
+    total_ms = evs[0][0].elapsed_time(evs[-1][4])
+    op_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(4)]
+    ms_step = max_over_ranks(total_ms / args.steps, world)
+
+    # ---- end to end through the public one-call API with host buffers
+    def e2e_step():
+        d["x"].copy_(x_host, non_blocking=True)
+        moe.moe_forward(L, d["x"], d["w_router"], d["corr_bias"], d["w_gate_up"], d["w_down"],
+                        wsgu, wsd, out, ws, stream=stream)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup // 2)):
+        e2e_step()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    moe.read_device_status(ws, stream)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        fl = mw.flops(w)
+        ffn_flops = fl["routed"] + fl["shared"]
+        ffn_s = op_ms[2] / 1e3
+        achieved = ffn_flops / ffn_s / 1e12
+        peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        tokens_s = world * T / (ms_step / 1e3)
+        line = {
+            "metric": METRIC, "value": tokens_s, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+            "data": "synthetic (seeded N(0,1) activations, N(0,0.02^2) weights, random init)",
+            "config": {"workload": w.name, "T": T, "H": H, "E": E, "k": k, "S": S, "I": w.I,
+                       "route_scale": w.route_scale, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (expert weights %.1f GB)" % (mw.weight_bytes(w) / 1e9)},
+            "tflops": world * fl["total"] / (ms_step / 1e3) / 1e12,
+            "op_ms": {"route": op_ms[0], "permute": op_ms[1], "expert_ffn": op_ms[2], "combine": op_ms[3]},
+            "roofline": {"kernel": "grouped expert GEMMs (gate_up + down launches of moe_expert_ffn)",
+                         "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak,
+                         "peak_source": f"{peak_src} bf16_tflops_sustained",
+                         "traffic": NCU_TRAFFIC_BYTES.get(w.name)},
+            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+                    "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
+            "gpu_launches": moe.forward_kernel_count(L) * args.steps,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, inputs)
+        print(json.dumps(line), flush=True)
+    finish(world)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)   # at least three untimed warm-up steps
+    if args.impl == "reference":
+        reference_arm(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+        return
+    world, rank, local = dist_setup(args)
+    gpu_arm(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,186 @@
+/*
+ * inkling_moe.h — C ABI of libinklingmoe.so, the B200 (sm_100a) forward pass
+ * of the Inkling mixture-of-experts feed-forward layer.
+ *
+ * The layer, as the NeMo AutoModel Inkling pages state it ("layers" page):
+ *   - InklingGate: fp32 router logits over a gate weight bank of E routed rows
+ *     followed by S shared rows; selection of k experts by sigmoid score plus
+ *     the fp32 correction bias (InklingCorrectionBias); output weights from a
+ *     softmax over the log-sigmoid of the k selected routed logits
+ *     concatenated with the S shared logits, times route_scale*global_scale.
+ *     The first k weights go to the routed experts, the last S (the gammas)
+ *     to the always-on shared experts.
+ *   - InklingSharedExperts: every token through every shared expert, each
+ *     output weighted by its gamma, summed.
+ *   - routed experts: fused gate/up projection whose output interleaves
+ *     gate and up channels ([g0, u0, g1, u1, ...]), SwiGLU scaled by the
+ *     routing weight (inkling_swiglu), down projection.
+ *   - InklingMoE.forward: shared plus routed, recombined per token; leading
+ *     dims of the input are flattened to tokens by the caller; padded tokens
+ *     are excluded from routed dispatch.
+ *
+ * Conventions shared by every entry point
+ *   - All tensors are caller-owned DEVICE buffers, row-major and contiguous,
+ *     16-byte aligned.  The library never allocates or frees memory.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL means the legacy default stream).  The host-side argument check
+ *     runs before any launch; a non-OK return means nothing was launched
+ *     (MOE_ERR_CUDA: a launch was attempted and CUDA reported an error).
+ *   - Weights use the checkpoint's [out_features, in_features] orientation
+ *     (the pages note the fused projection stays in the checkpoint layout so
+ *     loading needs only transpose views):
+ *       w_router   [E+S, H] fp32    rows 0..E-1 routed, E..E+S-1 shared
+ *       corr_bias  [E]      fp32
+ *       w_gate_up  [E, 2I, H]       row 2j = gate_j, row 2j+1 = up_j
+ *       w_down     [E, H, I]
+ *       ws_gate_up [S, 2I, H], ws_down [S, H, I]   (shared experts)
+ *     x, the expert weights, x_perm and out share `dtype`; the expert output
+ *     rows y_routed / y_shared are fp32 in every dtype (they are summed in
+ *     fp32 and rounded once, in moe_combine).
+ *   - Sizes: T = num_tokens, H = hidden, E = n_routed, k = top_k,
+ *     S = n_shared, I = intermediate.  Limits: 1 <= k <= min(E, 16),
+ *     E <= 1024, S <= 8, H % 64 == 0, I % 64 == 0, T*(k+S) < 2^31.
+ *     T = 0 is accepted and launches nothing.
+ *   - `workspace` is a device buffer of at least moe_workspace_size() bytes.
+ *     Its first 256 bytes hold a sticky device status word; zero them once
+ *     with moe_workspace_init() before first use.  Kernels that detect a bad
+ *     index or a stalled pipeline record it there instead of faulting;
+ *     moe_read_device_status() reads and clears it.
+ *   - Calls sharing one workspace must be ordered on one stream.
+ */
+#ifndef INKLING_MOE_H
+#define INKLING_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned buffer */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid layer outside this build's limits */
+  MOE_ERR_WORKSPACE = 3,     /* workspace smaller than moe_workspace_size() */
+  MOE_ERR_CUDA = 4,          /* the CUDA runtime reported an error */
+  MOE_ERR_DEVICE_CHECK = 5,  /* a kernel saw an out-of-range index */
+  MOE_ERR_TIMEOUT = 6        /* a kernel's bounded pipeline wait expired */
+} moe_status_t;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+
+/* Layer description (the MoE fields of InklingTextConfig, with T added). */
+typedef struct {
+  int64_t num_tokens;    /* T: product of the input's leading dims */
+  int32_t hidden;        /* H: hidden_size */
+  int32_t n_routed;      /* E: n_routed_experts */
+  int32_t top_k;         /* k: num_experts_per_tok */
+  int32_t n_shared;      /* S: n_shared_experts */
+  int32_t intermediate;  /* I: moe_intermediate_size (shared experts too) */
+  int32_t dtype;         /* moe_dtype_t of x, expert weights and outputs */
+  float route_scale;     /* route_scale */
+  float global_scale;    /* the gate's global_scale parameter (1.0 at init) */
+} moe_layer_desc_t;
+
+/* Workspace bytes every entry point below accepts for this layer. */
+moe_status_t moe_workspace_size(const moe_layer_desc_t* desc, size_t* bytes);
+
+/* Zero the device status word at the head of `workspace` (async). */
+moe_status_t moe_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Read the device status word (synchronises `stream`), then clear it.
+ * Returns MOE_OK, MOE_ERR_DEVICE_CHECK or MOE_ERR_TIMEOUT; `*device_code`
+ * receives the raw word (0 when clean; may be NULL). */
+moe_status_t moe_read_device_status(void* workspace, void* stream, int32_t* device_code);
+
+/*
+ * moe_route — InklingGate.forward (layers page, InklingGate docstring;
+ * InklingCorrectionBias.forward).
+ *   x            [T, H]    dtype
+ *   w_router     [E+S, H]  fp32
+ *   corr_bias    [E]       fp32 (selection only)
+ *   topk_w       [T, k]    fp32 out: routed weights, best expert first
+ *   topk_idx     [T, k]    int32 out: expert ids by descending score
+ *                          sigmoid(z)+bias; ties go to the lower id
+ *   shared_gamma [T, S]    fp32 out (may be NULL when S == 0)
+ * Logits are computed in fp32.  Sum over a token of topk_w and shared_gamma
+ * equals route_scale*global_scale.
+ */
+moe_status_t moe_route(const moe_layer_desc_t* desc, const void* x, const float* w_router,
+                       const float* corr_bias, float* topk_w, int32_t* topk_idx,
+                       float* shared_gamma, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/*
+ * moe_permute — grouped dispatch order for the routed experts (layers page,
+ * InklingMoE docstring: grouped routed experts; InklingMoE.forward: padded
+ * tokens are excluded from routed dispatch).  Every live (token t, choice j)
+ * pair becomes one row; rows are ordered by (expert, token) ascending.
+ *   topk_idx       [T, k] int32 in, values in [0, E)
+ *   padding_mask   [T] uint8 (nonzero = padded) or NULL
+ *   x              [T, H] dtype in
+ *   expert_offsets [E+1] int32 out: rows of expert e are [off[e], off[e+1])
+ *   perm_slot      [T*k] int32 out: for row r < off[E], the slot t*k+j it holds
+ *   inv_perm       [T*k] int32 out: for slot t*k+j, its row, or -1 if padded
+ *   x_perm         [T*k, H] dtype out: row r = x[perm_slot[r] / k]
+ * The order is deterministic (no atomics decide it).
+ */
+moe_status_t moe_permute(const moe_layer_desc_t* desc, const int32_t* topk_idx,
+                         const uint8_t* padding_mask, const void* x, int32_t* expert_offsets,
+                         int32_t* perm_slot, int32_t* inv_perm, void* x_perm, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/*
+ * moe_expert_ffn — the routed experts over the permuted rows and the shared
+ * experts over all tokens (layers page: inkling_swiglu, InklingSharedExperts).
+ * For routed row r of expert e (token t, choice j, weight w = topk_w[t*k+j]):
+ *   y_routed[r] = ( w * silu(G[0::2]) * G[1::2] ) @ w_down[e]^T,
+ *   G = x_perm[r] @ w_gate_up[e]^T                       (fp32 accumulation)
+ * and for shared expert s and token t (weight shared_gamma[t*S+s]) the same
+ * with x[t] and ws_*[s] into y_shared[s*T + t].  The activated rows are
+ * rounded to dtype before the down projection; y rows are written in fp32.
+ *   x [T,H], x_perm [T*k,H], expert_offsets, perm_slot, topk_w [T*k],
+ *   shared_gamma [T*S] (NULL iff S == 0), weights as above,
+ *   y_routed [T*k, H] fp32 out (rows < off[E] written), y_shared [S*T, H] fp32 out.
+ */
+moe_status_t moe_expert_ffn(const moe_layer_desc_t* desc, const void* x, const void* x_perm,
+                            const int32_t* expert_offsets, const int32_t* perm_slot,
+                            const float* topk_w, const float* shared_gamma,
+                            const void* w_gate_up, const void* w_down, const void* ws_gate_up,
+                            const void* ws_down, void* y_routed, void* y_shared,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * moe_combine — InklingMoE.forward recombination:
+ *   out[t] = sum_s y_shared[s*T + t] + sum_{j<k, inv_perm[t*k+j] >= 0} y_routed[inv_perm[t*k+j]]
+ * summed in fp32 in that fixed order, rounded once to dtype.  y_routed and
+ * y_shared are fp32; out [T, H] has `dtype`.
+ */
+moe_status_t moe_combine(const moe_layer_desc_t* desc, const void* y_routed, const void* y_shared,
+                         const int32_t* inv_perm, void* out, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/*
+ * moe_forward — InklingMoE.forward in one call: moe_route, moe_permute,
+ * moe_expert_ffn, moe_combine with every intermediate in `workspace`.
+ *   out [T, H] dtype.  topk_w, topk_idx, shared_gamma are optional outputs
+ *   (NULL: kept in the workspace).  padding_mask may be NULL.
+ */
+moe_status_t moe_forward(const moe_layer_desc_t* desc, const void* x, const float* w_router,
+                         const float* corr_bias, const void* w_gate_up, const void* w_down,
+                         const void* ws_gate_up, const void* ws_down, const uint8_t* padding_mask,
+                         void* out, float* topk_w, int32_t* topk_idx, float* shared_gamma,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Number of kernels moe_forward launches for this layer (for launch accounting). */
+int32_t moe_forward_kernel_count(const moe_layer_desc_t* desc);
+
+const char* moe_status_string(moe_status_t status);
+int32_t moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INKLING_MOE_H */

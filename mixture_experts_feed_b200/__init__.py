@@ -1,0 +1,277 @@
+"""Python binding of libinklingmoe.so, the B200 Inkling MoE feed-forward.
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch supplies device memory and streams.  The entry points keep
+the C names (``moe_route``, ``moe_permute``, ``moe_expert_ffn``,
+``moe_combine``, ``moe_forward``) and take torch tensors whose data pointers
+are handed to the C ABI unchanged; shapes, dtypes and contiguity are checked
+here so that a mistake raises instead of reaching the GPU.
+
+There is no CPU fallback: importing this package raises when the shared
+library has not been built (``python -m mixture_experts_feed_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libinklingmoe.so")
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} is missing; build it with `python -m mixture_experts_feed_b200.build`")
+
+LIB = ctypes.CDLL(_LIB_PATH)
+LIB_PATH = _LIB_PATH
+
+MOE_F32, MOE_BF16 = 0, 1
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
+          4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_CHECK", 6: "MOE_ERR_TIMEOUT"}
+
+
+class LayerDesc(ctypes.Structure):
+    """``moe_layer_desc_t``."""
+    _fields_ = [("num_tokens", ctypes.c_int64), ("hidden", ctypes.c_int32),
+                ("n_routed", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("n_shared", ctypes.c_int32), ("intermediate", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("route_scale", ctypes.c_float),
+                ("global_scale", ctypes.c_float)]
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = LIB.moe_status_string(status).decode()
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({msg})")
+
+
+_P = ctypes.c_void_p
+_DESC = ctypes.POINTER(LayerDesc)
+LIB.moe_status_string.restype = ctypes.c_char_p
+LIB.moe_status_string.argtypes = [ctypes.c_int]
+LIB.moe_version.restype = ctypes.c_int32
+LIB.moe_forward_kernel_count.restype = ctypes.c_int32
+LIB.moe_forward_kernel_count.argtypes = [_DESC]
+LIB.moe_workspace_size.argtypes = [_DESC, ctypes.POINTER(ctypes.c_size_t)]
+LIB.moe_workspace_init.argtypes = [_P, ctypes.c_size_t, _P]
+LIB.moe_read_device_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_int32)]
+LIB.moe_route.argtypes = [_DESC, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+LIB.moe_permute.argtypes = [_DESC, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+LIB.moe_expert_ffn.argtypes = [_DESC] + [_P] * 13 + [ctypes.c_size_t, _P]
+LIB.moe_combine.argtypes = [_DESC, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+LIB.moe_forward.argtypes = [_DESC] + [_P] * 13 + [ctypes.c_size_t, _P]
+for _f in ("moe_workspace_size", "moe_workspace_init", "moe_read_device_status", "moe_route",
+           "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward"):
+    getattr(LIB, _f).restype = ctypes.c_int
+
+
+@dataclass(frozen=True)
+class Layer:
+    """Sizes and scales of one Inkling MoE layer (the ``InklingTextConfig`` MoE fields)."""
+    T: int
+    H: int
+    E: int
+    k: int
+    S: int
+    I: int
+    dtype: torch.dtype = torch.bfloat16
+    route_scale: float = 1.0
+    global_scale: float = 1.0
+
+    def desc(self) -> LayerDesc:
+        code = {torch.float32: MOE_F32, torch.bfloat16: MOE_BF16}.get(self.dtype)
+        if code is None:
+            raise ValueError(f"unsupported dtype {self.dtype}")
+        return LayerDesc(self.T, self.H, self.E, self.k, self.S, self.I, code,
+                         self.route_scale, self.global_scale)
+
+    @staticmethod
+    def from_workload(w) -> "Layer":
+        return Layer(w.T, w.H, w.E, w.k, w.S, w.I, w.torch_dtype, w.route_scale, w.global_scale)
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise MoEError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _expect(t: Optional[torch.Tensor], name: str, shape, dtype, allow_none=False) -> None:
+    if t is None:
+        if allow_none:
+            return
+        raise ValueError(f"{name} is required")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype} != {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def workspace_size(layer: Layer) -> int:
+    n = ctypes.c_size_t(0)
+    _check(LIB.moe_workspace_size(ctypes.byref(layer.desc()), ctypes.byref(n)), "moe_workspace_size")
+    return n.value
+
+
+def new_workspace(layer: Layer, device=None, stream=None) -> torch.Tensor:
+    """Allocate (with torch) and initialise a workspace for ``layer``."""
+    ws = torch.empty(workspace_size(layer), dtype=torch.uint8, device=device or "cuda")
+    _check(LIB.moe_workspace_init(ws.data_ptr(), ws.numel(), _stream(stream)), "moe_workspace_init")
+    return ws
+
+
+def read_device_status(ws: torch.Tensor, stream=None) -> int:
+    """Read and clear the device status word; raises MoEError when it is set."""
+    code = ctypes.c_int32(0)
+    st = LIB.moe_read_device_status(ws.data_ptr(), _stream(stream), ctypes.byref(code))
+    if st != 0:
+        err = MoEError(st, f"device status 0x{code.value:x}")
+        err.device_code = code.value
+        raise err
+    return code.value
+
+
+def moe_route(layer: Layer, x, w_router, corr_bias, topk_w, topk_idx, shared_gamma, ws, stream=None):
+    L = layer
+    _expect(x, "x", (L.T, L.H), L.dtype)
+    _expect(w_router, "w_router", (L.E + L.S, L.H), torch.float32)
+    _expect(corr_bias, "corr_bias", (L.E,), torch.float32)
+    _expect(topk_w, "topk_w", (L.T, L.k), torch.float32)
+    _expect(topk_idx, "topk_idx", (L.T, L.k), torch.int32)
+    _expect(shared_gamma, "shared_gamma", (L.T, L.S), torch.float32, allow_none=L.S == 0)
+    _check(LIB.moe_route(ctypes.byref(L.desc()), _ptr(x), _ptr(w_router), _ptr(corr_bias),
+                         _ptr(topk_w), _ptr(topk_idx), _ptr(shared_gamma), ws.data_ptr(),
+                         ws.numel(), _stream(stream)), "moe_route")
+
+
+def moe_permute(layer: Layer, topk_idx, padding_mask, x, expert_offsets, perm_slot, inv_perm,
+                x_perm, ws, stream=None):
+    L = layer
+    _expect(topk_idx, "topk_idx", (L.T, L.k), torch.int32)
+    _expect(padding_mask, "padding_mask", (L.T,), torch.uint8, allow_none=True)
+    _expect(x, "x", (L.T, L.H), L.dtype)
+    _expect(expert_offsets, "expert_offsets", (L.E + 1,), torch.int32)
+    _expect(perm_slot, "perm_slot", (L.T * L.k,), torch.int32)
+    _expect(inv_perm, "inv_perm", (L.T * L.k,), torch.int32)
+    _expect(x_perm, "x_perm", (L.T * L.k, L.H), L.dtype)
+    _check(LIB.moe_permute(ctypes.byref(L.desc()), _ptr(topk_idx), _ptr(padding_mask), _ptr(x),
+                           _ptr(expert_offsets), _ptr(perm_slot), _ptr(inv_perm), _ptr(x_perm),
+                           ws.data_ptr(), ws.numel(), _stream(stream)), "moe_permute")
+
+
+def moe_expert_ffn(layer: Layer, x, x_perm, expert_offsets, perm_slot, topk_w, shared_gamma,
+                   w_gate_up, w_down, ws_gate_up, ws_down, y_routed, y_shared, ws, stream=None):
+    L = layer
+    _expect(x, "x", (L.T, L.H), L.dtype)
+    _expect(x_perm, "x_perm", (L.T * L.k, L.H), L.dtype)
+    _expect(expert_offsets, "expert_offsets", (L.E + 1,), torch.int32)
+    _expect(perm_slot, "perm_slot", (L.T * L.k,), torch.int32)
+    if topk_w.numel() != L.T * L.k or topk_w.dtype != torch.float32 or not topk_w.is_contiguous():
+        raise ValueError("topk_w must be a contiguous fp32 tensor of T*k entries")
+    if L.S > 0 and (shared_gamma is None or shared_gamma.numel() != L.T * L.S):
+        raise ValueError("shared_gamma must hold T*S entries")
+    _expect(w_gate_up, "w_gate_up", (L.E, 2 * L.I, L.H), L.dtype)
+    _expect(w_down, "w_down", (L.E, L.H, L.I), L.dtype)
+    _expect(ws_gate_up, "ws_gate_up", (L.S, 2 * L.I, L.H), L.dtype, allow_none=L.S == 0)
+    _expect(ws_down, "ws_down", (L.S, L.H, L.I), L.dtype, allow_none=L.S == 0)
+    _expect(y_routed, "y_routed", (L.T * L.k, L.H), torch.float32)
+    _expect(y_shared, "y_shared", (L.S * L.T, L.H), torch.float32, allow_none=L.S == 0)
+    _check(LIB.moe_expert_ffn(ctypes.byref(L.desc()), _ptr(x), _ptr(x_perm), _ptr(expert_offsets),
+                              _ptr(perm_slot), _ptr(topk_w), _ptr(shared_gamma), _ptr(w_gate_up),
+                              _ptr(w_down), _ptr(ws_gate_up), _ptr(ws_down), _ptr(y_routed),
+                              _ptr(y_shared), ws.data_ptr(), ws.numel(), _stream(stream)),
+           "moe_expert_ffn")
+
+
+def moe_combine(layer: Layer, y_routed, y_shared, inv_perm, out, ws, stream=None):
+    L = layer
+    _expect(y_routed, "y_routed", (L.T * L.k, L.H), torch.float32)
+    _expect(y_shared, "y_shared", (L.S * L.T, L.H), torch.float32, allow_none=L.S == 0)
+    _expect(inv_perm, "inv_perm", (L.T * L.k,), torch.int32)
+    _expect(out, "out", (L.T, L.H), L.dtype)
+    _check(LIB.moe_combine(ctypes.byref(L.desc()), _ptr(y_routed), _ptr(y_shared), _ptr(inv_perm),
+                           _ptr(out), ws.data_ptr(), ws.numel(), _stream(stream)), "moe_combine")
+
+
+def moe_forward(layer: Layer, x, w_router, corr_bias, w_gate_up, w_down, ws_gate_up, ws_down,
+                out, ws, padding_mask=None, topk_w=None, topk_idx=None, shared_gamma=None,
+                stream=None):
+    L = layer
+    _expect(x, "x", (L.T, L.H), L.dtype)
+    _expect(w_router, "w_router", (L.E + L.S, L.H), torch.float32)
+    _expect(corr_bias, "corr_bias", (L.E,), torch.float32)
+    _expect(w_gate_up, "w_gate_up", (L.E, 2 * L.I, L.H), L.dtype)
+    _expect(w_down, "w_down", (L.E, L.H, L.I), L.dtype)
+    _expect(ws_gate_up, "ws_gate_up", (L.S, 2 * L.I, L.H), L.dtype, allow_none=L.S == 0)
+    _expect(ws_down, "ws_down", (L.S, L.H, L.I), L.dtype, allow_none=L.S == 0)
+    _expect(out, "out", (L.T, L.H), L.dtype)
+    _expect(padding_mask, "padding_mask", (L.T,), torch.uint8, allow_none=True)
+    _expect(topk_w, "topk_w", (L.T, L.k), torch.float32, allow_none=True)
+    _expect(topk_idx, "topk_idx", (L.T, L.k), torch.int32, allow_none=True)
+    _expect(shared_gamma, "shared_gamma", (L.T, L.S), torch.float32, allow_none=True)
+    _check(LIB.moe_forward(ctypes.byref(L.desc()), _ptr(x), _ptr(w_router), _ptr(corr_bias),
+                           _ptr(w_gate_up), _ptr(w_down), _ptr(ws_gate_up), _ptr(ws_down),
+                           _ptr(padding_mask), _ptr(out), _ptr(topk_w), _ptr(topk_idx),
+                           _ptr(shared_gamma), ws.data_ptr(), ws.numel(), _stream(stream)),
+           "moe_forward")
+
+
+def forward_kernel_count(layer: Layer) -> int:
+    return int(LIB.moe_forward_kernel_count(ctypes.byref(layer.desc())))
+
+
+class InklingMoE:
+    """Device-resident weights of one layer plus its workspace; ``__call__``
+    runs ``moe_forward`` on ``x`` of shape ``[..., H]`` (leading dims are
+    flattened to tokens, as ``InklingMoE.forward`` does)."""
+
+    def __init__(self, weights: dict, E: int, k: int, S: int, route_scale: float,
+                 global_scale: float = 1.0, device="cuda"):
+        self.w = {n: t.to(device).contiguous() for n, t in weights.items() if n != "x"}
+        self.E, self.k, self.S = E, k, S
+        self.H = self.w["w_router"].shape[1]
+        self.I = self.w["w_down"].shape[2]
+        self.dtype = self.w["w_gate_up"].dtype
+        self.route_scale, self.global_scale = route_scale, global_scale
+        self.device = device
+        self._ws = None
+        self._ws_T = -1
+
+    def layer(self, T: int) -> Layer:
+        return Layer(T, self.H, self.E, self.k, self.S, self.I, self.dtype, self.route_scale,
+                     self.global_scale)
+
+    def __call__(self, x: torch.Tensor, padding_mask: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+        lead = x.shape[:-1]
+        xt = x.reshape(-1, self.H).contiguous()
+        L = self.layer(xt.shape[0])
+        if self._ws is None or self._ws_T < L.T:
+            self._ws = new_workspace(L, device=self.device, stream=stream)
+            self._ws_T = L.T
+        out = torch.empty_like(xt)
+        pm = None
+        if padding_mask is not None:
+            pm = padding_mask.reshape(-1).to(device=xt.device, dtype=torch.uint8).contiguous()
+        w = self.w
+        moe_forward(L, xt, w["w_router"], w["corr_bias"], w["w_gate_up"], w["w_down"],
+                    w.get("ws_gate_up") if self.S else None, w.get("ws_down") if self.S else None,
+                    out, self._ws, padding_mask=pm, stream=stream)
+        return out.reshape(*lead, self.H)

@@ -1,0 +1,100 @@
+// Recombination of shared and routed expert outputs (Inkling layers page,
+// InklingMoE.forward):
+//   out[t] = sum_s y_shared[s*T + t] + sum_j y_routed[inv_perm[t*k + j]]
+// in fp32, in that fixed order (shared s ascending, then choices j
+// ascending), rounded once to the output dtype.  The rows are fp32.  The routing weights are
+// already folded into the rows (inkling_swiglu scales the activated output),
+// so the sum is unweighted.  One block per token; 16-byte vector loads and
+// stores along the hidden dim, coalesced across the block.  HBM-bound.
+#include <algorithm>
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+// acc[0..V) += 4*V/4 consecutive fp32 values (V = 8 or 4)
+template <int V>
+__device__ __forceinline__ void add_vec(float (&acc)[V], const float* p) {
+#pragma unroll
+  for (int i = 0; i < V / 4; ++i) {
+    const float4 q = __ldcs(reinterpret_cast<const float4*>(p) + i);
+    acc[4 * i + 0] += q.x;
+    acc[4 * i + 1] += q.y;
+    acc[4 * i + 2] += q.z;
+    acc[4 * i + 3] += q.w;
+  }
+}
+
+__device__ __forceinline__ void store_vec(__nv_bfloat16* p, const float (&acc)[8]) {
+  uint4 q;
+  q.x = pack_bf16x2(acc[0], acc[1]);
+  q.y = pack_bf16x2(acc[2], acc[3]);
+  q.z = pack_bf16x2(acc[4], acc[5]);
+  q.w = pack_bf16x2(acc[6], acc[7]);
+  *reinterpret_cast<uint4*>(p) = q;
+}
+
+__device__ __forceinline__ void store_vec(float* p, const float (&acc)[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+}
+
+template <typename TY>
+__global__ void __launch_bounds__(256)
+    combine_kernel(const float* __restrict__ y_routed, const float* __restrict__ y_shared,
+                   const int32_t* __restrict__ inv_perm, TY* __restrict__ out, int64_t T, int H,
+                   int k, int S, int64_t rows_cap, int32_t* status) {
+  constexpr int V = 16 / sizeof(TY);   // one 16-byte output store per vector
+  __shared__ int s_rows[32];
+  const int nv = H / V;
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    if (threadIdx.x < k) {
+      int r = inv_perm[t * k + threadIdx.x];
+      if (r >= rows_cap) {
+        record_status(status, DEV_BAD_ROW);
+        r = -1;
+      }
+      s_rows[threadIdx.x] = r;
+    }
+    __syncthreads();
+    for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+      float acc[V];
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc[i] = 0.0f;
+      for (int s = 0; s < S; ++s)
+        add_vec(acc, y_shared + (static_cast<int64_t>(s) * T + t) * H + static_cast<int64_t>(v) * V);
+      for (int j = 0; j < k; ++j) {
+        const int r = s_rows[j];
+        if (r >= 0) add_vec(acc, y_routed + static_cast<int64_t>(r) * H + static_cast<int64_t>(v) * V);
+      }
+      store_vec(out + t * H + static_cast<int64_t>(v) * V, acc);
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const Layer& L, const void* y_routed, const void* y_shared,
+                           const int32_t* inv_perm, void* out, int32_t* status, int num_sms,
+                           cudaStream_t stream) {
+  const unsigned grid =
+      static_cast<unsigned>(std::min<int64_t>(L.T, static_cast<int64_t>(num_sms) * 8));
+  const int64_t cap = L.T * L.k;
+  if (L.dtype == MOE_BF16)
+    combine_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+        static_cast<const float*>(y_routed), static_cast<const float*>(y_shared), inv_perm,
+        static_cast<__nv_bfloat16*>(out), L.T, L.H, L.k, L.S, cap, status);
+  else
+    combine_kernel<float><<<grid, 256, 0, stream>>>(
+        static_cast<const float*>(y_routed), static_cast<const float*>(y_shared), inv_perm,
+        static_cast<float*>(out), L.T, L.H, L.k, L.S, cap, status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

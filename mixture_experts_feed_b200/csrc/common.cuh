@@ -1,0 +1,49 @@
+// Shared device helpers of the Inkling MoE kernels: status word, bounded
+// waits, bf16 packing.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "inkling_moe.h"
+
+namespace moe {
+
+// Device status word codes (first int32 of the workspace).  Sticky: the first
+// kernel to record a problem wins.
+enum DeviceCode : int32_t {
+  DEV_OK = 0,
+  DEV_BAD_EXPERT_ID = 0x101,   // topk_idx outside [0, E)
+  DEV_BAD_ROW = 0x102,         // inv_perm / perm_slot outside its range
+  DEV_WAIT_TIMEOUT = 0x201,    // a pipeline wait ran past its time limit
+};
+
+// Bounded waits give up after this many nanoseconds of %globaltimer.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
+
+__device__ __forceinline__ void record_status(int32_t* status, int32_t code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+template <typename T> struct Vec16;   // 16-byte vector of T
+template <> struct Vec16<float> { static constexpr int N = 4; };
+template <> struct Vec16<__nv_bfloat16> { static constexpr int N = 8; };
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace moe

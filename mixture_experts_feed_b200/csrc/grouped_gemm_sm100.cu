@@ -1,0 +1,402 @@
+// Grouped expert GEMMs on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// One persistent kernel computes, for every group of rows (a routed expert or
+// a shared expert, see grouping.cuh), D = A_rows @ W_g^T with bf16 operands
+// and an fp32 accumulator in tensor memory, then runs a fused epilogue:
+//   kGateUp: the accumulator columns interleave gate and up channels
+//            ([g0, u0, g1, u1, ...], the fused gate_up_proj layout of the
+//            Inkling layers page, inkling_swiglu); the epilogue writes
+//            h = w * silu(g) * u in bf16, w the row's routing weight (routed
+//            rows: topk_w of the row's slot; shared rows: the token's gamma).
+//   kDown:   the epilogue writes D in fp32 (the down projection); the rows
+//            stay fp32 until the recombination rounds the layer output once
+//            (rounding them to bf16 as well would put a correct pipeline at
+//            about 2% of the output RMS, the edge of the 2e-2 bound).
+//
+// Roles (192 threads, one CTA per SM):
+//   warp 0      TMA producer: A tile [128 rows x 64 K] and B tile
+//               [256 rows x 64 K] per stage, 128-byte swizzle, 4 stages.
+//   warp 1      TMEM allocator and MMA issuer (one thread): 4 x
+//               tcgen05.mma M128 N256 K16 per stage into one of two
+//               accumulators (2 x 256 TMEM columns).
+//   warps 2..5  epilogue: tcgen05.ld the accumulator rows (warp w reads TMEM
+//               lanes 32*(w%4) .. +31), fused math, 16-byte global stores.
+// The two accumulators let the epilogue of tile i overlap the MMAs of i+1.
+// All waits are bounded (sm100_ptx.cuh); on a timeout every role stops,
+// the status word records it and TMEM is released.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "grouping.cuh"
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+namespace sm100 {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;   // two 256-column fp32 accumulators
+constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+
+enum Mode { kGateUp = 0, kDown = 1 };
+
+struct alignas(64) GemmParams {
+  CUtensorMap tmA[2];   // A operand of routed (0) and shared (1) groups: 2-D [rows, K]
+  CUtensorMap tmB[2];   // weights of routed (0) and shared (1) groups: 3-D [G][N][K]
+  const int32_t* offsets;     // [E+1]
+  const int32_t* perm_slot;   // [rows] slot of each permuted row (kGateUp weights)
+  const float* topk_w;        // [T*k]
+  const float* gamma;         // [T*S]
+  void* out[2];               // output of routed (0) and shared (1) groups
+  int32_t* status;
+  int64_t T;
+  int64_t a1_base, a1_stride; // shared group s reads A rows from a1_base + s*a1_stride
+  int E, S, K, N;
+  int ld_out;                 // output row length in elements
+  int rows_cap;               // rows of the routed A operand (bound of offsets)
+};
+
+struct SmemLayout {
+  static constexpr int kA = 0;
+  static constexpr int kB = STAGES * A_BYTES;
+  static constexpr int kBars = kB + STAGES * B_BYTES;
+  // full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
+  static constexpr int kNumBars = 2 * STAGES + 5;
+  static constexpr int kMisc = kBars + kNumBars * 8;   // tmem base, abort, bad
+  static constexpr int kTables = kMisc + 16;
+};
+
+__host__ __device__ inline int smem_bytes(int E, int S) {
+  return 1024 /* alignment slack */ + SmemLayout::kTables + 4 * ((E + 1) + (E + S + 1));
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem + SmemLayout::kA;
+  uint8_t* sB = smem + SmemLayout::kB;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SmemLayout::kBars);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = bars + 2 * STAGES + 2;
+  uint64_t* drain = bars + 2 * STAGES + 4;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + SmemLayout::kMisc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SmemLayout::kMisc + 4);
+  int* s_bad = reinterpret_cast<int*>(smem + SmemLayout::kMisc + 8);
+  int* s_off = reinterpret_cast<int*>(smem + SmemLayout::kTables);
+  int* s_tile = s_off + (p.E + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = p.E + p.S;
+  const int n_tiles = (p.N + BN - 1) / BN;
+  const int k_blocks = p.K / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int i = 0; i < STAGES; ++i) {
+        mbar_init(&full[i], 1);
+        mbar_init(&empty[i], 1);
+      }
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&tfull[i], 1);
+        mbar_init(&tempty[i], 4);   // one arrive per epilogue warp
+      }
+      mbar_init(drain, 1);
+      *s_abort = 0;
+      *s_bad = 0;
+      fence_mbar_init();
+      fence_proxy_async_smem();
+      prefetch_tmap(&p.tmA[0]);
+      prefetch_tmap(&p.tmA[1]);
+      prefetch_tmap(&p.tmB[0]);
+      prefetch_tmap(&p.tmB[1]);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    tmem_alloc(s_tmem, TMEM_COLS);
+    tmem_relinquish();
+  } else if (warp == 2) {
+    build_tile_prefix(p.offsets, p.E, p.S, p.T, BM, n_tiles, p.rows_cap, s_off, s_tile, s_bad);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem_base = *s_tmem;
+  const int total_tiles = s_tile[G];
+  if (threadIdx.x == 0 && *s_bad) record_status(p.status, DEV_BAD_ROW);
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------ TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    int last_parity[STAGES];
+#pragma unroll
+    for (int i = 0; i < STAGES; ++i) last_parity[i] = -1;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      int g, m, n;
+      decode_tile(tile, s_tile, G, s_off, p.E, p.T, BM, g, m, n);
+      const GroupInfo gi = group_info(g, s_off, p.E, p.T, p.a1_base, p.a1_stride);
+      const void* tmA = &p.tmA[gi.src];
+      const void* tmB = &p.tmB[gi.src];
+      const int a_row = static_cast<int>(gi.a_row0) + m * BM;
+      bool ok = true;
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, s_abort, p.status)) { ok = false; break; }
+        mbar_arrive_expect_tx(&full[stage], A_BYTES + B_BYTES);
+        tma_load_2d(sA + stage * A_BYTES, tmA, &full[stage], kb * BK, a_row);
+        tma_load_3d(sB + stage * B_BYTES, tmB, &full[stage], kb * BK, n * BN, gi.b_idx);
+        last_parity[stage] = static_cast<int>(phase);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+    }
+    // Wait (bounded) until the last load issued on every stage has landed,
+    // so that no copy still writes shared memory when the block exits.
+    const uint64_t t0 = globaltimer_ns();
+    for (int i = 0; i < STAGES; ++i) {
+      if (last_parity[i] < 0) continue;
+      while (!mbar_try_wait(&full[i], static_cast<uint32_t>(last_parity[i]))) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) { record_status(p.status, DEV_WAIT_TIMEOUT); break; }
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t aphase = (it >> 1) & 1;
+      if (!mbar_wait(&tempty[acc], aphase ^ 1u, s_abort, p.status)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        if (!mbar_wait(&full[stage], phase, s_abort, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t adesc = smem_desc_kmajor_sw128(smem_u32(sA + stage * A_BYTES));
+        const uint64_t bdesc = smem_desc_kmajor_sw128(smem_u32(sB + stage * B_BYTES));
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          // +32 bytes per K=16 step inside the 128-byte swizzle atom
+          mma_bf16_ss(d_tmem, adesc + static_cast<uint64_t>(2 * kk),
+                      bdesc + static_cast<uint64_t>(2 * kk), IDESC, (kb | kk) != 0 ? 1u : 0u);
+        }
+        mma_commit(&empty[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      mma_commit(&tfull[acc]);
+    }
+    // Every MMA this thread issued must be complete before TMEM is freed.
+    mma_commit(drain);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(drain, 0)) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs) { record_status(p.status, DEV_WAIT_TIMEOUT); break; }
+    }
+  } else if (warp >= 2) {
+    // --------------------------------------------------------- epilogue
+    const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
+    const int row_in_tile = quarter * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+      int g, m, n;
+      decode_tile(tile, s_tile, G, s_off, p.E, p.T, BM, g, m, n);
+      const GroupInfo gi = group_info(g, s_off, p.E, p.T, p.a1_base, p.a1_stride);
+      const int acc = it & 1;
+      const uint32_t aphase = (it >> 1) & 1;
+      if (!mbar_wait(&tfull[acc], aphase, s_abort, p.status)) break;
+      tc_fence_after();
+
+      const int r = m * BM + row_in_tile;          // row inside the group
+      const bool valid = r < gi.rows;
+      const int64_t out_row = gi.out_row0 + r;
+      float w = 1.0f;
+      if (MODE == kGateUp && valid) {
+        if (gi.src == 0) {
+          const int slot = p.perm_slot[gi.a_row0 + r];
+          if (slot >= 0 && slot < p.rows_cap) {
+            w = p.topk_w[slot];
+          } else {
+            record_status(p.status, DEV_BAD_ROW);
+            w = 0.0f;
+          }
+        } else {
+          w = p.gamma[static_cast<int64_t>(r) * p.S + gi.s];
+        }
+      }
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int col0 = n * BN + c * 32;
+        if (col0 >= p.N) break;                    // warp-uniform
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * 32), v);
+        tmem_ld_wait();
+        if (!valid) continue;
+        if (MODE == kGateUp) {
+          uint32_t packed[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float g0 = __uint_as_float(v[4 * i + 0]);
+            const float u0 = __uint_as_float(v[4 * i + 1]);
+            const float g1 = __uint_as_float(v[4 * i + 2]);
+            const float u1 = __uint_as_float(v[4 * i + 3]);
+            const float h0 = w * (g0 / (1.0f + __expf(-g0))) * u0;
+            const float h1 = w * (g1 / (1.0f + __expf(-g1))) * u1;
+            packed[i] = pack_bf16x2(h0, h1);
+          }
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out[gi.src]);
+          uint4* dst = reinterpret_cast<uint4*>(out + out_row * p.ld_out + col0 / 2);
+          dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+        } else {
+          float* out = static_cast<float*>(p.out[gi.src]);
+          uint4* dst = reinterpret_cast<uint4*>(out + out_row * p.ld_out + col0);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------- host side
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2-D bf16 map over [rows, K] (K contiguous), box [BM rows, BK], 128B swizzle.
+static bool encode_a(CUtensorMap* m, const void* base, int64_t rows, int K) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  cuuint32_t box[2] = {BK, BM};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D bf16 map over [G][N][K] (K contiguous), box [1][BN][BK], 128B swizzle.
+static bool encode_b(CUtensorMap* m, const void* base, int G, int N, int K) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(G)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2,
+                           static_cast<cuuint64_t>(K) * 2 * static_cast<cuuint64_t>(N)};
+  cuuint32_t box[3] = {BK, BN, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+static cudaError_t launch_mode(const GemmParams& p, int sms, cudaStream_t stream) {
+  const int smem = smem_bytes(p.E, p.S);
+  static int configured_smem[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && configured_smem[dev] < smem) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured_smem[dev] = smem;
+  }
+  grouped_gemm_kernel<MODE><<<sms, NUM_THREADS, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace sm100
+
+int sm100_gemm_max_smem(int E, int S) { return sm100::smem_bytes(E, S); }
+
+// gate_up: A0 = x_perm [T*k, H], A1 = x [T, H]; out0 = h rows [0, T*k),
+// out1 = h rows T*k + s*T + t.  down: A0 = A1 = h [T*k + S*T, I];
+// out0 = y_routed, out1 = y_shared.
+cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_perm,
+                                   const int32_t* offsets, const int32_t* perm_slot,
+                                   const float* topk_w, const float* gamma, const void* w_gate_up,
+                                   const void* w_down, const void* ws_gate_up,
+                                   const void* ws_down, void* h, void* y_routed, void* y_shared,
+                                   int32_t* status, int num_sms, cudaStream_t stream,
+                                   bool* map_error) {
+  using namespace sm100;
+  *map_error = false;
+  const int64_t Rk = L.T * L.k;                 // routed row capacity
+  const int64_t Rh = Rk + static_cast<int64_t>(L.S) * L.T;
+  __nv_bfloat16* hb = static_cast<__nv_bfloat16*>(h);
+
+  // ---------------- gate_up: [rows, H] x [2I, H]^T -> SwiGLU -> h [rows, I]
+  GemmParams g{};
+  bool ok = encode_a(&g.tmA[0], x_perm, Rk, L.H) && encode_a(&g.tmA[1], x, L.T, L.H) &&
+            encode_b(&g.tmB[0], w_gate_up, L.E, 2 * L.I, L.H);
+  if (ok && L.S > 0) ok = encode_b(&g.tmB[1], ws_gate_up, L.S, 2 * L.I, L.H);
+  else g.tmB[1] = g.tmB[0];
+  if (!ok) { *map_error = true; return cudaErrorInvalidValue; }
+  g.offsets = offsets; g.perm_slot = perm_slot; g.topk_w = topk_w; g.gamma = gamma;
+  g.out[0] = hb;
+  g.out[1] = hb + Rk * L.I;
+  g.status = status;
+  g.T = L.T; g.a1_base = 0; g.a1_stride = 0;
+  g.E = L.E; g.S = L.S; g.K = L.H; g.N = 2 * L.I; g.ld_out = L.I;
+  g.rows_cap = static_cast<int>(Rk);
+  cudaError_t e = launch_mode<kGateUp>(g, num_sms, stream);
+  if (e != cudaSuccess) return e;
+
+  // ---------------- down: h [rows, I] x [H, I]^T -> y [rows, H]
+  GemmParams d{};
+  ok = encode_a(&d.tmA[0], h, Rh, L.I) && encode_b(&d.tmB[0], w_down, L.E, L.H, L.I);
+  d.tmA[1] = d.tmA[0];
+  if (ok && L.S > 0) ok = encode_b(&d.tmB[1], ws_down, L.S, L.H, L.I);
+  else d.tmB[1] = d.tmB[0];
+  if (!ok) { *map_error = true; return cudaErrorInvalidValue; }
+  d.offsets = offsets; d.perm_slot = perm_slot; d.topk_w = topk_w; d.gamma = gamma;
+  d.out[0] = y_routed;
+  d.out[1] = y_shared;
+  d.status = status;
+  d.T = L.T; d.a1_base = Rk; d.a1_stride = L.T;
+  d.E = L.E; d.S = L.S; d.K = L.I; d.N = L.H; d.ld_out = L.H;
+  d.rows_cap = static_cast<int>(Rk);
+  return launch_mode<kDown>(d, num_sms, stream);
+}
+
+}  // namespace moe

@@ -1,0 +1,114 @@
+// Group and tile bookkeeping of the grouped expert GEMMs.
+//
+// A launch covers G = E + S groups.  Group g < E is routed expert g: its rows
+// are the permuted rows [off[g], off[g+1]) of the routed A operand, its
+// weights are slice g of the routed weight tensor, its outputs go to the same
+// rows of output 0.  Group E + s is shared expert s: its rows are all T
+// tokens, read from A operand 1 starting at row a1_base + s * a1_stride,
+// weights are slice s of the shared weight tensor, outputs go to rows
+// s * T + t of output 1.
+//
+// Tiles are numbered group by group; inside a group, n-tile by n-tile, and
+// inside an n-tile, m-tile by m-tile (consecutive tiles share one weight
+// strip, so CTAs running together reuse it from L2).
+#pragma once
+
+#include <stdint.h>
+
+namespace moe {
+
+struct GroupInfo {
+  int src;           // 0 = routed operands, 1 = shared operands
+  int b_idx;         // weight slice inside its tensor
+  int s;             // shared expert index (src == 1)
+  int rows;          // rows in this group
+  int64_t a_row0;    // first A row of the group
+  int64_t out_row0;  // first output row of the group
+};
+
+__device__ __forceinline__ GroupInfo group_info(int g, const int* s_off, int E, int64_t T,
+                                                int64_t a1_base, int64_t a1_stride) {
+  GroupInfo gi;
+  if (g < E) {
+    gi.src = 0;
+    gi.b_idx = g;
+    gi.s = -1;
+    gi.a_row0 = s_off[g];
+    gi.rows = s_off[g + 1] - s_off[g];
+    gi.out_row0 = s_off[g];
+  } else {
+    const int s = g - E;
+    gi.src = 1;
+    gi.b_idx = s;
+    gi.s = s;
+    gi.a_row0 = a1_base + static_cast<int64_t>(s) * a1_stride;
+    gi.rows = static_cast<int>(T);
+    gi.out_row0 = static_cast<int64_t>(s) * T;
+  }
+  return gi;
+}
+
+// Warp 0 of the block fills s_off[0..E] from global memory and
+// s_tile[0..G] with the exclusive prefix of per-group tile counts.
+// Offsets outside [0, rows_cap] or decreasing are clamped to an empty group
+// and reported through `bad` (set to 1).
+__device__ inline void build_tile_prefix(const int32_t* __restrict__ offsets, int E, int S,
+                                         int64_t T, int BM, int n_tiles, int rows_cap, int* s_off,
+                                         int* s_tile, int* bad) {
+  const int lane = threadIdx.x & 31;
+  for (int i = lane; i <= E; i += 32) s_off[i] = offsets[i];
+  __syncwarp();
+  if (lane == 0) {
+    // clamp to a monotone sequence inside [0, rows_cap]
+    int prev = 0;
+    for (int i = 0; i <= E; ++i) {
+      int v = s_off[i];
+      if (v < prev || v > rows_cap || (i == 0 && v != 0)) {
+        *bad = 1;
+        v = v < prev ? prev : (v > rows_cap ? rows_cap : v);
+        if (i == 0) v = 0;
+      }
+      s_off[i] = v;
+      prev = v;
+    }
+  }
+  __syncwarp();
+  const int G = E + S;
+  int carry = 0;
+  if (lane == 0) s_tile[0] = 0;
+  for (int base = 0; base < G; base += 32) {
+    const int g = base + lane;
+    int cnt = 0;
+    if (g < G) {
+      const int rows = g < E ? (s_off[g + 1] - s_off[g]) : static_cast<int>(T);
+      cnt = ((rows + BM - 1) / BM) * n_tiles;
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += v;
+    }
+    if (g < G) s_tile[g + 1] = carry + incl;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  __syncwarp();
+}
+
+// Map a linear tile id to (group, m-tile, n-tile) using the prefix table.
+__device__ __forceinline__ void decode_tile(int tile, const int* s_tile, int G, const int* s_off,
+                                            int E, int64_t T, int BM, int& g, int& m, int& n) {
+  int lo = 0, hi = G - 1;   // find last g with s_tile[g] <= tile
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_tile[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  g = lo;
+  const int rows = g < E ? (s_off[g + 1] - s_off[g]) : static_cast<int>(T);
+  const int mt = (rows + BM - 1) / BM;
+  const int local = tile - s_tile[g];
+  n = local / mt;
+  m = local - n * mt;
+}
+
+}  // namespace moe

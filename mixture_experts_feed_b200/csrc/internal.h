@@ -1,0 +1,52 @@
+// Launch functions behind the C ABI (not exported).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+struct Layer {
+  int64_t T;
+  int H, E, k, S, I;
+  int dtype;   // MOE_F32 / MOE_BF16
+  float route_scale, global_scale;
+};
+
+// router.cu
+cudaError_t launch_router_logits(const Layer& L, const void* x, const float* w_router,
+                                 float* logits, cudaStream_t stream);
+cudaError_t launch_router_topk(const Layer& L, const float* logits, const float* corr_bias,
+                               float* topk_w, int32_t* topk_idx, float* shared_gamma,
+                               cudaStream_t stream);
+
+// permute.cu
+cudaError_t launch_permute(const Layer& L, const int32_t* topk_idx, const uint8_t* padding_mask,
+                           const void* x, int32_t* offsets, int32_t* perm_slot, int32_t* inv_perm,
+                           void* x_perm, int32_t* counts, int32_t* status, int num_sms,
+                           cudaStream_t stream);
+
+// grouped_gemm_sm100.cu (bf16, tcgen05)
+cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_perm,
+                                   const int32_t* offsets, const int32_t* perm_slot,
+                                   const float* topk_w, const float* gamma, const void* w_gate_up,
+                                   const void* w_down, const void* ws_gate_up,
+                                   const void* ws_down, void* h, void* y_routed, void* y_shared,
+                                   int32_t* status, int num_sms, cudaStream_t stream,
+                                   bool* map_error);
+int sm100_gemm_max_smem(int E, int S);
+
+// grouped_gemm_simt.cu (fp32, CUDA cores)
+cudaError_t launch_expert_ffn_f32(const Layer& L, const void* x, const void* x_perm,
+                                  const int32_t* offsets, const int32_t* perm_slot,
+                                  const float* topk_w, const float* gamma, const void* w_gate_up,
+                                  const void* w_down, const void* ws_gate_up, const void* ws_down,
+                                  void* h, void* y_routed, void* y_shared, int32_t* status,
+                                  int num_sms, cudaStream_t stream);
+
+// combine.cu
+cudaError_t launch_combine(const Layer& L, const void* y_routed, const void* y_shared,
+                           const int32_t* inv_perm, void* out, int32_t* status, int num_sms,
+                           cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,311 @@
+// The C ABI of libinklingmoe.so (declared in include/inkling_moe.h): argument
+// checks, workspace layout and the order of launches.  Every step of the
+// layer runs in this library's kernels; there is no host compute path.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "inkling_moe.h"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kVersion = 1;
+constexpr size_t kStatusBytes = 256;
+constexpr size_t kRegionAlign = 1024;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct WsLayout {
+  size_t status, logits, counts, topk_w, topk_idx, gamma, offsets, perm_slot, inv_perm, x_perm,
+      h, y_routed, y_shared, total;
+};
+
+WsLayout ws_layout(const Layer& L) {
+  WsLayout w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes > 0 ? bytes : 1, kRegionAlign);
+    return o;
+  };
+  const size_t elt = L.dtype == MOE_BF16 ? 2 : 4;
+  const size_t T = static_cast<size_t>(L.T);
+  const size_t Rk = T * L.k;
+  const size_t Rh = Rk + T * L.S;
+  w.status = take(kStatusBytes);
+  w.logits = take(T * (L.E + L.S) * 4);
+  w.counts = take(static_cast<size_t>(L.E) * 4);
+  w.topk_w = take(Rk * 4);
+  w.topk_idx = take(Rk * 4);
+  w.gamma = take(T * L.S * 4);
+  w.offsets = take((static_cast<size_t>(L.E) + 1) * 4);
+  w.perm_slot = take(Rk * 4);
+  w.inv_perm = take(Rk * 4);
+  w.x_perm = take(Rk * L.H * elt);
+  w.h = take(Rh * L.I * elt);
+  w.y_routed = take(Rk * L.H * 4);   // expert output rows stay fp32
+  w.y_shared = take(T * L.S * L.H * 4);
+  w.total = off;
+  return w;
+}
+
+moe_status_t check_desc(const moe_layer_desc_t* d, Layer* L) {
+  if (d == nullptr) return MOE_ERR_INVALID_ARG;
+  if (d->num_tokens < 0 || d->hidden <= 0 || d->n_routed <= 0 || d->top_k <= 0 ||
+      d->n_shared < 0 || d->intermediate <= 0)
+    return MOE_ERR_INVALID_ARG;
+  if (d->top_k > d->n_routed) return MOE_ERR_INVALID_ARG;
+  if (d->dtype != MOE_F32 && d->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (!isfinite(d->route_scale) || !isfinite(d->global_scale)) return MOE_ERR_INVALID_ARG;
+  if (d->top_k > 16 || d->n_routed > 1024 || d->n_shared > 8) return MOE_ERR_UNSUPPORTED;
+  if (d->hidden % 64 != 0 || d->intermediate % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  const int64_t rows = d->num_tokens * (static_cast<int64_t>(d->top_k) + d->n_shared);
+  if (d->num_tokens > (int64_t{1} << 31) / 32 || rows >= (int64_t{1} << 31))
+    return MOE_ERR_UNSUPPORTED;
+  L->T = d->num_tokens;
+  L->H = d->hidden;
+  L->E = d->n_routed;
+  L->k = d->top_k;
+  L->S = d->n_shared;
+  L->I = d->intermediate;
+  L->dtype = d->dtype;
+  L->route_scale = d->route_scale;
+  L->global_scale = d->global_scale;
+  return MOE_OK;
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+moe_status_t check_ws(const Layer& L, const void* ws, size_t bytes) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255) != 0) return MOE_ERR_INVALID_ARG;
+  if (bytes < ws_layout(L).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+template <typename P>
+P* region(void* ws, size_t off) {
+  return reinterpret_cast<P*>(static_cast<uint8_t*>(ws) + off);
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                        \
+  do {                                       \
+    const moe_status_t _s = (expr);          \
+    if (_s != MOE_OK) return _s;             \
+  } while (0)
+
+moe_status_t route_impl(const Layer& L, const void* x, const float* w_router,
+                        const float* corr_bias, float* topk_w, int32_t* topk_idx,
+                        float* shared_gamma, void* ws, cudaStream_t stream) {
+  const WsLayout w = ws_layout(L);
+  float* logits = region<float>(ws, w.logits);
+  MOE_TRY(cuda_status(launch_router_logits(L, x, w_router, logits, stream)));
+  return cuda_status(launch_router_topk(L, logits, corr_bias, topk_w, topk_idx, shared_gamma, stream));
+}
+
+moe_status_t permute_impl(const Layer& L, const int32_t* topk_idx, const uint8_t* pad,
+                          const void* x, int32_t* offsets, int32_t* perm_slot, int32_t* inv_perm,
+                          void* x_perm, void* ws, cudaStream_t stream) {
+  const WsLayout w = ws_layout(L);
+  return cuda_status(launch_permute(L, topk_idx, pad, x, offsets, perm_slot, inv_perm, x_perm,
+                                    region<int32_t>(ws, w.counts), region<int32_t>(ws, w.status),
+                                    num_sms(), stream));
+}
+
+moe_status_t ffn_impl(const Layer& L, const void* x, const void* x_perm, const int32_t* offsets,
+                      const int32_t* perm_slot, const float* topk_w, const float* gamma,
+                      const void* wgu, const void* wd, const void* wsgu, const void* wsd,
+                      void* y_routed, void* y_shared, void* ws, cudaStream_t stream) {
+  const WsLayout w = ws_layout(L);
+  void* h = region<void>(ws, w.h);
+  int32_t* status = region<int32_t>(ws, w.status);
+  if (L.dtype == MOE_BF16) {
+    bool map_error = false;
+    const cudaError_t e = launch_expert_ffn_bf16(L, x, x_perm, offsets, perm_slot, topk_w, gamma,
+                                                 wgu, wd, wsgu, wsd, h, y_routed, y_shared,
+                                                 status, num_sms(), stream, &map_error);
+    if (map_error) return MOE_ERR_INVALID_ARG;
+    return cuda_status(e);
+  }
+  return cuda_status(launch_expert_ffn_f32(L, x, x_perm, offsets, perm_slot, topk_w, gamma, wgu,
+                                           wd, wsgu, wsd, h, y_routed, y_shared, status,
+                                           num_sms(), stream));
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status_t moe_workspace_size(const moe_layer_desc_t* desc, size_t* bytes) {
+  Layer L;
+  MOE_TRY(check_desc(desc, &L));
+  if (bytes == nullptr) return MOE_ERR_INVALID_ARG;
+  *bytes = ws_layout(L).total;
+  return MOE_OK;
+}
+
+moe_status_t moe_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+  if (workspace == nullptr || workspace_bytes < kStatusBytes) return MOE_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(workspace, 0, kStatusBytes, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_read_device_status(void* workspace, void* stream, int32_t* device_code) {
+  if (workspace == nullptr) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t code = 0;
+  MOE_TRY(cuda_status(cudaMemcpyAsync(&code, workspace, sizeof(code), cudaMemcpyDeviceToHost, s)));
+  MOE_TRY(cuda_status(cudaStreamSynchronize(s)));
+  MOE_TRY(cuda_status(cudaMemsetAsync(workspace, 0, sizeof(code), s)));
+  if (device_code != nullptr) *device_code = code;
+  if (code == 0) return MOE_OK;
+  return code == DEV_WAIT_TIMEOUT ? MOE_ERR_TIMEOUT : MOE_ERR_DEVICE_CHECK;
+}
+
+moe_status_t moe_route(const moe_layer_desc_t* desc, const void* x, const float* w_router,
+                       const float* corr_bias, float* topk_w, int32_t* topk_idx,
+                       float* shared_gamma, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  Layer L;
+  MOE_TRY(check_desc(desc, &L));
+  if (!aligned16(x) || !aligned16(w_router) || corr_bias == nullptr || topk_w == nullptr ||
+      topk_idx == nullptr || (L.S > 0 && shared_gamma == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(L, workspace, workspace_bytes));
+  if (L.T == 0) return MOE_OK;
+  return route_impl(L, x, w_router, corr_bias, topk_w, topk_idx, shared_gamma, workspace,
+                    static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_permute(const moe_layer_desc_t* desc, const int32_t* topk_idx,
+                         const uint8_t* padding_mask, const void* x, int32_t* expert_offsets,
+                         int32_t* perm_slot, int32_t* inv_perm, void* x_perm, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  Layer L;
+  MOE_TRY(check_desc(desc, &L));
+  if (topk_idx == nullptr || !aligned16(x) || expert_offsets == nullptr || perm_slot == nullptr ||
+      inv_perm == nullptr || !aligned16(x_perm))
+    return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(L, workspace, workspace_bytes));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (L.T == 0) {
+    return cuda_status(cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (L.E + 1), s));
+  }
+  return permute_impl(L, topk_idx, padding_mask, x, expert_offsets, perm_slot, inv_perm, x_perm,
+                      workspace, s);
+}
+
+moe_status_t moe_expert_ffn(const moe_layer_desc_t* desc, const void* x, const void* x_perm,
+                            const int32_t* expert_offsets, const int32_t* perm_slot,
+                            const float* topk_w, const float* shared_gamma,
+                            const void* w_gate_up, const void* w_down, const void* ws_gate_up,
+                            const void* ws_down, void* y_routed, void* y_shared,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  Layer L;
+  MOE_TRY(check_desc(desc, &L));
+  if (!aligned16(x) || !aligned16(x_perm) || expert_offsets == nullptr || perm_slot == nullptr ||
+      topk_w == nullptr || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(y_routed))
+    return MOE_ERR_INVALID_ARG;
+  if (L.S > 0 && (shared_gamma == nullptr || !aligned16(ws_gate_up) || !aligned16(ws_down) ||
+                  !aligned16(y_shared)))
+    return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(L, workspace, workspace_bytes));
+  if (L.T == 0) return MOE_OK;
+  return ffn_impl(L, x, x_perm, expert_offsets, perm_slot, topk_w, shared_gamma, w_gate_up, w_down,
+                  ws_gate_up, ws_down, y_routed, y_shared, workspace,
+                  static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_combine(const moe_layer_desc_t* desc, const void* y_routed, const void* y_shared,
+                         const int32_t* inv_perm, void* out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  Layer L;
+  MOE_TRY(check_desc(desc, &L));
+  if (!aligned16(y_routed) || inv_perm == nullptr || !aligned16(out) ||
+      (L.S > 0 && !aligned16(y_shared)))
+    return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(L, workspace, workspace_bytes));
+  if (L.T == 0) return MOE_OK;
+  const WsLayout w = ws_layout(L);
+  return cuda_status(launch_combine(L, y_routed, y_shared, inv_perm, out,
+                                    region<int32_t>(workspace, w.status), num_sms(),
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_forward(const moe_layer_desc_t* desc, const void* x, const float* w_router,
+                         const float* corr_bias, const void* w_gate_up, const void* w_down,
+                         const void* ws_gate_up, const void* ws_down, const uint8_t* padding_mask,
+                         void* out, float* topk_w, int32_t* topk_idx, float* shared_gamma,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  Layer L;
+  MOE_TRY(check_desc(desc, &L));
+  if (!aligned16(x) || !aligned16(w_router) || corr_bias == nullptr || !aligned16(w_gate_up) ||
+      !aligned16(w_down) || !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
+  if (L.S > 0 && (!aligned16(ws_gate_up) || !aligned16(ws_down))) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(L, workspace, workspace_bytes));
+  if (L.T == 0) return MOE_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const WsLayout w = ws_layout(L);
+  float* tw = topk_w ? topk_w : region<float>(workspace, w.topk_w);
+  int32_t* ti = topk_idx ? topk_idx : region<int32_t>(workspace, w.topk_idx);
+  float* sg = shared_gamma ? shared_gamma : region<float>(workspace, w.gamma);
+  int32_t* offsets = region<int32_t>(workspace, w.offsets);
+  int32_t* perm_slot = region<int32_t>(workspace, w.perm_slot);
+  int32_t* inv_perm = region<int32_t>(workspace, w.inv_perm);
+  void* x_perm = region<void>(workspace, w.x_perm);
+  void* y_routed = region<void>(workspace, w.y_routed);
+  void* y_shared = region<void>(workspace, w.y_shared);
+  MOE_TRY(route_impl(L, x, w_router, corr_bias, tw, ti, sg, workspace, s));
+  MOE_TRY(permute_impl(L, ti, padding_mask, x, offsets, perm_slot, inv_perm, x_perm, workspace, s));
+  MOE_TRY(ffn_impl(L, x, x_perm, offsets, perm_slot, tw, sg, w_gate_up, w_down, ws_gate_up,
+                   ws_down, y_routed, y_shared, workspace, s));
+  return cuda_status(launch_combine(L, y_routed, y_shared, inv_perm, out,
+                                    region<int32_t>(workspace, w.status), num_sms(), s));
+}
+
+int32_t moe_forward_kernel_count(const moe_layer_desc_t* desc) {
+  Layer L;
+  if (check_desc(desc, &L) != MOE_OK || L.T == 0) return 0;
+  // router: logits + top-k; permute: count, scan, compact, gather;
+  // experts: gate_up + down; combine.
+  return 2 + 4 + 2 + 1;
+}
+
+const char* moe_status_string(moe_status_t status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported layer shape";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_CHECK: return "device-side index check failed";
+    case MOE_ERR_TIMEOUT: return "device pipeline wait timed out";
+  }
+  return "unknown status";
+}
+
+int32_t moe_version(void) { return kVersion; }
+
+}  // extern "C"

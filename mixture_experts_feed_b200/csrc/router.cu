@@ -1,0 +1,214 @@
+// InklingGate on the GPU (Inkling layers page, InklingGate docstring and
+// InklingCorrectionBias.forward).
+//
+// Two kernels:
+//   router_logits_kernel  z[t, e] = sum_h x[t, h] * Wr[e, h] in fp32 (the
+//                         gate runs in fp32: gate_precision=torch.float32),
+//                         for all E routed + S shared rows of the gate bank.
+//                         Tiled SIMT fp32 GEMM (64 tokens x 64 rows x 32 K).
+//   router_topk_kernel    one warp per token: selection score
+//                         sigmoid(z) + bias over the routed rows, k rounds of
+//                         a warp-shuffle argmax (ties to the lower expert id),
+//                         then the weights.  The softmax over
+//                         log-sigmoid(z) of [selected ++ shared] equals
+//                         sigmoid(z_i) / sum sigmoid(z), which is what the
+//                         kernel evaluates, times route_scale*global_scale.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int RL_BM = 64, RL_BN = 64, RL_BK = 32, RL_THREADS = 256;
+
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 q = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
+template <typename TX>
+__global__ void __launch_bounds__(RL_THREADS)
+    router_logits_kernel(const TX* __restrict__ x, const float* __restrict__ w,
+                         float* __restrict__ z, int64_t T, int H, int NE) {
+  __shared__ __align__(16) float As[RL_BK][RL_BM + 4];
+  __shared__ __align__(16) float Bs[RL_BK][RL_BN + 4];
+  const int tid = threadIdx.x;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * RL_BM;
+  const int n0 = blockIdx.y * RL_BN;
+  const int tx = tid & 15, ty = tid >> 4;
+  const int lr = tid >> 2, lk = (tid & 3) * 8;
+  const int64_t arow = m0 + lr;
+  const int brow = n0 + lr;
+  const bool a_ok = arow < T, b_ok = brow < NE;
+  const TX* ap = x + (a_ok ? arow : 0) * H + lk;
+  const float* bp = w + static_cast<int64_t>(b_ok ? brow : 0) * H + lk;
+
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+
+  for (int k0 = 0; k0 < H; k0 += RL_BK) {
+    float av[8], bv[8];
+    if (a_ok) load8(ap + k0, av); else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) av[i] = 0.0f;
+    }
+    if (b_ok) load8(bp + k0, bv); else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) bv[i] = 0.0f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      As[lk + i][lr] = av[i];
+      Bs[lk + i][lr] = bv[i];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < RL_BK; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
+      const float ar[4] = {a.x, a.y, a.z, a.w};
+      const float br[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(ar[i], br[j], acc[i][j]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t row = m0 + ty * 4 + i;
+    if (row >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int col = n0 + tx * 4 + j;
+      if (col < NE) z[row * NE + col] = acc[i][j];
+    }
+  }
+}
+
+__device__ __forceinline__ float sigmoidf_(float v) { return 1.0f / (1.0f + expf(-v)); }
+
+constexpr int TK_WARPS = 8;
+
+// PL: routed scores held per lane (E <= 32 * PL).
+template <int PL>
+__global__ void __launch_bounds__(TK_WARPS * 32)
+    router_topk_kernel(const float* __restrict__ z, const float* __restrict__ bias, int64_t T,
+                       int E, int k, int S, float scale, float* __restrict__ topk_w,
+                       int32_t* __restrict__ topk_idx, float* __restrict__ gamma) {
+  __shared__ int s_chosen[TK_WARPS][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * TK_WARPS + warp;
+  if (t >= T) return;
+  const int NE = E + S;
+  const float* zt = z + t * NE;
+
+  float sel[PL];
+#pragma unroll
+  for (int i = 0; i < PL; ++i) {
+    const int e = lane + 32 * i;
+    const float v = e < E ? sigmoidf_(zt[e]) + bias[e] : -INFINITY;
+    sel[i] = isnan(v) ? -INFINITY : v;   // a NaN score ranks last, never breaks the argmax
+  }
+  uint32_t taken = 0;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < PL; ++i) {
+      const int e = lane + 32 * i;
+      const bool avail = e < E && !((taken >> i) & 1u);
+      // strict '>' keeps the lowest id among this lane's equal scores
+      if (avail && (bi == 0x7fffffff || sel[i] > bv)) {
+        bv = sel[i];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, d);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, d);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    bi = __shfl_sync(0xffffffffu, bi, 0);
+    if (bi >= E) bi = 0;   // unreachable for k <= E; keeps every index in range
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == 0) s_chosen[warp][j] = bi;
+  }
+  __syncwarp();
+  float sg = 0.0f;
+  if (lane < k) sg = sigmoidf_(zt[s_chosen[warp][lane]]);
+  else if (lane < k + S) sg = sigmoidf_(zt[E + (lane - k)]);
+  float sum = sg;
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
+  const float wv = sg / sum * scale;
+  if (lane < k) {
+    topk_w[t * k + lane] = wv;
+    topk_idx[t * k + lane] = s_chosen[warp][lane];
+  } else if (lane < k + S) {
+    gamma[t * S + (lane - k)] = wv;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_router_logits(const Layer& L, const void* x, const float* w_router,
+                                 float* logits, cudaStream_t stream) {
+  const int NE = L.E + L.S;
+  dim3 grid(static_cast<unsigned>(ceil_div(L.T, RL_BM)), static_cast<unsigned>(ceil_div(NE, RL_BN)));
+  if (L.dtype == MOE_BF16)
+    router_logits_kernel<__nv_bfloat16><<<grid, RL_THREADS, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(x), w_router, logits, L.T, L.H, NE);
+  else
+    router_logits_kernel<float><<<grid, RL_THREADS, 0, stream>>>(static_cast<const float*>(x),
+                                                                 w_router, logits, L.T, L.H, NE);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_topk(const Layer& L, const float* logits, const float* corr_bias,
+                               float* topk_w, int32_t* topk_idx, float* shared_gamma,
+                               cudaStream_t stream) {
+  const unsigned grid = static_cast<unsigned>(ceil_div(L.T, TK_WARPS));
+  const float scale = L.route_scale * L.global_scale;
+  const int pl = static_cast<int>(ceil_div(L.E, 32));
+#define MOE_TOPK(PLV)                                                                         \
+  router_topk_kernel<PLV><<<grid, TK_WARPS * 32, 0, stream>>>(logits, corr_bias, L.T, L.E, L.k, \
+                                                              L.S, scale, topk_w, topk_idx,     \
+                                                              shared_gamma)
+  if (pl <= 1) MOE_TOPK(1);
+  else if (pl <= 2) MOE_TOPK(2);
+  else if (pl <= 4) MOE_TOPK(4);
+  else if (pl <= 8) MOE_TOPK(8);
+  else if (pl <= 16) MOE_TOPK(16);
+  else MOE_TOPK(32);
+#undef MOE_TOPK
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -92,27 +92,39 @@ def select_topk(scores: torch.Tensor, k: int) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(order[:, :k])).to(torch.int64)
 
 
-def gate(x, w_router, corr_bias, n_routed: int, top_k: int, n_shared: int,
-         route_scale: float, global_scale: float) -> Dict[str, torch.Tensor]:
-    """``InklingGate.forward``: returns (topk_weights, topk_indices, shared_gammas).
-
-    Weights: p = softmax([logsig(z_sel_0..k-1) ++ logsig(z_shared_0..S-1)]),
-    then every entry times route_scale * global_scale; the first k entries
-    are the routed weights, the last S the shared gammas (``InklingGate``
-    docstring).  The correction bias enters the selection only.
-    """
-    E, k, S = n_routed, top_k, n_shared
-    z = router_logits(x, w_router)                       # [T, E+S]
-    scores = selection_scores(z[:, :E], corr_bias)       # [T, E]
-    idx = select_topk(scores, k)                         # [T, k]
+def routing_weights(z: torch.Tensor, idx: torch.Tensor, n_routed: int, n_shared: int,
+                    route_scale: float, global_scale: float):
+    """Weights of a given selection: p = softmax([logsig(z_sel_0..k-1) ++
+    logsig(z_shared_0..S-1)]), every entry times route_scale * global_scale;
+    the first k entries are the routed weights, the last S the shared gammas
+    (``InklingGate`` docstring)."""
+    E, S = n_routed, n_shared
+    k = idx.shape[1]
     z_sel = torch.gather(z[:, :E], 1, idx)               # [T, k]
     v = torch.cat([F.logsigmoid(z_sel), F.logsigmoid(z[:, E:E + S])], dim=1)
     p = torch.softmax(v, dim=1)
     scale = float(route_scale) * float(global_scale)
+    return p[:, :k] * scale, p[:, k:] * scale
+
+
+def gate(x, w_router, corr_bias, n_routed: int, top_k: int, n_shared: int,
+         route_scale: float, global_scale: float,
+         given_topk_idx: Optional[torch.Tensor] = None) -> Dict[str, torch.Tensor]:
+    """``InklingGate.forward``: returns (topk_weights, topk_indices, shared_gammas).
+
+    The correction bias enters the selection only; the weights follow
+    ``routing_weights``.  ``given_topk_idx`` replaces the selection (used to
+    evaluate the layer on a selection decided elsewhere, e.g. at a near-tie).
+    """
+    E, k, S = n_routed, top_k, n_shared
+    z = router_logits(x, w_router)                       # [T, E+S]
+    scores = selection_scores(z[:, :E], corr_bias)       # [T, E]
+    idx = select_topk(scores, k) if given_topk_idx is None else given_topk_idx.to(torch.int64)
+    topk_w, gamma = routing_weights(z, idx, E, S, route_scale, global_scale)
     # diagnostic: the selection margin between the k-th and (k+1)-th score
     ranked = torch.gather(scores, 1, select_topk(scores, min(k + 1, E)))
     gap = (ranked[:, k - 1] - ranked[:, k]) if k < E else torch.full((z.shape[0],), float("inf"), dtype=F64)
-    return {"topk_w": p[:, :k] * scale, "topk_idx": idx, "shared_gamma": p[:, k:] * scale,
+    return {"topk_w": topk_w, "topk_idx": idx, "shared_gamma": gamma,
             "logits": z, "scores": scores, "gap": gap}
 
 
@@ -167,11 +179,13 @@ def moe_forward(inputs: Dict[str, torch.Tensor], n_routed: int, top_k: int, n_sh
                 route_scale: float, global_scale: float,
                 tokens: Optional[torch.Tensor] = None,
                 padding_mask: Optional[torch.Tensor] = None,
-                threads: Optional[int] = None) -> Dict[str, torch.Tensor]:
+                threads: Optional[int] = None,
+                given_topk_idx: Optional[torch.Tensor] = None) -> Dict[str, torch.Tensor]:
     """``InklingMoE.forward``: out[t] = shared(t) + sum_j y[t, j], j ascending.
 
     ``tokens`` restricts the evaluation to a subset of token rows (the layer
     is per-token, so each row's result is the same as in a full run).
+    ``given_topk_idx`` (rows matching ``tokens``) replaces the selection.
     Returns float64 tensors for the evaluated rows.
     """
     if threads is not None:
@@ -181,7 +195,7 @@ def moe_forward(inputs: Dict[str, torch.Tensor], n_routed: int, top_k: int, n_sh
     if padding_mask is not None:
         pm = padding_mask if tokens is None else padding_mask[tokens]
     g = gate(x, inputs["w_router"], inputs["corr_bias"], n_routed, top_k, n_shared,
-             route_scale, global_scale)
+             route_scale, global_scale, given_topk_idx=given_topk_idx)
     x64 = _f64(x)
     sh = shared_experts(x64, g["shared_gamma"], inputs["ws_gate_up"], inputs["ws_down"])
     y = routed_experts(x64, g["topk_idx"], g["topk_w"], inputs["w_gate_up"], inputs["w_down"], pm)
@@ -191,10 +205,12 @@ def moe_forward(inputs: Dict[str, torch.Tensor], n_routed: int, top_k: int, n_sh
     return {"out": out, "shared": sh, "routed": y, **g}
 
 
-def moe_forward_workload(inputs, w, tokens=None, padding_mask=None, threads=None):
+def moe_forward_workload(inputs, w, tokens=None, padding_mask=None, threads=None,
+                         given_topk_idx=None):
     """``moe_forward`` with the layer constants taken from a workload record."""
     return moe_forward(inputs, w.E, w.k, w.S, w.route_scale, w.global_scale,
-                       tokens=tokens, padding_mask=padding_mask, threads=threads)
+                       tokens=tokens, padding_mask=padding_mask, threads=threads,
+                       given_topk_idx=given_topk_idx)
 
 
 # ------------------------------------------------------------- permutation

@@ -1,0 +1,117 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point the header declares, and rejects bad arguments on the host before any
+CUDA call.  No compute call is made here."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import mixture_experts_feed_b200 as moe
+import moe_workloads as mw
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                      "include", "inkling_moe.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_five_ops():
+    names = declared_functions()
+    for f in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
+              "moe_workspace_size"):
+        assert f in names
+
+
+def test_library_exports_every_declared_symbol():
+    for name in declared_functions():
+        assert hasattr(moe.LIB, name), f"{name} not exported by {moe.LIB_PATH}"
+
+
+def test_version_and_strings():
+    assert moe.LIB.moe_version() >= 1
+    for code in range(7):
+        assert moe.LIB.moe_status_string(code)
+
+
+def test_desc_struct_layout_matches_header():
+    # int64 + 6 x int32 + 2 x float, naturally aligned
+    assert ctypes.sizeof(moe.LayerDesc) == 40
+    assert moe.LayerDesc.route_scale.offset == 32
+
+
+@pytest.mark.parametrize("w", mw.ORDERED, ids=[w.name for w in mw.ORDERED])
+def test_workspace_size_covers_intermediates(w):
+    L = moe.Layer.from_workload(w)
+    n = moe.workspace_size(L)
+    el = 4 if w.dtype == "f32" else 2
+    Rk = w.T * w.k
+    need = el * (Rk * w.H + (Rk + w.S * w.T) * w.I) + 4 * (Rk + w.S * w.T) * w.H
+    assert n >= need
+    assert moe.forward_kernel_count(L) == 9
+
+
+def _status(fn, *args):
+    return getattr(moe.LIB, fn)(*args)
+
+
+def test_invalid_descriptors_are_rejected():
+    n = ctypes.c_size_t(0)
+    bad = [
+        moe.Layer(4, 128, 8, 0, 1, 64),        # k = 0
+        moe.Layer(4, 128, 8, 9, 1, 64),        # k > E
+        moe.Layer(-1, 128, 8, 2, 1, 64),       # T < 0
+        moe.Layer(4, 0, 8, 2, 1, 64),          # H = 0
+    ]
+    for L in bad:
+        assert _status("moe_workspace_size", ctypes.byref(L.desc()), ctypes.byref(n)) == 1
+    unsupported = [
+        moe.Layer(4, 100, 8, 2, 1, 64),        # H not a multiple of 64
+        moe.Layer(4, 128, 8, 2, 1, 48),        # I not a multiple of 64
+        moe.Layer(4, 128, 2048, 2, 1, 64),     # E > 1024
+        moe.Layer(4, 128, 64, 17, 1, 64),      # k > 16
+        moe.Layer(4, 128, 8, 2, 9, 64),        # S > 8
+    ]
+    for L in unsupported:
+        assert _status("moe_workspace_size", ctypes.byref(L.desc()), ctypes.byref(n)) == 2
+    assert _status("moe_workspace_size", None, ctypes.byref(n)) == 1
+    assert _status("moe_workspace_size", ctypes.byref(moe.Layer(4, 128, 8, 2, 1, 64).desc()), None) == 1
+
+
+def test_null_and_misaligned_pointers_are_rejected_before_launch():
+    L = moe.Layer(16, 128, 8, 2, 1, 64)
+    d = ctypes.byref(L.desc())
+    fake = 1 << 20          # aligned, never dereferenced: the checks fail first
+    ws_ok = moe.workspace_size(L)
+    # null x
+    assert _status("moe_route", d, None, fake, fake, fake, fake, fake, fake, ws_ok, None) == 1
+    # misaligned x
+    assert _status("moe_route", d, fake + 2, fake, fake, fake, fake, fake, fake, ws_ok, None) == 1
+    # missing gamma with S > 0
+    assert _status("moe_route", d, fake, fake, fake, fake, fake, None, fake, ws_ok, None) == 1
+    # workspace too small
+    assert _status("moe_route", d, fake, fake, fake, fake, fake, fake, fake, ws_ok - 1, None) == 3
+    # workspace misaligned
+    assert _status("moe_route", d, fake, fake, fake, fake, fake, fake, fake + 16, ws_ok, None) == 1
+    assert _status("moe_permute", d, None, None, fake, fake, fake, fake, fake, fake, ws_ok, None) == 1
+    assert _status("moe_expert_ffn", d, fake, fake, fake, fake, fake, None, fake, fake, fake, fake,
+                   fake, fake, fake, ws_ok, None) == 1
+    assert _status("moe_combine", d, fake, fake, fake, None, fake, ws_ok, None) == 1
+    assert _status("moe_forward", d, fake, fake, fake, fake, fake, None, fake, None, fake,
+                   None, None, None, fake, ws_ok, None) == 1
+    assert _status("moe_workspace_init", None, 1024, None) == 1
+    assert _status("moe_read_device_status", None, None, None) == 1
+
+
+def test_binding_checks_shapes_on_host():
+    L = moe.Layer(4, 128, 8, 2, 1, 64, torch.float32)
+    x = torch.zeros(4, 64)   # wrong H, on CPU: rejected before the C call
+    with pytest.raises(ValueError):
+        moe.moe_combine(L, x, x, torch.zeros(8, dtype=torch.int32), x, torch.zeros(16, dtype=torch.uint8))

@@ -328,8 +328,8 @@ def test_planted_raw_shared_logits_is_caught(monkeypatch):
     is told apart by the two-token example."""
     real_gate = oracle.gate
 
-    def reading_b(x, w_router, corr_bias, E, k, S, rs, gs):
-        r = real_gate(x, w_router, corr_bias, E, k, S, rs, gs)
+    def reading_b(x, w_router, corr_bias, E, k, S, rs, gs, given_topk_idx=None):
+        r = real_gate(x, w_router, corr_bias, E, k, S, rs, gs, given_topk_idx)
         z = r["logits"]
         v = torch.cat([F.logsigmoid(torch.gather(z[:, :E], 1, r["topk_idx"])), z[:, E:E + S]], 1)
         p = torch.softmax(v, 1) * rs * gs
