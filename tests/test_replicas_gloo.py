@@ -1,0 +1,61 @@
+"""Host logic of bench.py's replica mode on CPU, world size 2, gloo.
+
+The layer has no exchange step, so N GPUs run N independent replicas; the
+only cross-rank work is the timing reduction (max over ranks) and the
+barriers around the timed region.  These run here as two CPU processes.
+"""
+from __future__ import annotations
+
+import os
+import socket
+import subprocess
+import sys
+
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port),
+                       "RANK": str(rank), "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank)})
+    sys.path.insert(0, ROOT)
+    import bench
+    w, r, _ = bench.dist_setup(None)
+    assert (w, r) == (world, rank)
+    per_rank_ms = [3.0, 7.5][rank]
+    bench.barrier(w)
+    got = bench.max_over_ranks(per_rank_ms, w)
+    q.put((rank, got))
+    bench.finish(w)
+
+
+def test_max_over_ranks_world2_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    results = dict(q.get(timeout=10) for _ in range(2))
+    assert results == {0: 7.5, 1: 7.5}
+
+
+def test_reference_arm_nonzero_rank_exits_without_work():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True,
+                       timeout=120)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""
