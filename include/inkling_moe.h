@@ -132,6 +132,31 @@ moe_status_t moe_permute(const moe_layer_desc_t* desc, const int32_t* topk_idx,
                          size_t workspace_bytes, void* stream);
 
 /*
+ * moe_permute_noalloc — moe_permute without a workspace, for callers that
+ * cannot allocate device memory (for example a plugin inside an inference
+ * engine that plans all device memory ahead of time and forbids allocation
+ * in its enqueue step, or a process held to a fixed device-memory budget).
+ * The pages have no counterpart of this entry point; it is an addition for
+ * such callers.  Arguments, outputs and results are those of moe_permute.
+ *   - The per-expert counters live in a static device array of 1024 int32
+ *     (4 KiB) that every GPU loading the library keeps until exit, so
+ *     E must be <= 1024 (else MOE_ERR_UNSUPPORTED).
+ *   - The first call on a device looks up that array's device address (a
+ *     one-time set-up per device); make that first call before any stream
+ *     capture.
+ *   - All calls share the array and it keeps the last call's contents; each
+ *     call clears it on `stream` first.  Calls that overlap on the GPU
+ *     (other streams or threads) race on it: order them.
+ *   - With no status word, an out-of-range expert id is skipped (its slot
+ *     gets inv_perm = -1) but not reported.
+ * It allocates nothing (no cudaMalloc, no cudaFree).
+ */
+moe_status_t moe_permute_noalloc(const moe_layer_desc_t* desc, const int32_t* topk_idx,
+                                 const uint8_t* padding_mask, const void* x,
+                                 int32_t* expert_offsets, int32_t* perm_slot, int32_t* inv_perm,
+                                 void* x_perm, void* stream);
+
+/*
  * moe_expert_ffn — the routed experts over the permuted rows and the shared
  * experts over all tokens (layers page: inkling_swiglu, InklingSharedExperts).
  * For routed row r of expert e (token t, choice j, weight w = topk_w[t*k+j]):

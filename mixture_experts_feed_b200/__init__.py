@@ -61,11 +61,12 @@ LIB.moe_workspace_init.argtypes = [_P, ctypes.c_size_t, _P]
 LIB.moe_read_device_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_int32)]
 LIB.moe_route.argtypes = [_DESC, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 LIB.moe_permute.argtypes = [_DESC, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+LIB.moe_permute_noalloc.argtypes = [_DESC, _P, _P, _P, _P, _P, _P, _P, _P]
 LIB.moe_expert_ffn.argtypes = [_DESC] + [_P] * 13 + [ctypes.c_size_t, _P]
 LIB.moe_combine.argtypes = [_DESC, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 LIB.moe_forward.argtypes = [_DESC] + [_P] * 13 + [ctypes.c_size_t, _P]
 for _f in ("moe_workspace_size", "moe_workspace_init", "moe_read_device_status", "moe_route",
-           "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward"):
+           "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_combine", "moe_forward"):
     getattr(LIB, _f).restype = ctypes.c_int
 
 
@@ -174,6 +175,24 @@ def moe_permute(layer: Layer, topk_idx, padding_mask, x, expert_offsets, perm_sl
     _check(LIB.moe_permute(ctypes.byref(L.desc()), _ptr(topk_idx), _ptr(padding_mask), _ptr(x),
                            _ptr(expert_offsets), _ptr(perm_slot), _ptr(inv_perm), _ptr(x_perm),
                            ws.data_ptr(), ws.numel(), _stream(stream)), "moe_permute")
+
+
+def moe_permute_noalloc(layer: Layer, topk_idx, padding_mask, x, expert_offsets, perm_slot,
+                        inv_perm, x_perm, stream=None):
+    """``moe_permute`` without a workspace, for callers that cannot allocate
+    device memory (its scratch is a static device array; E <= 1024; calls
+    that overlap on the GPU race on that array)."""
+    L = layer
+    _expect(topk_idx, "topk_idx", (L.T, L.k), torch.int32)
+    _expect(padding_mask, "padding_mask", (L.T,), torch.uint8, allow_none=True)
+    _expect(x, "x", (L.T, L.H), L.dtype)
+    _expect(expert_offsets, "expert_offsets", (L.E + 1,), torch.int32)
+    _expect(perm_slot, "perm_slot", (L.T * L.k,), torch.int32)
+    _expect(inv_perm, "inv_perm", (L.T * L.k,), torch.int32)
+    _expect(x_perm, "x_perm", (L.T * L.k, L.H), L.dtype)
+    _check(LIB.moe_permute_noalloc(ctypes.byref(L.desc()), _ptr(topk_idx), _ptr(padding_mask),
+                                   _ptr(x), _ptr(expert_offsets), _ptr(perm_slot), _ptr(inv_perm),
+                                   _ptr(x_perm), _stream(stream)), "moe_permute_noalloc")
 
 
 def moe_expert_ffn(layer: Layer, x, x_perm, expert_offsets, perm_slot, topk_w, shared_gamma,

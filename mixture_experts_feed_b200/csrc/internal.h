@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "inkling_moe.h"
+
 namespace moe {
 
 struct Layer {
@@ -12,6 +14,11 @@ struct Layer {
   int dtype;   // MOE_F32 / MOE_BF16
   float route_scale, global_scale;
 };
+
+// moe_api.cu: SM count of the current device (cached per device), and the
+// host-side check of a layer description (fills `L` when it returns MOE_OK).
+int device_sm_count();
+moe_status_t validate_desc(const moe_layer_desc_t* d, Layer* L);
 
 // router.cu
 cudaError_t launch_router_logits(const Layer& L, const void* x, const float* w_router,

@@ -86,7 +86,11 @@ moe_status_t check_ws(const Layer& L, const void* ws, size_t bytes) {
   return MOE_OK;
 }
 
-int num_sms() {
+}  // namespace
+
+moe_status_t validate_desc(const moe_layer_desc_t* d, Layer* L) { return check_desc(d, L); }
+
+int device_sm_count() {
   static int cached[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -99,6 +103,10 @@ int num_sms() {
   }
   return cached[dev];
 }
+
+namespace {
+
+int num_sms() { return device_sm_count(); }
 
 template <typename P>
 P* region(void* ws, size_t off) {
