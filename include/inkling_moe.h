@@ -17,7 +17,7 @@
  *     routing weight (inkling_swiglu), down projection.
  *   - InklingMoE.forward: shared plus routed, recombined per token; leading
  *     dims of the input are flattened to tokens by the caller; padded tokens
- *     are excluded from routed dispatch.
+ *     never reach a routed expert.
  *
  * Conventions shared by every entry point
  *   - All tensors are caller-owned DEVICE buffers, row-major and contiguous,
@@ -27,8 +27,8 @@
  *     runs before any launch; a non-OK return means nothing was launched
  *     (MOE_ERR_CUDA: a launch was attempted and CUDA reported an error).
  *   - Weights use the checkpoint's [out_features, in_features] orientation
- *     (the pages note the fused projection stays in the checkpoint layout so
- *     loading needs only transpose views):
+ *     (the pages keep the fused projection in the checkpoint's layout, which
+ *     loading reaches through a transposed view):
  *       w_router   [E+S, H] fp32    rows 0..E-1 routed, E..E+S-1 shared
  *       corr_bias  [E]      fp32
  *       w_gate_up  [E, 2I, H]       row 2j = gate_j, row 2j+1 = up_j
@@ -115,7 +115,7 @@ moe_status_t moe_route(const moe_layer_desc_t* desc, const void* x, const float*
 /*
  * moe_permute — grouped dispatch order for the routed experts (layers page,
  * InklingMoE docstring: grouped routed experts; InklingMoE.forward: padded
- * tokens are excluded from routed dispatch).  Every live (token t, choice j)
+ * tokens never reach a routed expert).  Every live (token t, choice j)
  * pair becomes one row; rows are ordered by (expert, token) ascending.
  *   topk_idx       [T, k] int32 in, values in [0, E)
  *   padding_mask   [T] uint8 (nonzero = padded) or NULL

@@ -3,7 +3,7 @@
 //   out[t] = sum_s y_shared[s*T + t] + sum_j y_routed[inv_perm[t*k + j]]
 // in fp32, in that fixed order (shared s ascending, then choices j
 // ascending), rounded once to the output dtype.  The rows are fp32.  The routing weights are
-// already folded into the rows (inkling_swiglu scales the activated output),
+// already folded into the rows (inkling_swiglu multiplies silu(g)*u by them),
 // so the sum is unweighted.  One block per token; 16-byte vector loads and
 // stores along the hidden dim, coalesced across the block.  HBM-bound.
 #include <algorithm>

@@ -1,4 +1,4 @@
-// Grouped expert GEMMs on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+// Grouped GEMMs on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
 // One persistent kernel computes, for every group of rows (a routed expert or
 // a shared expert, see grouping.cuh), D = A_rows @ W_g^T with bf16 operands
@@ -12,18 +12,28 @@
 //            stay fp32 until the recombination rounds the layer output once
 //            (rounding them to bf16 as well would put a correct pipeline at
 //            about 2% of the output RMS, the edge of the 2e-2 bound).
+//   kRouter: router logits z = x @ Wr^T, the fp32 router bank split exactly
+//            into three bf16 parts (W = W0 + W1 + W2) so that every product
+//            is exact.  The tensor-core accumulator loses about one fp32 ulp
+//            of its own magnitude per MMA step (measured: 5.7e-5 in z over a
+//            3 x 6144 chain), so each accumulation chain is kept to one
+//            64-deep K block: the MMA writes a fresh block sum, and the
+//            epilogue warps add the block sums in fp32 registers with
+//            round-to-nearest adds.  fp32 logits out.  One group (all T
+//            tokens), N = E + S, 128-column tiles.
 //
 // Roles (192 threads, one CTA per SM):
 //   warp 0      TMA producer: A tile [128 rows x 64 K] and B tile
-//               [256 rows x 64 K] per stage, 128-byte swizzle, 4 stages.
+//               [BN rows x 64 K] per stage, 128-byte swizzle, 4 stages.
 //   warp 1      TMEM allocator and MMA issuer (one thread): 4 x
-//               tcgen05.mma M128 N256 K16 per stage into one of two
-//               accumulators (2 x 256 TMEM columns).
+//               tcgen05.mma M128 N<=BN K16 per stage into one of two
+//               accumulators (2 x BN TMEM columns).
 //   warps 2..5  epilogue: tcgen05.ld the accumulator rows (warp w reads TMEM
-//               lanes 32*(w%4) .. +31), fused math, 16-byte global stores.
-// The two accumulators let the epilogue of tile i overlap the MMAs of i+1.
-// All waits are bounded (sm100_ptx.cuh); on a timeout every role stops,
-// the status word records it and TMEM is released.
+//               lanes 32*(w%4) .. +31), fused math, global stores.
+// The two accumulators let the epilogue of one tile (or, for kRouter, one K
+// block) overlap the MMAs of the next.  All waits are bounded
+// (sm100_ptx.cuh); on a timeout every role stops, the status word records it
+// and TMEM is released.  No TMA load uses cluster multicast.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -37,16 +47,19 @@ namespace moe {
 namespace sm100 {
 
 constexpr int BM = 128;
-constexpr int BN = 256;
 constexpr int BK = 64;
 constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
 constexpr int NUM_THREADS = 192;
-constexpr uint32_t TMEM_COLS = 512;   // two 256-column fp32 accumulators
-constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
 
-enum Mode { kGateUp = 0, kDown = 1 };
+enum Mode { kGateUp = 0, kDown = 1, kRouter = 2 };
+
+template <int MODE> struct Tile {
+  static constexpr int BN = MODE == kRouter ? 128 : 256;   // accumulator columns
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;            // two accumulators
+  static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+};
 
 struct alignas(64) GemmParams {
   CUtensorMap tmA[2];   // A operand of routed (0) and shared (1) groups: 2-D [rows, K]
@@ -62,47 +75,86 @@ struct alignas(64) GemmParams {
   int E, S, K, N;
   int ld_out;                 // output row length in elements
   int rows_cap;               // rows of the routed A operand (bound of offsets)
+  int ksplit;                 // kRouter: K-range splits (each writes its own partial)
+  int64_t split_stride;       // kRouter: elements between partial outputs
 };
 
-struct SmemLayout {
+// Per epilogue warp, a 32 x 32 fp32 staging tile (row stride 36 floats:
+// 16-byte aligned, and each quarter-warp's 16-byte accesses hit distinct banks).
+constexpr int STAGE_LD = 36;
+constexpr int STAGE_WARP_BYTES = 32 * STAGE_LD * 4;
+
+template <int MODE> struct SmemLayout {
   static constexpr int kA = 0;
   static constexpr int kB = STAGES * A_BYTES;
-  static constexpr int kBars = kB + STAGES * B_BYTES;
+  static constexpr int kStage = kB + STAGES * Tile<MODE>::B_BYTES;   // 4 x STAGE_WARP_BYTES
+  static constexpr int kBars = kStage + 4 * STAGE_WARP_BYTES;
   // full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
   static constexpr int kNumBars = 2 * STAGES + 5;
   static constexpr int kMisc = kBars + kNumBars * 8;   // tmem base, abort, bad
   static constexpr int kTables = kMisc + 16;
 };
 
+template <int MODE>
 __host__ __device__ inline int smem_bytes(int E, int S) {
-  return 1024 /* alignment slack */ + SmemLayout::kTables + 4 * ((E + 1) + (E + S + 1));
+  return 1024 /* alignment slack */ + SmemLayout<MODE>::kTables + 4 * ((E + 1) + (E + S + 1));
+}
+
+// Write one warp's 32 rows x 32 fp32 columns through the staging tile so that
+// each store instruction covers 4 whole 128-byte row segments.
+__device__ __forceinline__ void store_rows_f32(float* st, const uint32_t (&v)[32], int lane,
+                                               float* out, int64_t row0, int rows_left,
+                                               int64_t ld, int col0) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    *reinterpret_cast<uint4*>(st + lane * STAGE_LD + 4 * q) =
+        make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  __syncwarp();
+  const int sub_row = lane >> 3;          // 0..3
+  const int sub_col = (lane & 7) * 4;     // 0..28
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int rr = it * 4 + sub_row;      // row inside the warp's 32
+    const float4 val = *reinterpret_cast<const float4*>(st + rr * STAGE_LD + sub_col);
+    if (rr < rows_left)
+      *reinterpret_cast<float4*>(out + (row0 + rr) * ld + col0 + sub_col) = val;
+  }
+  __syncwarp();
 }
 
 template <int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
+  using TL = Tile<MODE>;
+  using SL = SmemLayout<MODE>;
+  constexpr int BN = TL::BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* sA = smem + SmemLayout::kA;
-  uint8_t* sB = smem + SmemLayout::kB;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SmemLayout::kBars);
+  uint8_t* sA = smem + SL::kA;
+  uint8_t* sB = smem + SL::kB;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SL::kBars);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
   uint64_t* tempty = bars + 2 * STAGES + 2;
   uint64_t* drain = bars + 2 * STAGES + 4;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + SmemLayout::kMisc);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SmemLayout::kMisc + 4);
-  int* s_bad = reinterpret_cast<int*>(smem + SmemLayout::kMisc + 8);
-  int* s_off = reinterpret_cast<int*>(smem + SmemLayout::kTables);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + SL::kMisc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SL::kMisc + 4);
+  int* s_bad = reinterpret_cast<int*>(smem + SL::kMisc + 8);
+  int* s_off = reinterpret_cast<int*>(smem + SL::kTables);
   int* s_tile = s_off + (p.E + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = p.E + p.S;
-  const int n_tiles = (p.N + BN - 1) / BN;
-  const int k_blocks = p.K / BK;
+  // kRouter folds its K splits into the n-tile index: nv = n * ksplit + ks
+  const int ksplit = MODE == kRouter ? p.ksplit : 1;
+  const int n_tiles = (p.N + BN - 1) / BN * ksplit;
+  const int k_blocks = p.K / BK;                               // per weight part
+  const int k_total = MODE == kRouter ? 3 * k_blocks : k_blocks;
+  // K-block range [kt_begin(ks), kt_begin(ks + 1)) of split ks
+  auto kt_begin = [&](int ks) { return static_cast<int>(static_cast<int64_t>(k_total) * ks / ksplit); };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -126,7 +178,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    tmem_alloc(s_tmem, TMEM_COLS);
+    tmem_alloc(s_tmem, TL::TMEM_COLS);
     tmem_relinquish();
   } else if (warp == 2) {
     build_tile_prefix(p.offsets, p.E, p.S, p.T, BM, n_tiles, p.rows_cap, s_off, s_tile, s_bad);
@@ -147,18 +199,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
     for (int i = 0; i < STAGES; ++i) last_parity[i] = -1;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      int g, m, n;
-      decode_tile(tile, s_tile, G, s_off, p.E, p.T, BM, g, m, n);
+      int g, m, nv;
+      decode_tile(tile, s_tile, G, s_off, p.E, p.T, BM, g, m, nv);
+      const int n = nv / ksplit, ks = nv - n * ksplit;
       const GroupInfo gi = group_info(g, s_off, p.E, p.T, p.a1_base, p.a1_stride);
       const void* tmA = &p.tmA[gi.src];
       const void* tmB = &p.tmB[gi.src];
       const int a_row = static_cast<int>(gi.a_row0) + m * BM;
       bool ok = true;
-      for (int kb = 0; kb < k_blocks; ++kb) {
+      for (int kt = kt_begin(ks); kt < kt_begin(ks + 1); ++kt) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, s_abort, p.status)) { ok = false; break; }
-        mbar_arrive_expect_tx(&full[stage], A_BYTES + B_BYTES);
+        // router: part 2 (smallest) first, then 1, then 0
+        const int kb = MODE == kRouter ? kt % k_blocks : kt;
+        const int slice = MODE == kRouter ? 2 - kt / k_blocks : gi.b_idx;
+        mbar_arrive_expect_tx(&full[stage], A_BYTES + TL::B_BYTES);
         tma_load_2d(sA + stage * A_BYTES, tmA, &full[stage], kb * BK, a_row);
-        tma_load_3d(sB + stage * B_BYTES, tmB, &full[stage], kb * BK, n * BN, gi.b_idx);
+        tma_load_3d(sB + stage * TL::B_BYTES, tmB, &full[stage], kb * BK, n * BN, slice);
         last_parity[stage] = static_cast<int>(phase);
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
@@ -177,30 +233,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------- MMA issuer
     int stage = 0;
     uint32_t phase = 0;
-    int it = 0;
+    int it = 0;   // accumulator hand-offs so far (tiles, or K blocks for kRouter)
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++it) {
-      const int acc = it & 1;
-      const uint32_t aphase = (it >> 1) & 1;
-      if (!mbar_wait(&tempty[acc], aphase ^ 1u, s_abort, p.status)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-      for (int kb = 0; kb < k_blocks; ++kb) {
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      int g, m, nv;
+      decode_tile(tile, s_tile, G, s_off, p.E, p.T, BM, g, m, nv);
+      const int n = nv / ksplit, ks = nv - n * ksplit;
+      // the last n-tile of a ragged N runs a narrower MMA (N multiple of 16)
+      const int n_here = min(BN, p.N - n * BN);
+      const uint32_t idesc = n_here >= BN ? TL::IDESC : idesc_bf16_f32(BM, (n_here + 15) & ~15);
+      if (MODE != kRouter) {
+        const int acc = it & 1;
+        if (!mbar_wait(&tempty[acc], ((it >> 1) & 1) ^ 1u, s_abort, p.status)) { ok = false; break; }
+        tc_fence_after();
+      }
+      for (int kb = kt_begin(ks); kb < kt_begin(ks + 1); ++kb) {
+        const int acc = it & 1;
+        if (MODE == kRouter) {   // one hand-off per K block
+          if (!mbar_wait(&tempty[acc], ((it >> 1) & 1) ^ 1u, s_abort, p.status)) { ok = false; break; }
+          tc_fence_after();
+        }
         if (!mbar_wait(&full[stage], phase, s_abort, p.status)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         const uint64_t adesc = smem_desc_kmajor_sw128(smem_u32(sA + stage * A_BYTES));
-        const uint64_t bdesc = smem_desc_kmajor_sw128(smem_u32(sB + stage * B_BYTES));
+        const uint64_t bdesc = smem_desc_kmajor_sw128(smem_u32(sB + stage * TL::B_BYTES));
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           // +32 bytes per K=16 step inside the 128-byte swizzle atom
+          // router: a fresh block sum per K block; experts: accumulate over the tile
+          const bool accumulate = MODE == kRouter ? (kk != 0) : ((kb | kk) != 0);
           mma_bf16_ss(d_tmem, adesc + static_cast<uint64_t>(2 * kk),
-                      bdesc + static_cast<uint64_t>(2 * kk), IDESC, (kb | kk) != 0 ? 1u : 0u);
+                      bdesc + static_cast<uint64_t>(2 * kk), idesc, accumulate ? 1u : 0u);
         }
         mma_commit(&empty[stage]);
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        if (MODE == kRouter) {
+          mma_commit(&tfull[acc]);
+          ++it;
+        }
       }
       if (!ok) break;
-      mma_commit(&tfull[acc]);
+      if (MODE != kRouter) {
+        mma_commit(&tfull[it & 1]);
+        ++it;
+      }
     }
     // Every MMA this thread issued must be complete before TMEM is freed.
     mma_commit(drain);
@@ -212,19 +289,63 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // --------------------------------------------------------- epilogue
     const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
     const int row_in_tile = quarter * 32 + lane;
+    float* st = reinterpret_cast<float*>(smem + SL::kStage) + (warp - 2) * (STAGE_WARP_BYTES / 4);
+    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     int it = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
-      int g, m, n;
-      decode_tile(tile, s_tile, G, s_off, p.E, p.T, BM, g, m, n);
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      int g, m, nv;
+      decode_tile(tile, s_tile, G, s_off, p.E, p.T, BM, g, m, nv);
+      const int n = nv / ksplit, ks = nv - n * ksplit;
       const GroupInfo gi = group_info(g, s_off, p.E, p.T, p.a1_base, p.a1_stride);
-      const int acc = it & 1;
-      const uint32_t aphase = (it >> 1) & 1;
-      if (!mbar_wait(&tfull[acc], aphase, s_abort, p.status)) break;
-      tc_fence_after();
-
       const int r = m * BM + row_in_tile;          // row inside the group
       const bool valid = r < gi.rows;
       const int64_t out_row = gi.out_row0 + r;
+      const int rows_left = gi.rows - (m * BM + quarter * 32);   // rows of this warp's 32
+
+      if (MODE == kRouter) {
+        // Sum the per-K-block accumulators in fp32 registers (round to nearest).
+        float run[BN];
+#pragma unroll
+        for (int i = 0; i < BN; ++i) run[i] = 0.0f;
+        for (int kb = kt_begin(ks); kb < kt_begin(ks + 1); ++kb) {
+          const int acc = it & 1;
+          if (!mbar_wait(&tfull[acc], (it >> 1) & 1, s_abort, p.status)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c) {
+            if (n * BN + c * 32 < p.N) {            // warp-uniform
+              uint32_t v[32];
+              tmem_ld_32x32b_x32(t_lane + static_cast<uint32_t>(acc * BN + c * 32), v);
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) run[c * 32 + i] += __uint_as_float(v[i]);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[acc]);
+          ++it;
+        }
+        if (!ok) break;
+        float* out = static_cast<float*>(p.out[gi.src]) + ks * p.split_stride;
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          const int col0 = n * BN + c * 32;
+          if (col0 < p.N) {
+            uint32_t v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(run[c * 32 + i]);
+            store_rows_f32(st, v, lane, out, gi.out_row0 + m * BM + quarter * 32, rows_left,
+                           p.ld_out, col0);
+          }
+        }
+        continue;
+      }
+
+      const int acc = it & 1;
+      if (!mbar_wait(&tfull[acc], (it >> 1) & 1, s_abort, p.status)) break;
+      tc_fence_after();
       float w = 1.0f;
       if (MODE == kGateUp && valid) {
         if (gi.src == 0) {
@@ -239,8 +360,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           w = p.gamma[static_cast<int64_t>(r) * p.S + gi.s];
         }
       }
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                             static_cast<uint32_t>(acc * BN);
+      const uint32_t t_row = t_lane + static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         const int col0 = n * BN + c * 32;
@@ -248,8 +368,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t v[32];
         tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * 32), v);
         tmem_ld_wait();
-        if (!valid) continue;
         if (MODE == kGateUp) {
+          if (!valid) continue;
           uint32_t packed[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -266,16 +386,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
           dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
         } else {
-          float* out = static_cast<float*>(p.out[gi.src]);
-          uint4* dst = reinterpret_cast<uint4*>(out + out_row * p.ld_out + col0);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          store_rows_f32(st, v, lane, static_cast<float*>(p.out[gi.src]),
+                         gi.out_row0 + m * BM + quarter * 32, rows_left, p.ld_out, col0);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
+      ++it;
     }
   }
 
@@ -283,7 +401,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc(tmem_base, TL::TMEM_COLS);
   }
 }
 
@@ -314,15 +432,15 @@ static bool encode_a(CUtensorMap* m, const void* base, int64_t rows, int K) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D bf16 map over [G][N][K] (K contiguous), box [1][BN][BK], 128B swizzle.
-static bool encode_b(CUtensorMap* m, const void* base, int G, int N, int K) {
+// 3-D bf16 map over [G][N][K] (K contiguous), box [1][bn][BK], 128B swizzle.
+static bool encode_b(CUtensorMap* m, const void* base, int G, int N, int K, int bn) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N),
                         static_cast<cuuint64_t>(G)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2,
                            static_cast<cuuint64_t>(K) * 2 * static_cast<cuuint64_t>(N)};
-  cuuint32_t box[3] = {BK, BN, 1};
+  cuuint32_t box[3] = {BK, static_cast<cuuint32_t>(bn), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -331,7 +449,7 @@ static bool encode_b(CUtensorMap* m, const void* base, int G, int N, int K) {
 
 template <int MODE>
 static cudaError_t launch_mode(const GemmParams& p, int sms, cudaStream_t stream) {
-  const int smem = smem_bytes(p.E, p.S);
+  const int smem = smem_bytes<MODE>(p.E, p.S);
   static int configured_smem[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -347,8 +465,6 @@ static cudaError_t launch_mode(const GemmParams& p, int sms, cudaStream_t stream
 
 }  // namespace sm100
 
-int sm100_gemm_max_smem(int E, int S) { return sm100::smem_bytes(E, S); }
-
 // gate_up: A0 = x_perm [T*k, H], A1 = x [T, H]; out0 = h rows [0, T*k),
 // out1 = h rows T*k + s*T + t.  down: A0 = A1 = h [T*k + S*T, I];
 // out0 = y_routed, out1 = y_shared.
@@ -360,6 +476,7 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
                                    int32_t* status, int num_sms, cudaStream_t stream,
                                    bool* map_error) {
   using namespace sm100;
+  constexpr int BN = Tile<kGateUp>::BN;
   *map_error = false;
   const int64_t Rk = L.T * L.k;                 // routed row capacity
   const int64_t Rh = Rk + static_cast<int64_t>(L.S) * L.T;
@@ -368,8 +485,8 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   // ---------------- gate_up: [rows, H] x [2I, H]^T -> SwiGLU -> h [rows, I]
   GemmParams g{};
   bool ok = encode_a(&g.tmA[0], x_perm, Rk, L.H) && encode_a(&g.tmA[1], x, L.T, L.H) &&
-            encode_b(&g.tmB[0], w_gate_up, L.E, 2 * L.I, L.H);
-  if (ok && L.S > 0) ok = encode_b(&g.tmB[1], ws_gate_up, L.S, 2 * L.I, L.H);
+            encode_b(&g.tmB[0], w_gate_up, L.E, 2 * L.I, L.H, BN);
+  if (ok && L.S > 0) ok = encode_b(&g.tmB[1], ws_gate_up, L.S, 2 * L.I, L.H, BN);
   else g.tmB[1] = g.tmB[0];
   if (!ok) { *map_error = true; return cudaErrorInvalidValue; }
   g.offsets = offsets; g.perm_slot = perm_slot; g.topk_w = topk_w; g.gamma = gamma;
@@ -379,14 +496,15 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   g.T = L.T; g.a1_base = 0; g.a1_stride = 0;
   g.E = L.E; g.S = L.S; g.K = L.H; g.N = 2 * L.I; g.ld_out = L.I;
   g.rows_cap = static_cast<int>(Rk);
+  g.ksplit = 1;
   cudaError_t e = launch_mode<kGateUp>(g, num_sms, stream);
   if (e != cudaSuccess) return e;
 
-  // ---------------- down: h [rows, I] x [H, I]^T -> y [rows, H]
+  // ---------------- down: h [rows, I] x [H, I]^T -> y [rows, H] (fp32)
   GemmParams d{};
-  ok = encode_a(&d.tmA[0], h, Rh, L.I) && encode_b(&d.tmB[0], w_down, L.E, L.H, L.I);
+  ok = encode_a(&d.tmA[0], h, Rh, L.I) && encode_b(&d.tmB[0], w_down, L.E, L.H, L.I, BN);
   d.tmA[1] = d.tmA[0];
-  if (ok && L.S > 0) ok = encode_b(&d.tmB[1], ws_down, L.S, L.H, L.I);
+  if (ok && L.S > 0) ok = encode_b(&d.tmB[1], ws_down, L.S, L.H, L.I, BN);
   else d.tmB[1] = d.tmB[0];
   if (!ok) { *map_error = true; return cudaErrorInvalidValue; }
   d.offsets = offsets; d.perm_slot = perm_slot; d.topk_w = topk_w; d.gamma = gamma;
@@ -396,7 +514,38 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   d.T = L.T; d.a1_base = Rk; d.a1_stride = L.T;
   d.E = L.E; d.S = L.S; d.K = L.I; d.N = L.H; d.ld_out = L.H;
   d.rows_cap = static_cast<int>(Rk);
+  d.ksplit = 1;
   return launch_mode<kDown>(d, num_sms, stream);
 }
+
+// Router logits on the tensor cores: ksplit partial sums z_s[T, ld_z] (fp32,
+// ld_z = E+S rounded up to 32, consecutive in `logits`) with
+// sum_s z_s = x [T, H] @ (W0 + W1 + W2)^T, W_p the bf16 parts [3][E+S][H].
+cudaError_t launch_router_logits_sm100(const Layer& L, const void* x, const void* w_parts,
+                                       float* logits, int ld_z, int ksplit, int32_t* status,
+                                       int num_sms, cudaStream_t stream, bool* map_error) {
+  using namespace sm100;
+  *map_error = false;
+  const int NE = L.E + L.S;
+  GemmParams r{};
+  const bool ok = encode_a(&r.tmA[0], x, L.T, L.H) &&
+                  encode_b(&r.tmB[0], w_parts, 3, NE, L.H, Tile<kRouter>::BN);
+  if (!ok) { *map_error = true; return cudaErrorInvalidValue; }
+  r.tmA[1] = r.tmA[0];
+  r.tmB[1] = r.tmB[0];
+  r.offsets = nullptr; r.perm_slot = nullptr; r.topk_w = nullptr; r.gamma = nullptr;
+  r.out[0] = logits;
+  r.out[1] = logits;
+  r.status = status;
+  r.T = L.T; r.a1_base = 0; r.a1_stride = 0;
+  r.E = 0; r.S = 1;                 // one group: all T tokens
+  r.K = L.H; r.N = NE; r.ld_out = ld_z;
+  r.rows_cap = 0;
+  r.ksplit = ksplit;
+  r.split_stride = L.T * static_cast<int64_t>(ld_z);
+  return launch_mode<kRouter>(r, num_sms, stream);
+}
+
+int sm100_gemm_max_smem(int E, int S) { return sm100::smem_bytes<sm100::kGateUp>(E, S); }
 
 }  // namespace moe

@@ -56,9 +56,13 @@ __device__ inline void build_tile_prefix(const int32_t* __restrict__ offsets, in
                                          int64_t T, int BM, int n_tiles, int rows_cap, int* s_off,
                                          int* s_tile, int* bad) {
   const int lane = threadIdx.x & 31;
-  for (int i = lane; i <= E; i += 32) s_off[i] = offsets[i];
+  if (E == 0) {
+    if (lane == 0) s_off[0] = 0;
+  } else {
+    for (int i = lane; i <= E; i += 32) s_off[i] = offsets[i];
+  }
   __syncwarp();
-  if (lane == 0) {
+  if (lane == 0 && E > 0) {
     // clamp to a monotone sequence inside [0, rows_cap]
     int prev = 0;
     for (int i = 0; i <= E; ++i) {

@@ -20,10 +20,13 @@ struct Layer {
 int device_sm_count();
 moe_status_t validate_desc(const moe_layer_desc_t* d, Layer* L);
 
-// router.cu
+// router.cu (logits row stride `ld` = E+S rounded up to 32)
+cudaError_t launch_router_split(const Layer& L, const float* w_router, void* w_parts,
+                                int num_sms, cudaStream_t stream);
 cudaError_t launch_router_logits(const Layer& L, const void* x, const float* w_router,
-                                 float* logits, cudaStream_t stream);
-cudaError_t launch_router_topk(const Layer& L, const float* logits, const float* corr_bias,
+                                 float* logits, int ld, cudaStream_t stream);
+cudaError_t launch_router_topk(const Layer& L, const float* logits, int ld, int ksplit,
+                               const float* corr_bias,
                                float* topk_w, int32_t* topk_idx, float* shared_gamma,
                                cudaStream_t stream);
 
@@ -42,6 +45,9 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
                                    int32_t* status, int num_sms, cudaStream_t stream,
                                    bool* map_error);
 int sm100_gemm_max_smem(int E, int S);
+cudaError_t launch_router_logits_sm100(const Layer& L, const void* x, const void* w_parts,
+                                       float* logits, int ld_z, int ksplit, int32_t* status,
+                                       int num_sms, cudaStream_t stream, bool* map_error);
 
 // grouped_gemm_simt.cu (fp32, CUDA cores)
 cudaError_t launch_expert_ffn_f32(const Layer& L, const void* x, const void* x_perm,

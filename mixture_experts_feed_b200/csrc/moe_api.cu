@@ -20,9 +20,25 @@ constexpr size_t kRegionAlign = 1024;
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct WsLayout {
-  size_t status, logits, counts, topk_w, topk_idx, gamma, offsets, perm_slot, inv_perm, x_perm,
+  size_t status, logits, wparts, counts, topk_w, topk_idx, gamma, offsets, perm_slot, inv_perm, x_perm,
       h, y_routed, y_shared, total;
 };
+
+// Row stride of the router logits: E+S rounded up to 32 (whole 32-column
+// chunks of the tensor-core epilogue stay inside a row).
+int logits_ld(const Layer& L) { return (L.E + L.S + 31) / 32 * 32; }
+
+// K splits of the tensor-core router: enough CTAs for a B200's 148 SMs when
+// T is small, at most 32.  A function of the layer shape only, so the
+// partial-sum order (and every result) is the same on any device.
+int router_ksplit(const Layer& L) {
+  if (L.dtype != MOE_BF16) return 1;
+  const int64_t tiles = (L.T + 127) / 128 * ((L.E + L.S + 127) / 128);
+  int64_t ks = 148 / (tiles > 0 ? tiles : 1);
+  if (ks < 1) ks = 1;
+  if (ks > 32) ks = 32;
+  return static_cast<int>(ks);
+}
 
 WsLayout ws_layout(const Layer& L) {
   WsLayout w{};
@@ -37,7 +53,8 @@ WsLayout ws_layout(const Layer& L) {
   const size_t Rk = T * L.k;
   const size_t Rh = Rk + T * L.S;
   w.status = take(kStatusBytes);
-  w.logits = take(T * (L.E + L.S) * 4);
+  w.logits = take(T * logits_ld(L) * 4 * router_ksplit(L));
+  w.wparts = take(L.dtype == MOE_BF16 ? 3 * static_cast<size_t>(L.E + L.S) * L.H * 2 : 0);
   w.counts = take(static_cast<size_t>(L.E) * 4);
   w.topk_w = take(Rk * 4);
   w.topk_idx = take(Rk * 4);
@@ -126,8 +143,22 @@ moe_status_t route_impl(const Layer& L, const void* x, const float* w_router,
                         float* shared_gamma, void* ws, cudaStream_t stream) {
   const WsLayout w = ws_layout(L);
   float* logits = region<float>(ws, w.logits);
-  MOE_TRY(cuda_status(launch_router_logits(L, x, w_router, logits, stream)));
-  return cuda_status(launch_router_topk(L, logits, corr_bias, topk_w, topk_idx, shared_gamma, stream));
+  const int ld = logits_ld(L);
+  const int ksplit = router_ksplit(L);
+  if (L.dtype == MOE_BF16) {
+    void* parts = region<void>(ws, w.wparts);
+    MOE_TRY(cuda_status(launch_router_split(L, w_router, parts, num_sms(), stream)));
+    bool map_error = false;
+    const cudaError_t e = launch_router_logits_sm100(L, x, parts, logits, ld, ksplit,
+                                                     region<int32_t>(ws, w.status), num_sms(),
+                                                     stream, &map_error);
+    if (map_error) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(cuda_status(e));
+  } else {
+    MOE_TRY(cuda_status(launch_router_logits(L, x, w_router, logits, ld, stream)));
+  }
+  return cuda_status(launch_router_topk(L, logits, ld, ksplit, corr_bias, topk_w, topk_idx,
+                                        shared_gamma, stream));
 }
 
 moe_status_t permute_impl(const Layer& L, const int32_t* topk_idx, const uint8_t* pad,
@@ -296,9 +327,9 @@ moe_status_t moe_forward(const moe_layer_desc_t* desc, const void* x, const floa
 int32_t moe_forward_kernel_count(const moe_layer_desc_t* desc) {
   Layer L;
   if (check_desc(desc, &L) != MOE_OK || L.T == 0) return 0;
-  // router: logits + top-k; permute: count, scan, compact, gather;
-  // experts: gate_up + down; combine.
-  return 2 + 4 + 2 + 1;
+  // router: (bf16: split + tensor-core logits | fp32: logits) + top-k;
+  // permute: count, scan, compact, gather; experts: gate_up + down; combine.
+  return (L.dtype == MOE_BF16 ? 3 : 2) + 4 + 2 + 1;
 }
 
 const char* moe_status_string(moe_status_t status) {

@@ -1,11 +1,16 @@
 // InklingGate on the GPU (Inkling layers page, InklingGate docstring and
 // InklingCorrectionBias.forward).
 //
-// Two kernels:
-//   router_logits_kernel  z[t, e] = sum_h x[t, h] * Wr[e, h] in fp32 (the
-//                         gate runs in fp32: gate_precision=torch.float32),
-//                         for all E routed + S shared rows of the gate bank.
-//                         Tiled SIMT fp32 GEMM (64 tokens x 64 rows x 32 K).
+// Kernels:
+//   router_split_kernel   (bf16 layers) splits the fp32 gate bank exactly into
+//                         three bf16 parts W = W0 + W1 + W2 (8 + 8 + 8
+//                         significand bits), so that the logits can run on the
+//                         tensor cores with every product exact in fp32
+//                         (grouped_gemm_sm100.cu, kRouter).
+//   router_logits_kernel  (fp32 layers) z[t, e] = sum_h x[t, h] * Wr[e, h] in
+//                         fp32 FFMA, tiled 64 tokens x 64 rows x 32 K.
+//   Both give fp32 logits for all E routed + S shared rows of the gate bank
+//   (the gate runs in fp32: gate_precision=torch.float32).
 //   router_topk_kernel    one warp per token: selection score
 //                         sigmoid(z) + bias over the routed rows, k rounds of
 //                         a warp-shuffle argmax (ties to the lower expert id),
@@ -13,6 +18,8 @@
 //                         log-sigmoid(z) of [selected ++ shared] equals
 //                         sigmoid(z_i) / sum sigmoid(z), which is what the
 //                         kernel evaluates, times route_scale*global_scale.
+#include <algorithm>
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -44,10 +51,28 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
   }
 }
 
+// Exact three-way bf16 split of fp32 values: each part is the round-to-
+// nearest bf16 of what the previous parts left over; the residual after
+// three parts is zero for every finite fp32 input of normal range.
+__global__ void router_split_kernel(const float* __restrict__ w, __nv_bfloat16* __restrict__ parts,
+                                    int64_t n) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const float v = w[i];
+    const __nv_bfloat16 p0 = __float2bfloat16_rn(v);
+    const float r0 = v - __bfloat162float(p0);
+    const __nv_bfloat16 p1 = __float2bfloat16_rn(r0);
+    const float r1 = r0 - __bfloat162float(p1);
+    parts[i] = p0;
+    parts[n + i] = p1;
+    parts[2 * n + i] = __float2bfloat16_rn(r1);
+  }
+}
+
 template <typename TX>
 __global__ void __launch_bounds__(RL_THREADS)
     router_logits_kernel(const TX* __restrict__ x, const float* __restrict__ w,
-                         float* __restrict__ z, int64_t T, int H, int NE) {
+                         float* __restrict__ z, int64_t T, int H, int NE, int ld) {
   __shared__ __align__(16) float As[RL_BK][RL_BM + 4];
   __shared__ __align__(16) float Bs[RL_BK][RL_BN + 4];
   const int tid = threadIdx.x;
@@ -103,7 +128,7 @@ __global__ void __launch_bounds__(RL_THREADS)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int col = n0 + tx * 4 + j;
-      if (col < NE) z[row * NE + col] = acc[i][j];
+      if (col < NE) z[row * ld + col] = acc[i][j];
     }
   }
 }
@@ -115,21 +140,28 @@ constexpr int TK_WARPS = 8;
 // PL: routed scores held per lane (E <= 32 * PL).
 template <int PL>
 __global__ void __launch_bounds__(TK_WARPS * 32)
-    router_topk_kernel(const float* __restrict__ z, const float* __restrict__ bias, int64_t T,
-                       int E, int k, int S, float scale, float* __restrict__ topk_w,
-                       int32_t* __restrict__ topk_idx, float* __restrict__ gamma) {
+    router_topk_kernel(const float* __restrict__ z, int ld, int ksplit,
+                       const float* __restrict__ bias, int64_t T, int E, int k, int S, float scale,
+                       float* __restrict__ topk_w, int32_t* __restrict__ topk_idx,
+                       float* __restrict__ gamma) {
   __shared__ int s_chosen[TK_WARPS][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * TK_WARPS + warp;
   if (t >= T) return;
-  const int NE = E + S;
-  const float* zt = z + t * NE;
+  const float* zt = z + t * ld;
+  const int64_t split = T * static_cast<int64_t>(ld);
+  // logit of row e: the K-split partial sums added in split order
+  auto logit = [&](int e) {
+    float v = zt[e];
+    for (int s2 = 1; s2 < ksplit; ++s2) v += zt[s2 * split + e];
+    return v;
+  };
 
   float sel[PL];
 #pragma unroll
   for (int i = 0; i < PL; ++i) {
     const int e = lane + 32 * i;
-    const float v = e < E ? sigmoidf_(zt[e]) + bias[e] : -INFINITY;
+    const float v = e < E ? sigmoidf_(logit(e)) + bias[e] : -INFINITY;
     sel[i] = isnan(v) ? -INFINITY : v;   // a NaN score ranks last, never breaks the argmax
   }
   uint32_t taken = 0;
@@ -162,8 +194,8 @@ __global__ void __launch_bounds__(TK_WARPS * 32)
   }
   __syncwarp();
   float sg = 0.0f;
-  if (lane < k) sg = sigmoidf_(zt[s_chosen[warp][lane]]);
-  else if (lane < k + S) sg = sigmoidf_(zt[E + (lane - k)]);
+  if (lane < k) sg = sigmoidf_(logit(s_chosen[warp][lane]));
+  else if (lane < k + S) sg = sigmoidf_(logit(E + (lane - k)));
   float sum = sg;
 #pragma unroll
   for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
@@ -178,27 +210,36 @@ __global__ void __launch_bounds__(TK_WARPS * 32)
 
 }  // namespace
 
+cudaError_t launch_router_split(const Layer& L, const float* w_router, void* w_parts,
+                                int num_sms, cudaStream_t stream) {
+  const int64_t n = static_cast<int64_t>(L.E + L.S) * L.H;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ceil_div(n, 256), num_sms * 8));
+  router_split_kernel<<<grid, 256, 0, stream>>>(w_router, static_cast<__nv_bfloat16*>(w_parts), n);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_router_logits(const Layer& L, const void* x, const float* w_router,
-                                 float* logits, cudaStream_t stream) {
+                                 float* logits, int ld, cudaStream_t stream) {
   const int NE = L.E + L.S;
   dim3 grid(static_cast<unsigned>(ceil_div(L.T, RL_BM)), static_cast<unsigned>(ceil_div(NE, RL_BN)));
   if (L.dtype == MOE_BF16)
     router_logits_kernel<__nv_bfloat16><<<grid, RL_THREADS, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(x), w_router, logits, L.T, L.H, NE);
+        static_cast<const __nv_bfloat16*>(x), w_router, logits, L.T, L.H, NE, ld);
   else
     router_logits_kernel<float><<<grid, RL_THREADS, 0, stream>>>(static_cast<const float*>(x),
-                                                                 w_router, logits, L.T, L.H, NE);
+                                                                 w_router, logits, L.T, L.H, NE, ld);
   return cudaGetLastError();
 }
 
-cudaError_t launch_router_topk(const Layer& L, const float* logits, const float* corr_bias,
-                               float* topk_w, int32_t* topk_idx, float* shared_gamma,
-                               cudaStream_t stream) {
+cudaError_t launch_router_topk(const Layer& L, const float* logits, int ld, int ksplit,
+                               const float* corr_bias, float* topk_w, int32_t* topk_idx,
+                               float* shared_gamma, cudaStream_t stream) {
   const unsigned grid = static_cast<unsigned>(ceil_div(L.T, TK_WARPS));
   const float scale = L.route_scale * L.global_scale;
   const int pl = static_cast<int>(ceil_div(L.E, 32));
 #define MOE_TOPK(PLV)                                                                         \
-  router_topk_kernel<PLV><<<grid, TK_WARPS * 32, 0, stream>>>(logits, corr_bias, L.T, L.E, L.k, \
+  router_topk_kernel<PLV><<<grid, TK_WARPS * 32, 0, stream>>>(logits, ld, ksplit, corr_bias, L.T, \
+                                                              L.E, L.k,                        \
                                                               L.S, scale, topk_w, topk_idx,     \
                                                               shared_gamma)
   if (pl <= 1) MOE_TOPK(1);

@@ -8,9 +8,9 @@ no routing, no activation, no matrix product.
 Shapes follow the pages' statement of the layer (NeMo AutoModel Inkling
 ``layers`` page: ``InklingGate``, ``InklingSharedExperts``, ``inkling_swiglu``;
 ``configuration`` page: ``InklingTextConfig``).  Weight orientation is the
-checkpoint's ``[out_features, in_features]`` form, the one of which the pages
-say distributed loading only needs transpose views (``InklingSharedExperts``
-docstring):
+checkpoint's ``[out_features, in_features]`` form: the pages keep the fused
+projection in the checkpoint's layout so that loading it takes no more than a
+transposed view (``InklingSharedExperts`` docstring):
 
   x           [T, H]        activations, N(0, 1)
   w_router    [E+S, H] f32  gate weight bank: E routed rows then S shared rows,

@@ -32,7 +32,7 @@ log-sigmoid applies to the whole concatenated vector, shared logits included;
 the gammas are scaled like the routed weights; ties in the selection score go
 to the lower expert index and the k chosen experts are returned in descending
 score order; weights are stored ``[out, in]`` (the checkpoint form that needs
-only transpose views); the router has no norm; padded tokens take no routed
+no more than a transposed view); the router has no norm; padded tokens take no routed
 rows but still receive the shared experts.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
@@ -131,7 +131,7 @@ def gate(x, w_router, corr_bias, n_routed: int, top_k: int, n_shared: int,
 # ------------------------------------------------------------------ experts
 def swiglu_interleaved(G: torch.Tensor, routing_weights: torch.Tensor) -> torch.Tensor:
     """``inkling_swiglu``: last axis is [g0, u0, g1, u1, ...]; ``::2`` is gate,
-    ``1::2`` is up; the activated output silu(g) * u is scaled by the routing
+    ``1::2`` is up; silu(g) * u is multiplied by the per-row routing
     weights (broadcast to ``[..., intermediate]``).  ``hidden_act='silu'``
     (``InklingTextConfig``): silu(g) = g * sigmoid(g).
     """
@@ -163,7 +163,7 @@ def routed_experts(x64: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tens
                    w_gate_up, w_down, padding_mask: Optional[torch.Tensor] = None) -> torch.Tensor:
     """y[t, j] = expert_mlp of token t through expert topk_idx[t, j] with
     weight topk_w[t, j]; padded tokens get no routed rows (``InklingMoE.forward``:
-    padded tokens are excluded from routed-expert dispatch).  Rows that chose
+    padded tokens never reach a routed expert).  Rows that chose
     the same expert are evaluated together; that grouping changes nothing but
     float64 rounding."""
     T, k = topk_idx.shape

@@ -55,7 +55,7 @@ def test_workspace_size_covers_intermediates(w):
     Rk = w.T * w.k
     need = el * (Rk * w.H + (Rk + w.S * w.T) * w.I) + 4 * (Rk + w.S * w.T) * w.H
     assert n >= need
-    assert moe.forward_kernel_count(L) == 9
+    assert moe.forward_kernel_count(L) == (10 if w.dtype == "bf16" else 9)
 
 
 def _status(fn, *args):
