@@ -41,7 +41,7 @@ __global__ void __launch_bounds__(SB_THREADS) grouped_gemm_simt_kernel(const Sim
   const int tid = threadIdx.x;
   if (tid == 0) s_bad = 0;
   __syncthreads();
-  if (tid < 32) build_tile_prefix(p.offsets, p.E, p.S, p.T, SB_M, n_tiles, p.rows_cap, s_off, s_tile, &s_bad);
+  if (tid < 32) build_tile_prefix(p.offsets, p.E, p.S, p.T, kAllTiles, SB_M, n_tiles, p.rows_cap, s_off, s_tile, &s_bad);
   __syncthreads();
   if (tid == 0 && s_bad) record_status(p.status, DEV_BAD_ROW);
   const int total = s_tile[G];
@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(SB_THREADS) grouped_gemm_simt_kernel(const Sim
 
   for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
     int g, m, n;
-    decode_tile(tile, s_tile, G, s_off, p.E, p.T, SB_M, g, m, n);
+    decode_tile(tile, s_tile, G, s_off, p.E, p.T, kAllTiles, SB_M, g, m, n);
     const GroupInfo gi = group_info(g, s_off, p.E, p.T, p.a1_base, p.a1_stride);
     const float* A = p.A[gi.src];
     const float* B = p.B[gi.src] + static_cast<int64_t>(gi.b_idx) * p.N * p.K;

@@ -16,22 +16,30 @@
 //            into three bf16 parts (W = W0 + W1 + W2) so that every product
 //            is exact.  The tensor-core accumulator loses about one fp32 ulp
 //            of its own magnitude per MMA step (measured: 5.7e-5 in z over a
-//            3 x 6144 chain), so each accumulation chain is kept to one
-//            64-deep K block: the MMA writes a fresh block sum, and the
-//            epilogue warps add the block sums in fp32 registers with
+//            3 x 6144 chain), so each accumulation chain is kept to two
+//            64-deep K blocks: the MMA writes a fresh chain sum, and the
+//            epilogue warps add the chain sums in fp32 registers with
 //            round-to-nearest adds.  fp32 logits out.  One group (all T
 //            tokens), N = E + S, 128-column tiles.
 //
-// Roles (192 threads, one CTA per SM):
-//   warp 0      TMA producer: A tile [128 rows x 64 K] and B tile
-//               [BN rows x 64 K] per stage, 128-byte swizzle, 4 stages.
-//   warp 1      TMEM allocator and MMA issuer (one thread): 4 x
-//               tcgen05.mma M128 N<=BN K16 per stage into one of two
-//               accumulators (2 x BN TMEM columns).
-//   warps 2..5  epilogue: tcgen05.ld the accumulator rows (warp w reads TMEM
-//               lanes 32*(w%4) .. +31), fused math, global stores.
+// The expert modes run on CTA pairs (clusters of two SMs, tcgen05
+// cta_group::2): a pair computes a 256-row x 256-column tile with M=256
+// MMAs; each CTA loads its own 128 A rows and half of the 256 B rows, so the
+// bytes each SM pulls per MMA drop by a third against one-SM 128 x 256 tiles
+// and six pipeline stages fit in shared memory.  The router runs one CTA per
+// tile (M=128).
+//
+// Roles (192 threads per CTA, one CTA per SM):
+//   warp 0      TMA producer: per stage, this CTA's A tile [128 rows x 64 K]
+//               and its B rows [BN/2 (pairs) or BN rows x 64 K], 128-byte
+//               swizzle; pair loads signal the rank-0 CTA's barrier.
+//   warp 1      TMEM allocator and (rank-0 CTA only) MMA issuer, one thread:
+//               4 x tcgen05.mma K16 per stage into one of two accumulators
+//               (2 x BN TMEM columns in each CTA).
+//   warps 2..5  epilogue: tcgen05.ld this CTA's accumulator rows (warp w
+//               reads TMEM lanes 32*(w%4) .. +31), fused math, global stores.
 // The two accumulators let the epilogue of one tile (or, for kRouter, one K
-// block) overlap the MMAs of the next.  All waits are bounded
+// chain) overlap the MMAs of the next.  All waits are bounded
 // (sm100_ptx.cuh); on a timeout every role stops, the status word records it
 // and TMEM is released.  No TMA load uses cluster multicast.
 #include <cuda.h>
@@ -46,19 +54,28 @@
 namespace moe {
 namespace sm100 {
 
-constexpr int BM = 128;
+constexpr int BM = 128;          // A rows per CTA
 constexpr int BK = 64;
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int NUM_THREADS = 192;
+// kRouter: K blocks per tensor-core accumulation chain (128-deep chains)
+constexpr int ROUTER_CHAIN = 2;
 
 enum Mode { kGateUp = 0, kDown = 1, kRouter = 2 };
 
-template <int MODE> struct Tile {
-  static constexpr int BN = MODE == kRouter ? 128 : 256;   // accumulator columns
-  static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr uint32_t TMEM_COLS = 2 * BN;            // two accumulators
-  static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+template <int MODE, bool PAIR_> struct Tile {
+  static constexpr bool PAIR = PAIR_;                       // CTA-pair (M=256) MMAs
+  // which m-tiles of each group the launch covers (grouping.cuh)
+  static constexpr int SET = PAIR ? kPairs : (MODE == kRouter ? kAllTiles : kSingles);
+  static constexpr int BN = MODE == kRouter ? 128 : 256;    // MMA N = accumulator columns
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;         // B rows one CTA loads
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
+  static constexpr int B_BOX = 128;                         // rows per B tensor-map box
+  static constexpr int B_LOADS = B_ROWS / B_BOX;            // boxes per stage
+  static constexpr int STAGES = PAIR ? 6 : 4;
+  static constexpr int TILE_M = PAIR ? 2 * BM : BM;         // rows per tile
+  static constexpr uint32_t TMEM_COLS = 2 * BN;             // two accumulators
+  static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, BN);
 };
 
 struct alignas(64) GemmParams {
@@ -84,10 +101,11 @@ struct alignas(64) GemmParams {
 constexpr int STAGE_LD = 36;
 constexpr int STAGE_WARP_BYTES = 32 * STAGE_LD * 4;
 
-template <int MODE> struct SmemLayout {
+template <int MODE, bool PAIR> struct SmemLayout {
+  static constexpr int STAGES = Tile<MODE, PAIR>::STAGES;
   static constexpr int kA = 0;
   static constexpr int kB = STAGES * A_BYTES;
-  static constexpr int kStage = kB + STAGES * Tile<MODE>::B_BYTES;   // 4 x STAGE_WARP_BYTES
+  static constexpr int kStage = kB + STAGES * Tile<MODE, PAIR>::B_BYTES;   // 4 x STAGE_WARP_BYTES
   static constexpr int kBars = kStage + 4 * STAGE_WARP_BYTES;
   // full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
   static constexpr int kNumBars = 2 * STAGES + 5;
@@ -95,9 +113,9 @@ template <int MODE> struct SmemLayout {
   static constexpr int kTables = kMisc + 16;
 };
 
-template <int MODE>
+template <int MODE, bool PAIR>
 __host__ __device__ inline int smem_bytes(int E, int S) {
-  return 1024 /* alignment slack */ + SmemLayout<MODE>::kTables + 4 * ((E + 1) + (E + S + 1));
+  return 1024 /* alignment slack */ + SmemLayout<MODE, PAIR>::kTables + 4 * ((E + 1) + (E + S + 1));
 }
 
 // Write one warp's 32 rows x 32 fp32 columns through the staging tile so that
@@ -122,12 +140,14 @@ __device__ __forceinline__ void store_rows_f32(float* st, const uint32_t (&v)[32
   __syncwarp();
 }
 
-template <int MODE>
+template <int MODE, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
-  using TL = Tile<MODE>;
-  using SL = SmemLayout<MODE>;
+  using TL = Tile<MODE, PAIR>;
+  using SL = SmemLayout<MODE, PAIR>;
   constexpr int BN = TL::BN;
+  constexpr int STAGES = TL::STAGES;
+  constexpr int SET = TL::SET;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -147,6 +167,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0;     // 0 = the pair's MMA issuer
+  const bool leader = rank == 0;
+  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   const int G = p.E + p.S;
   // kRouter folds its K splits into the n-tile index: nv = n * ksplit + ks
   const int ksplit = MODE == kRouter ? p.ksplit : 1;
@@ -164,7 +188,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       for (int i = 0; i < 2; ++i) {
         mbar_init(&tfull[i], 1);
-        mbar_init(&tempty[i], 4);   // one arrive per epilogue warp
+        mbar_init(&tempty[i], PAIR ? 8 : 4);   // one arrive per epilogue warp (of both CTAs)
       }
       mbar_init(drain, 1);
       *s_abort = 0;
@@ -178,13 +202,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    tmem_alloc(s_tmem, TL::TMEM_COLS);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(s_tmem, TL::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(s_tmem, TL::TMEM_COLS);
+      tmem_relinquish();
+    }
   } else if (warp == 2) {
-    build_tile_prefix(p.offsets, p.E, p.S, p.T, BM, n_tiles, p.rows_cap, s_off, s_tile, s_bad);
+    build_tile_prefix(p.offsets, p.E, p.S, p.T, SET, BM, n_tiles, p.rows_cap, s_off, s_tile, s_bad);
   }
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync();   // both CTAs' barriers exist before any cross-CTA signal
   tc_fence_after();
 
   const uint32_t tmem_base = *s_tmem;
@@ -198,58 +228,79 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int last_parity[STAGES];
 #pragma unroll
     for (int i = 0; i < STAGES; ++i) last_parity[i] = -1;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+    for (int tile = unit; tile < total_tiles; tile += units) {
       int g, m, nv;
-      decode_tile(tile, s_tile, G, s_off, p.E, p.T, BM, g, m, nv);
+      decode_tile(tile, s_tile, G, s_off, p.E, p.T, SET, BM, g, m, nv);
       const int n = nv / ksplit, ks = nv - n * ksplit;
       const GroupInfo gi = group_info(g, s_off, p.E, p.T, p.a1_base, p.a1_stride);
       const void* tmA = &p.tmA[gi.src];
       const void* tmB = &p.tmB[gi.src];
-      const int a_row = static_cast<int>(gi.a_row0) + m * BM;
+      const int a_row = static_cast<int>(gi.a_row0) + tile_first_row(m, gi.rows, SET, BM) +
+                        static_cast<int>(rank) * BM;
+      // pairs: this CTA's half of the tile's (possibly narrowed) N range
+      const int n_pad = (min(BN, p.N - n * BN) + 31) & ~31;
+      const int b_row = n * BN + (PAIR ? static_cast<int>(rank) * (n_pad >> 1) : 0);
       bool ok = true;
       for (int kt = kt_begin(ks); kt < kt_begin(ks + 1); ++kt) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, s_abort, p.status)) { ok = false; break; }
         // router: part 2 (smallest) first, then 1, then 0
         const int kb = MODE == kRouter ? kt % k_blocks : kt;
         const int slice = MODE == kRouter ? 2 - kt / k_blocks : gi.b_idx;
-        mbar_arrive_expect_tx(&full[stage], A_BYTES + TL::B_BYTES);
-        tma_load_2d(sA + stage * A_BYTES, tmA, &full[stage], kb * BK, a_row);
-        tma_load_3d(sB + stage * TL::B_BYTES, tmB, &full[stage], kb * BK, n * BN, slice);
+        if (PAIR) {
+          // both CTAs' bytes complete on the rank-0 CTA's barrier
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (A_BYTES + TL::B_BYTES));
+          const uint32_t bar0 = mapa_shared(&full[stage], 0);
+          tma_load_2d_pair(sA + stage * A_BYTES, tmA, bar0, kb * BK, a_row);
+          tma_load_3d_pair(sB + stage * TL::B_BYTES, tmB, bar0, kb * BK, b_row, slice);
+        } else {
+          mbar_arrive_expect_tx(&full[stage], A_BYTES + TL::B_BYTES);
+          tma_load_2d(sA + stage * A_BYTES, tmA, &full[stage], kb * BK, a_row);
+#pragma unroll
+          for (int i = 0; i < TL::B_LOADS; ++i)
+            tma_load_3d(sB + stage * TL::B_BYTES + i * (TL::B_BOX * BK * 2), tmB, &full[stage],
+                        kb * BK, b_row + i * TL::B_BOX, slice);
+        }
         last_parity[stage] = static_cast<int>(phase);
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
       if (!ok) break;
     }
     // Wait (bounded) until the last load issued on every stage has landed,
-    // so that no copy still writes shared memory when the block exits.
+    // so that no copy still writes shared memory when the block exits.  A
+    // pair's loads all complete on the rank-0 CTA's barriers; the other CTA
+    // is covered by the cluster barrier at the end.
     const uint64_t t0 = globaltimer_ns();
-    for (int i = 0; i < STAGES; ++i) {
+    for (int i = 0; i < STAGES && leader; ++i) {
       if (last_parity[i] < 0) continue;
       while (!mbar_try_wait(&full[i], static_cast<uint32_t>(last_parity[i]))) {
         if (globaltimer_ns() - t0 > kWaitLimitNs) { record_status(p.status, DEV_WAIT_TIMEOUT); break; }
       }
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1 && lane == 0 && leader) {
     // ------------------------------------------------------- MMA issuer
     int stage = 0;
     uint32_t phase = 0;
     int it = 0;   // accumulator hand-offs so far (tiles, or K blocks for kRouter)
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+    for (int tile = unit; tile < total_tiles && ok; tile += units) {
       int g, m, nv;
-      decode_tile(tile, s_tile, G, s_off, p.E, p.T, BM, g, m, nv);
+      decode_tile(tile, s_tile, G, s_off, p.E, p.T, SET, BM, g, m, nv);
       const int n = nv / ksplit, ks = nv - n * ksplit;
-      // the last n-tile of a ragged N runs a narrower MMA (N multiple of 16)
+      // the last n-tile of a ragged N runs a narrower MMA (N multiple of 32)
       const int n_here = min(BN, p.N - n * BN);
-      const uint32_t idesc = n_here >= BN ? TL::IDESC : idesc_bf16_f32(BM, (n_here + 15) & ~15);
+      const uint32_t idesc = n_here >= BN ? TL::IDESC : idesc_bf16_f32(TL::TILE_M, (n_here + 31) & ~31);
       if (MODE != kRouter) {
         const int acc = it & 1;
         if (!mbar_wait(&tempty[acc], ((it >> 1) & 1) ^ 1u, s_abort, p.status)) { ok = false; break; }
         tc_fence_after();
       }
-      for (int kb = kt_begin(ks); kb < kt_begin(ks + 1); ++kb) {
+      const int kb0 = kt_begin(ks), kb1 = kt_begin(ks + 1);
+      for (int kb = kb0; kb < kb1; ++kb) {
         const int acc = it & 1;
-        if (MODE == kRouter) {   // one hand-off per K block
+        // router: a hand-off at the start of every chain of ROUTER_CHAIN K blocks
+        const bool chain_start = MODE == kRouter && (kb - kb0) % ROUTER_CHAIN == 0;
+        const bool chain_end = MODE == kRouter && ((kb - kb0) % ROUTER_CHAIN == ROUTER_CHAIN - 1 || kb + 1 == kb1);
+        if (chain_start) {
           if (!mbar_wait(&tempty[acc], ((it >> 1) & 1) ^ 1u, s_abort, p.status)) { ok = false; break; }
           tc_fence_after();
         }
@@ -261,26 +312,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           // +32 bytes per K=16 step inside the 128-byte swizzle atom
-          // router: a fresh block sum per K block; experts: accumulate over the tile
-          const bool accumulate = MODE == kRouter ? (kk != 0) : ((kb | kk) != 0);
-          mma_bf16_ss(d_tmem, adesc + static_cast<uint64_t>(2 * kk),
-                      bdesc + static_cast<uint64_t>(2 * kk), idesc, accumulate ? 1u : 0u);
+          // router: a fresh sum per chain; experts: accumulate over the tile
+          const bool accumulate = MODE == kRouter ? (!chain_start || kk != 0) : ((kb | kk) != 0);
+          if (PAIR)
+            mma_bf16_ss_pair(d_tmem, adesc + static_cast<uint64_t>(2 * kk),
+                             bdesc + static_cast<uint64_t>(2 * kk), idesc, accumulate ? 1u : 0u);
+          else
+            mma_bf16_ss(d_tmem, adesc + static_cast<uint64_t>(2 * kk),
+                        bdesc + static_cast<uint64_t>(2 * kk), idesc, accumulate ? 1u : 0u);
         }
-        mma_commit(&empty[stage]);
+        if (PAIR) mma_commit_pair(&empty[stage], 0x3);   // frees the stage in both CTAs
+        else mma_commit(&empty[stage]);
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        if (MODE == kRouter) {
+        if (chain_end) {
           mma_commit(&tfull[acc]);
           ++it;
         }
       }
       if (!ok) break;
       if (MODE != kRouter) {
-        mma_commit(&tfull[it & 1]);
+        if (PAIR) mma_commit_pair(&tfull[it & 1], 0x3);
+        else mma_commit(&tfull[it & 1]);
         ++it;
       }
     }
     // Every MMA this thread issued must be complete before TMEM is freed.
-    mma_commit(drain);
+    if (PAIR) mma_commit_pair(drain, 0x1);
+    else mma_commit(drain);
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(drain, 0)) {
       if (globaltimer_ns() - t0 > kWaitLimitNs) { record_status(p.status, DEV_WAIT_TIMEOUT); break; }
@@ -293,33 +351,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     int it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+    for (int tile = unit; tile < total_tiles && ok; tile += units) {
       int g, m, nv;
-      decode_tile(tile, s_tile, G, s_off, p.E, p.T, BM, g, m, nv);
+      decode_tile(tile, s_tile, G, s_off, p.E, p.T, SET, BM, g, m, nv);
       const int n = nv / ksplit, ks = nv - n * ksplit;
       const GroupInfo gi = group_info(g, s_off, p.E, p.T, p.a1_base, p.a1_stride);
-      const int r = m * BM + row_in_tile;          // row inside the group
+      const int row0 = tile_first_row(m, gi.rows, SET, BM) + static_cast<int>(rank) * BM;   // this CTA's first row
+      const int r = row0 + row_in_tile;            // row inside the group
       const bool valid = r < gi.rows;
       const int64_t out_row = gi.out_row0 + r;
-      const int rows_left = gi.rows - (m * BM + quarter * 32);   // rows of this warp's 32
+      const int rows_left = gi.rows - (row0 + quarter * 32);   // rows of this warp's 32
 
       if (MODE == kRouter) {
         // Sum the per-K-block accumulators in fp32 registers (round to nearest).
         float run[BN];
 #pragma unroll
         for (int i = 0; i < BN; ++i) run[i] = 0.0f;
-        for (int kb = kt_begin(ks); kb < kt_begin(ks + 1); ++kb) {
+        const int kb0 = kt_begin(ks), kb1 = kt_begin(ks + 1);
+        const int chains = (kb1 - kb0 + ROUTER_CHAIN - 1) / ROUTER_CHAIN;
+        for (int ch = 0; ch < chains; ++ch) {
           const int acc = it & 1;
           if (!mbar_wait(&tfull[acc], (it >> 1) & 1, s_abort, p.status)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < BN / 32; ++c) {
+          for (int c = 0; c < BN / 32; c += 2) {
             if (n * BN + c * 32 < p.N) {            // warp-uniform
-              uint32_t v[32];
+              uint32_t v[32], v2[32];
               tmem_ld_32x32b_x32(t_lane + static_cast<uint32_t>(acc * BN + c * 32), v);
+              const bool second = n * BN + (c + 1) * 32 < p.N;
+              if (second) tmem_ld_32x32b_x32(t_lane + static_cast<uint32_t>(acc * BN + (c + 1) * 32), v2);
               tmem_ld_wait();
 #pragma unroll
               for (int i = 0; i < 32; ++i) run[c * 32 + i] += __uint_as_float(v[i]);
+              if (second) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) run[(c + 1) * 32 + i] += __uint_as_float(v2[i]);
+              }
             }
           }
           tc_fence_before();
@@ -336,7 +403,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t v[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(run[c * 32 + i]);
-            store_rows_f32(st, v, lane, out, gi.out_row0 + m * BM + quarter * 32, rows_left,
+            store_rows_f32(st, v, lane, out, gi.out_row0 + row0 + quarter * 32, rows_left,
                            p.ld_out, col0);
           }
         }
@@ -387,21 +454,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
         } else {
           store_rows_f32(st, v, lane, static_cast<float*>(p.out[gi.src]),
-                         gi.out_row0 + m * BM + quarter * 32, rows_left, p.ld_out, col0);
+                         gi.out_row0 + row0 + quarter * 32, rows_left, p.ld_out, col0);
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) {
+        if (PAIR) mbar_arrive_cluster(mapa_shared(&tempty[acc], 0));   // the issuer's barrier
+        else mbar_arrive(&tempty[acc]);
+      }
       ++it;
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync();   // no MMA or signal of the pair is still in flight
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TL::TMEM_COLS);
+    if (PAIR) tmem_dealloc_pair(tmem_base, TL::TMEM_COLS);
+    else tmem_dealloc(tmem_base, TL::TMEM_COLS);
   }
 }
 
@@ -447,20 +519,35 @@ static bool encode_b(CUtensorMap* m, const void* base, int G, int N, int K, int 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE>
+template <int MODE, bool PAIR>
 static cudaError_t launch_mode(const GemmParams& p, int sms, cudaStream_t stream) {
-  const int smem = smem_bytes<MODE>(p.E, p.S);
+  const int smem = smem_bytes<MODE, PAIR>(p.E, p.S);
   static int configured_smem[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && configured_smem[dev] < smem) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, PAIR>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     configured_smem[dev] = smem;
   }
-  grouped_gemm_kernel<MODE><<<sms, NUM_THREADS, smem, stream>>>(p);
-  return cudaGetLastError();
+  if (!PAIR) {
+    grouped_gemm_kernel<MODE, PAIR><<<sms, NUM_THREADS, smem, stream>>>(p);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);   // whole pairs
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, PAIR>, p);
 }
 
 }  // namespace sm100
@@ -476,7 +563,9 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
                                    int32_t* status, int num_sms, cudaStream_t stream,
                                    bool* map_error) {
   using namespace sm100;
-  constexpr int BN = Tile<kGateUp>::BN;
+  // B maps: box of 128 rows = the half of a 256-row n-tile one CTA of a pair
+  // loads; the single-CTA odd-tile launch loads both halves (two boxes)
+  constexpr int BROWS = Tile<kGateUp, true>::B_BOX;
   *map_error = false;
   const int64_t Rk = L.T * L.k;                 // routed row capacity
   const int64_t Rh = Rk + static_cast<int64_t>(L.S) * L.T;
@@ -485,8 +574,8 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   // ---------------- gate_up: [rows, H] x [2I, H]^T -> SwiGLU -> h [rows, I]
   GemmParams g{};
   bool ok = encode_a(&g.tmA[0], x_perm, Rk, L.H) && encode_a(&g.tmA[1], x, L.T, L.H) &&
-            encode_b(&g.tmB[0], w_gate_up, L.E, 2 * L.I, L.H, BN);
-  if (ok && L.S > 0) ok = encode_b(&g.tmB[1], ws_gate_up, L.S, 2 * L.I, L.H, BN);
+            encode_b(&g.tmB[0], w_gate_up, L.E, 2 * L.I, L.H, BROWS);
+  if (ok && L.S > 0) ok = encode_b(&g.tmB[1], ws_gate_up, L.S, 2 * L.I, L.H, BROWS);
   else g.tmB[1] = g.tmB[0];
   if (!ok) { *map_error = true; return cudaErrorInvalidValue; }
   g.offsets = offsets; g.perm_slot = perm_slot; g.topk_w = topk_w; g.gamma = gamma;
@@ -497,14 +586,19 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   g.E = L.E; g.S = L.S; g.K = L.H; g.N = 2 * L.I; g.ld_out = L.I;
   g.rows_cap = static_cast<int>(Rk);
   g.ksplit = 1;
-  cudaError_t e = launch_mode<kGateUp>(g, num_sms, stream);
+  // large groups' m-tiles two by two on CTA pairs, then every other m-tile on
+  // single CTAs (grouping.cuh); with fewer than kPairMinTiles m-tiles of rows
+  // no group can pair and the pair launch is skipped
+  const bool pairs = L.T > static_cast<int64_t>(kPairMinTiles - 1) * BM;
+  cudaError_t e = pairs ? launch_mode<kGateUp, true>(g, num_sms, stream) : cudaSuccess;
+  if (e == cudaSuccess) e = launch_mode<kGateUp, false>(g, num_sms, stream);
   if (e != cudaSuccess) return e;
 
   // ---------------- down: h [rows, I] x [H, I]^T -> y [rows, H] (fp32)
   GemmParams d{};
-  ok = encode_a(&d.tmA[0], h, Rh, L.I) && encode_b(&d.tmB[0], w_down, L.E, L.H, L.I, BN);
+  ok = encode_a(&d.tmA[0], h, Rh, L.I) && encode_b(&d.tmB[0], w_down, L.E, L.H, L.I, BROWS);
   d.tmA[1] = d.tmA[0];
-  if (ok && L.S > 0) ok = encode_b(&d.tmB[1], ws_down, L.S, L.H, L.I, BN);
+  if (ok && L.S > 0) ok = encode_b(&d.tmB[1], ws_down, L.S, L.H, L.I, BROWS);
   else d.tmB[1] = d.tmB[0];
   if (!ok) { *map_error = true; return cudaErrorInvalidValue; }
   d.offsets = offsets; d.perm_slot = perm_slot; d.topk_w = topk_w; d.gamma = gamma;
@@ -515,7 +609,9 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   d.E = L.E; d.S = L.S; d.K = L.I; d.N = L.H; d.ld_out = L.H;
   d.rows_cap = static_cast<int>(Rk);
   d.ksplit = 1;
-  return launch_mode<kDown>(d, num_sms, stream);
+  e = pairs ? launch_mode<kDown, true>(d, num_sms, stream) : cudaSuccess;
+  if (e == cudaSuccess) e = launch_mode<kDown, false>(d, num_sms, stream);
+  return e;
 }
 
 // Router logits on the tensor cores: ksplit partial sums z_s[T, ld_z] (fp32,
@@ -529,7 +625,7 @@ cudaError_t launch_router_logits_sm100(const Layer& L, const void* x, const void
   const int NE = L.E + L.S;
   GemmParams r{};
   const bool ok = encode_a(&r.tmA[0], x, L.T, L.H) &&
-                  encode_b(&r.tmB[0], w_parts, 3, NE, L.H, Tile<kRouter>::BN);
+                  encode_b(&r.tmB[0], w_parts, 3, NE, L.H, Tile<kRouter, false>::B_BOX);
   if (!ok) { *map_error = true; return cudaErrorInvalidValue; }
   r.tmA[1] = r.tmA[0];
   r.tmB[1] = r.tmB[0];
@@ -543,9 +639,9 @@ cudaError_t launch_router_logits_sm100(const Layer& L, const void* x, const void
   r.rows_cap = 0;
   r.ksplit = ksplit;
   r.split_stride = L.T * static_cast<int64_t>(ld_z);
-  return launch_mode<kRouter>(r, num_sms, stream);
+  return launch_mode<kRouter, false>(r, num_sms, stream);
 }
 
-int sm100_gemm_max_smem(int E, int S) { return sm100::smem_bytes<sm100::kGateUp>(E, S); }
+int sm100_gemm_max_smem(int E, int S) { return sm100::smem_bytes<sm100::kGateUp, true>(E, S); }
 
 }  // namespace moe

@@ -11,11 +11,42 @@
 // Tiles are numbered group by group; inside a group, n-tile by n-tile, and
 // inside an n-tile, m-tile by m-tile (consecutive tiles share one weight
 // strip, so CTAs running together reuse it from L2).
+//
+// A group's rows split into mt = ceil(rows / bm) m-tiles of bm rows.  A
+// launch covers them in one of three ways (TileSet):
+//   kAllTiles  every m-tile, one per tile                       (mt tiles)
+//   kPairs     groups with mt >= kPairMinTiles: m-tiles two by two, 2*bm rows
+//              per tile                                         (mt / 2 tiles)
+//   kSingles   the other groups' m-tiles, and the odd last m-tile of the
+//              paired groups, one per tile
+// kPairs and kSingles together cover every row exactly once.  Pairing is
+// kept to large groups because the odd last m-tile runs in the other launch
+// and reads the group's weight strip again; at 8+ m-tiles that costs at most
+// one strip read in eight.
 #pragma once
 
 #include <stdint.h>
 
 namespace moe {
+
+enum TileSet { kAllTiles = 0, kPairs = 1, kSingles = 2 };
+constexpr int kPairMinTiles = 8;
+
+__device__ __forceinline__ int tiles_of_rows(int rows, int set, int bm) {
+  const int mt = (rows + bm - 1) / bm;
+  const bool paired = mt >= kPairMinTiles;
+  if (set == kPairs) return paired ? mt / 2 : 0;
+  if (set == kSingles) return paired ? (mt & 1) : mt;
+  return mt;
+}
+
+// First row (inside its group) of tile m of a group with `rows` rows.
+__device__ __forceinline__ int tile_first_row(int m, int rows, int set, int bm) {
+  const int mt = (rows + bm - 1) / bm;
+  if (set == kPairs) return m * 2 * bm;
+  if (set == kSingles && mt >= kPairMinTiles) return (mt - 1) * bm;   // the odd last tile
+  return m * bm;
+}
 
 struct GroupInfo {
   int src;           // 0 = routed operands, 1 = shared operands
@@ -53,8 +84,8 @@ __device__ __forceinline__ GroupInfo group_info(int g, const int* s_off, int E, 
 // Offsets outside [0, rows_cap] or decreasing are clamped to an empty group
 // and reported through `bad` (set to 1).
 __device__ inline void build_tile_prefix(const int32_t* __restrict__ offsets, int E, int S,
-                                         int64_t T, int BM, int n_tiles, int rows_cap, int* s_off,
-                                         int* s_tile, int* bad) {
+                                         int64_t T, int set, int bm, int n_tiles, int rows_cap,
+                                         int* s_off, int* s_tile, int* bad) {
   const int lane = threadIdx.x & 31;
   if (E == 0) {
     if (lane == 0) s_off[0] = 0;
@@ -85,7 +116,7 @@ __device__ inline void build_tile_prefix(const int32_t* __restrict__ offsets, in
     int cnt = 0;
     if (g < G) {
       const int rows = g < E ? (s_off[g + 1] - s_off[g]) : static_cast<int>(T);
-      cnt = ((rows + BM - 1) / BM) * n_tiles;
+      cnt = tiles_of_rows(rows, set, bm) * n_tiles;
     }
     int incl = cnt;
 #pragma unroll
@@ -99,9 +130,11 @@ __device__ inline void build_tile_prefix(const int32_t* __restrict__ offsets, in
   __syncwarp();
 }
 
-// Map a linear tile id to (group, m-tile, n-tile) using the prefix table.
+// Map a linear tile id to (group, m, n-tile) using the prefix table; the
+// tile's first row is tile_first_row(m, rows, set, bm).
 __device__ __forceinline__ void decode_tile(int tile, const int* s_tile, int G, const int* s_off,
-                                            int E, int64_t T, int BM, int& g, int& m, int& n) {
+                                            int E, int64_t T, int set, int bm, int& g, int& m,
+                                            int& n) {
   int lo = 0, hi = G - 1;   // find last g with s_tile[g] <= tile
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -109,7 +142,7 @@ __device__ __forceinline__ void decode_tile(int tile, const int* s_tile, int G, 
   }
   g = lo;
   const int rows = g < E ? (s_off[g + 1] - s_off[g]) : static_cast<int>(T);
-  const int mt = (rows + BM - 1) / BM;
+  const int mt = tiles_of_rows(rows, set, bm);
   const int local = tile - s_tile[g];
   n = local / mt;
   m = local - n * mt;

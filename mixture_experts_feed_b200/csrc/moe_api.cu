@@ -328,8 +328,10 @@ int32_t moe_forward_kernel_count(const moe_layer_desc_t* desc) {
   Layer L;
   if (check_desc(desc, &L) != MOE_OK || L.T == 0) return 0;
   // router: (bf16: split + tensor-core logits | fp32: logits) + top-k;
-  // permute: count, scan, compact, gather; experts: gate_up + down; combine.
-  return (L.dtype == MOE_BF16 ? 3 : 2) + 4 + 2 + 1;
+  // permute: count, scan, compact, gather; experts: gate_up + down (bf16 with
+  // T > 896: CTA-pair launch + single-CTA launch each); combine.
+  const int experts = L.dtype == MOE_BF16 ? (L.T > 896 ? 4 : 2) : 2;
+  return (L.dtype == MOE_BF16 ? 3 : 2) + 4 + experts + 1;
 }
 
 const char* moe_status_string(moe_status_t status) {
