@@ -20,7 +20,8 @@
 //            64-deep K blocks: the MMA writes a fresh chain sum, and the
 //            epilogue warps add the chain sums in fp32 registers with
 //            round-to-nearest adds.  fp32 logits out.  One group (all T
-//            tokens), N = E + S, 128-column tiles.
+//            tokens), N = E + S, 160-column tiles (E + S = 129 in one tile,
+//            257 in two).
 //
 // The expert modes run on CTA pairs (clusters of two SMs, tcgen05
 // cta_group::2): a pair computes a 256-row x 256-column tile with M=256
@@ -67,14 +68,15 @@ template <int MODE, bool PAIR_> struct Tile {
   static constexpr bool PAIR = PAIR_;                       // CTA-pair (M=256) MMAs
   // which m-tiles of each group the launch covers (grouping.cuh)
   static constexpr int SET = PAIR ? kPairs : (MODE == kRouter ? kAllTiles : kSingles);
-  static constexpr int BN = MODE == kRouter ? 128 : 256;    // MMA N = accumulator columns
+  static constexpr int BN = MODE == kRouter ? 160 : 256;    // MMA N = accumulator columns
   static constexpr int B_ROWS = PAIR ? BN / 2 : BN;         // B rows one CTA loads
   static constexpr int B_BYTES = B_ROWS * BK * 2;
-  static constexpr int B_BOX = 128;                         // rows per B tensor-map box
+  static constexpr int B_BOX = MODE == kRouter ? BN : 128;  // rows per B tensor-map box
   static constexpr int B_LOADS = B_ROWS / B_BOX;            // boxes per stage
   static constexpr int STAGES = PAIR ? 6 : 4;
   static constexpr int TILE_M = PAIR ? 2 * BM : BM;         // rows per tile
-  static constexpr uint32_t TMEM_COLS = 2 * BN;             // two accumulators
+  // two accumulators, allocation rounded up to a power of two
+  static constexpr uint32_t TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
   static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, BN);
 };
 
@@ -378,7 +380,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (n * BN + c * 32 < p.N) {            // warp-uniform
               uint32_t v[32], v2[32];
               tmem_ld_32x32b_x32(t_lane + static_cast<uint32_t>(acc * BN + c * 32), v);
-              const bool second = n * BN + (c + 1) * 32 < p.N;
+              const bool second = c + 1 < BN / 32 && n * BN + (c + 1) * 32 < p.N;
               if (second) tmem_ld_32x32b_x32(t_lane + static_cast<uint32_t>(acc * BN + (c + 1) * 32), v2);
               tmem_ld_wait();
 #pragma unroll
@@ -586,10 +588,9 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   g.E = L.E; g.S = L.S; g.K = L.H; g.N = 2 * L.I; g.ld_out = L.I;
   g.rows_cap = static_cast<int>(Rk);
   g.ksplit = 1;
-  // large groups' m-tiles two by two on CTA pairs, then every other m-tile on
-  // single CTAs (grouping.cuh); with fewer than kPairMinTiles m-tiles of rows
-  // no group can pair and the pair launch is skipped
-  const bool pairs = L.T > static_cast<int64_t>(kPairMinTiles - 1) * BM;
+  // paired groups on CTA pairs, the rest on single CTAs (grouping.cuh); with
+  // T <= 128 every group has one m-tile and the pair launch is skipped
+  const bool pairs = L.T > BM;
   cudaError_t e = pairs ? launch_mode<kGateUp, true>(g, num_sms, stream) : cudaSuccess;
   if (e == cudaSuccess) e = launch_mode<kGateUp, false>(g, num_sms, stream);
   if (e != cudaSuccess) return e;

@@ -33,7 +33,7 @@ int logits_ld(const Layer& L) { return (L.E + L.S + 31) / 32 * 32; }
 // partial-sum order (and every result) is the same on any device.
 int router_ksplit(const Layer& L) {
   if (L.dtype != MOE_BF16) return 1;
-  const int64_t tiles = (L.T + 127) / 128 * ((L.E + L.S + 127) / 128);
+  const int64_t tiles = (L.T + 127) / 128 * ((L.E + L.S + 159) / 160);   // router tiles
   int64_t ks = 148 / (tiles > 0 ? tiles : 1);
   if (ks < 1) ks = 1;
   if (ks > 32) ks = 32;
@@ -329,8 +329,8 @@ int32_t moe_forward_kernel_count(const moe_layer_desc_t* desc) {
   if (check_desc(desc, &L) != MOE_OK || L.T == 0) return 0;
   // router: (bf16: split + tensor-core logits | fp32: logits) + top-k;
   // permute: count, scan, compact, gather; experts: gate_up + down (bf16 with
-  // T > 896: CTA-pair launch + single-CTA launch each); combine.
-  const int experts = L.dtype == MOE_BF16 ? (L.T > 896 ? 4 : 2) : 2;
+  // T > 128: CTA-pair launch + single-CTA launch each); combine.
+  const int experts = L.dtype == MOE_BF16 ? (L.T > 128 ? 4 : 2) : 2;
   return (L.dtype == MOE_BF16 ? 3 : 2) + 4 + experts + 1;
 }
 

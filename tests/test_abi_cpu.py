@@ -55,7 +55,7 @@ def test_workspace_size_covers_intermediates(w):
     Rk = w.T * w.k
     need = el * (Rk * w.H + (Rk + w.S * w.T) * w.I) + 4 * (Rk + w.S * w.T) * w.H
     assert n >= need
-    experts = (4 if w.T > 896 else 2) if w.dtype == "bf16" else 2
+    experts = (4 if w.T > 128 else 2) if w.dtype == "bf16" else 2
     assert moe.forward_kernel_count(L) == (3 if w.dtype == "bf16" else 2) + 4 + experts + 1
 
 

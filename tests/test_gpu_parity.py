@@ -92,7 +92,7 @@ def test_workload_full_size(w):
 
 
 def test_one_expert_takes_every_token():
-    w, inputs = small_case(1100, 256, 16, 2, 1, 128)   # 9 m-tiles: 4 CTA pairs + 1 single
+    w, inputs = small_case(1100, 256, 16, 2, 1, 128)   # 9 m-tiles: 5 CTA pairs, the last half padding
     inputs["corr_bias"] = torch.zeros(w.E)
     inputs["corr_bias"][0] = 5.0           # every token ranks expert 0 first
     L = moe.Layer.from_workload(w)
