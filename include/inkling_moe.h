@@ -198,6 +198,18 @@ moe_status_t moe_forward(const moe_layer_desc_t* desc, const void* x, const floa
                          void* out, float* topk_w, int32_t* topk_idx, float* shared_gamma,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * moe_selftest_wait_timeout — diagnostic of the stall detection (no
+ * counterpart on the pages).  Launches one block that waits, through the
+ * same bounded wait every pipeline stage of the grouped GEMM uses, on a
+ * barrier nothing arrives on.  After limit_ms (1..10000) the wait gives up
+ * and records a timeout in the workspace status word, so that a following
+ * moe_read_device_status() returns MOE_ERR_TIMEOUT; the kernel then returns
+ * normally and the CUDA context stays usable.
+ */
+moe_status_t moe_selftest_wait_timeout(void* workspace, size_t workspace_bytes, uint32_t limit_ms,
+                                       void* stream);
+
 /* Number of kernels moe_forward launches for this layer (for launch accounting). */
 int32_t moe_forward_kernel_count(const moe_layer_desc_t* desc);
 

@@ -8,7 +8,7 @@ are handed to the C ABI unchanged; shapes, dtypes and contiguity are checked
 here so that a mistake raises instead of reaching the GPU.
 
 There is no CPU fallback: importing this package raises when the shared
-library has not been built (``python -m mixture_experts_feed_b200.build``).
+library has not been built (``python mixture_experts_feed_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -23,7 +23,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libinkling
 
 if not os.path.exists(_LIB_PATH):
     raise ImportError(
-        f"{_LIB_PATH} is missing; build it with `python -m mixture_experts_feed_b200.build`")
+        f"{_LIB_PATH} is missing; build it with `python mixture_experts_feed_b200/build.py`")
 
 LIB = ctypes.CDLL(_LIB_PATH)
 LIB_PATH = _LIB_PATH
@@ -65,8 +65,10 @@ LIB.moe_permute_noalloc.argtypes = [_DESC, _P, _P, _P, _P, _P, _P, _P, _P]
 LIB.moe_expert_ffn.argtypes = [_DESC] + [_P] * 13 + [ctypes.c_size_t, _P]
 LIB.moe_combine.argtypes = [_DESC, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 LIB.moe_forward.argtypes = [_DESC] + [_P] * 13 + [ctypes.c_size_t, _P]
+LIB.moe_selftest_wait_timeout.argtypes = [_P, ctypes.c_size_t, ctypes.c_uint32, _P]
 for _f in ("moe_workspace_size", "moe_workspace_init", "moe_read_device_status", "moe_route",
-           "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_combine", "moe_forward"):
+           "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_combine", "moe_forward",
+           "moe_selftest_wait_timeout"):
     getattr(LIB, _f).restype = ctypes.c_int
 
 
@@ -250,6 +252,13 @@ def moe_forward(layer: Layer, x, w_router, corr_bias, w_gate_up, w_down, ws_gate
                            _ptr(padding_mask), _ptr(out), _ptr(topk_w), _ptr(topk_idx),
                            _ptr(shared_gamma), ws.data_ptr(), ws.numel(), _stream(stream)),
            "moe_forward")
+
+
+def selftest_wait_timeout(ws: torch.Tensor, limit_ms: int = 1000, stream=None) -> None:
+    """Launch the stall-detection self-test (see the header); the next
+    read_device_status() raises MoEError with MOE_ERR_TIMEOUT."""
+    _check(LIB.moe_selftest_wait_timeout(ws.data_ptr(), ws.numel(), limit_ms, _stream(stream)),
+           "moe_selftest_wait_timeout")
 
 
 def forward_kernel_count(layer: Layer) -> int:

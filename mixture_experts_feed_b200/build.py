@@ -1,6 +1,9 @@
 """Build libinklingmoe.so in-tree with nvcc for sm_100a.
 
-    python -m mixture_experts_feed_b200.build [--force] [--verbose]
+    python mixture_experts_feed_b200/build.py [--force] [--verbose] [--ptxas-verbose]
+
+Run it as a script (or load it by path): importing the package would load
+the library it builds.
 
 Objects go to ``_build/`` at the repository root; the shared library lands
 next to this file so that it travels with the source tree.
@@ -22,7 +25,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libinklingmoe.so")
 
 SOURCES = ["moe_api.cu", "router.cu", "permute.cu", "permute_noalloc.cu",
-           "grouped_gemm_sm100.cu", "grouped_gemm_simt.cu", "combine.cu"]
+           "grouped_gemm_sm100.cu", "grouped_gemm_simt.cu", "combine.cu", "selftest.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
                      "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

@@ -11,8 +11,12 @@ if TESTS not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
-    # The library is built in-tree; build it once if this checkout has none.
-    lib = os.path.join(ROOT, "mixture_experts_feed_b200", "libinklingmoe.so")
-    if not os.path.exists(lib):
-        from mixture_experts_feed_b200.build import build
-        build()
+    # The library is built in-tree; (re)build it when a source is newer than
+    # it.  build.py is loaded by path: importing the package would load the
+    # library before it exists.
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_inkling_moe_build", os.path.join(ROOT, "mixture_experts_feed_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()

@@ -108,6 +108,8 @@ def test_null_and_misaligned_pointers_are_rejected_before_launch():
     assert _status("moe_forward", d, fake, fake, fake, fake, fake, None, fake, None, fake,
                    None, None, None, fake, ws_ok, None) == 1
     assert _status("moe_workspace_init", None, 1024, None) == 1
+    assert _status("moe_selftest_wait_timeout", None, 1024, 100, None) == 1
+    assert _status("moe_selftest_wait_timeout", fake, 1024, 0, None) == 1
     assert _status("moe_read_device_status", None, None, None) == 1
 
 

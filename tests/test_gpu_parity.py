@@ -205,3 +205,21 @@ def test_out_of_range_expert_id_is_reported_not_faulted():
     assert int(off[-1]) == w.T * w.k - 1
     assert int(ip[5 * w.k + 1]) == -1
     assert moe.read_device_status(ws) == 0      # cleared by the read
+
+
+def test_stalled_wait_times_out_and_context_survives():
+    """A pipeline wait that nothing satisfies gives up after its limit (1 s
+    here), records a timeout the host reads, and the GPU keeps working."""
+    import time
+    w, inputs = small_case(64, 128, 8, 2, 1, 64)
+    L = moe.Layer.from_workload(w)
+    ws = moe.new_workspace(L)
+    t0 = time.perf_counter()
+    moe.selftest_wait_timeout(ws, limit_ms=1000)
+    with pytest.raises(moe.MoEError) as ei:
+        moe.read_device_status(ws)
+    elapsed = time.perf_counter() - t0
+    assert ei.value.status == 6 and ei.value.device_code == 0x201
+    assert 0.9 < elapsed < 30.0
+    r = run_forward(L, to_device(inputs), ws=ws)     # the context is still usable
+    assert torch.isfinite(r["out"].float()).all()
