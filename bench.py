@@ -37,10 +37,13 @@ import moe_workloads as mw  # noqa: E402
 METRIC = "Inkling MoE-layer tokens/s and TFLOP/s (% of B200 bf16 peak / % HBM BW), 1 GPU"
 DEFAULT_WORKLOAD = "bf16-T8192-H6144-E128k8S1-I2048"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes per launch of the expert GEMMs measured by ncu on this workload
-# (dram__bytes_read.sum + dram__bytes_write.sum); None until captured for the
-# current kernel build.
-NCU_TRAFFIC_BYTES = {}
+# DRAM bytes of one moe_expert_ffn call (its four grouped-GEMM launches) on
+# this workload, measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum,
+# one pass, first warm-up step); absent until captured for the current build.
+NCU_TRAFFIC_BYTES = {
+    "bf16-T8192-H6144-E128k8S1-I2048": 16838837760,
+    "zipf-bf16-T16384-H6144-E256k8S1-I1024": 9757464320,
+}
 
 
 def load_peaks():
@@ -277,21 +280,46 @@ def gpu_arm(args, world, rank, local):
     op_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(4)]
     ms_step = max_over_ranks(total_ms / args.steps, world)
 
-    # ---- end to end through the public one-call API with host buffers
-    def e2e_step():
-        d["x"].copy_(x_host, non_blocking=True)
-        moe.moe_forward(L, d["x"], d["w_router"], d["corr_bias"], d["w_gate_up"], d["w_down"],
-                        wsgu, wsd, out, ws, stream=stream)
-        out_host.copy_(out, non_blocking=True)
+    # ---- end to end through the public one-call API with host buffers: every
+    # step copies its input from pinned host memory and its output back.  Two
+    # device buffer sets and three streams let step i's upload and step i-1's
+    # download overlap step i-1's / step i's compute; each step still pays for
+    # its own copies, and the region ends when the last output is on the host.
+    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    x_dev = [d["x"], torch.empty_like(d["x"])]
+    out_dev = [out, torch.empty_like(out)]
+    out_host2 = [out_host, torch.empty_like(out_host).pin_memory()]
+    ev = {n: [torch.cuda.Event() for _ in range(2)] for n in ("h2d", "comp", "d2h")}
 
-    for _ in range(max(1, args.warmup // 2)):
-        e2e_step()
+    def e2e_steps(n):
+        for i in range(n):
+            b = i & 1
+            with torch.cuda.stream(h2d_s):
+                if i >= 2:
+                    h2d_s.wait_event(ev["comp"][b])                   # x_dev[b] free again
+                x_dev[b].copy_(x_host, non_blocking=True)
+                ev["h2d"][b].record(h2d_s)
+            stream.wait_event(ev["h2d"][b])
+            if i >= 2:
+                stream.wait_event(ev["d2h"][b])                       # out_dev[b] read back
+            moe.moe_forward(L, x_dev[b], d["w_router"], d["corr_bias"], d["w_gate_up"],
+                            d["w_down"], wsgu, wsd, out_dev[b], ws, stream=stream)
+            ev["comp"][b].record(stream)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(ev["comp"][b])
+                out_host2[b].copy_(out_dev[b], non_blocking=True)
+                ev["d2h"][b].record(d2h_s)
+
+    e2e_steps(max(2, args.warmup // 2))
+    torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize(dev)
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    h2d_s.wait_event(e0)
+    e2e_steps(args.steps)
+    stream.wait_stream(d2h_s)
+    stream.wait_stream(h2d_s)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
@@ -303,8 +331,29 @@ def gpu_arm(args, world, rank, local):
         fl = mw.flops(w)
         ffn_flops = fl["routed"] + fl["shared"]
         ffn_s = op_ms[2] / 1e3
-        achieved = ffn_flops / ffn_s / 1e12
+        # algorithmic bytes of moe_expert_ffn: the weights of every group with
+        # rows (routed experts with a nonzero count, every shared expert) once,
+        # x_perm / x rows read once, h written and read once in the dtype, the
+        # fp32 down rows written once
+        el = 2 if w.dtype == "bf16" else 4
+        counts = (off[1:] - off[:-1]).cpu()
+        touched = int((counts > 0).sum()) + S
+        rows = T * (k + S)
+        ffn_bytes = touched * 3 * H * w.I * el + rows * (H * el + 2 * w.I * el + 4 * H)
         peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        ridge = peak * 1e12 / (hbm_peak * 1e9)
+        if ffn_flops / ffn_bytes >= ridge:
+            roof = {"bound": "tensor", "achieved": ffn_flops / ffn_s / 1e12, "peak": peak,
+                    "unit": "TFLOP/s", "peak_source": f"{peak_src} bf16_tflops_sustained"}
+        else:
+            roof = {"bound": "hbm", "achieved": ffn_bytes / ffn_s / 1e9, "peak": hbm_peak,
+                    "unit": "GB/s", "peak_source": f"{peak_src} hbm_gbs"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["traffic"] = NCU_TRAFFIC_BYTES.get(w.name)
+        roof["algorithmic_bytes"] = ffn_bytes
+        roof["algorithmic_flops"] = ffn_flops
+        roof["touched_groups"] = touched
         tokens_s = world * T / (ms_step / 1e3)
         line = {
             "metric": METRIC, "value": tokens_s, "unit": "tokens/s", "n_gpus": world,
@@ -317,10 +366,7 @@ def gpu_arm(args, world, rank, local):
             "tflops": world * fl["total"] / (ms_step / 1e3) / 1e12,
             "op_ms": {"route": op_ms[0], "permute": op_ms[1], "expert_ffn": op_ms[2], "combine": op_ms[3]},
             "roofline": {"kernel": "grouped expert GEMMs (gate_up + down launches of moe_expert_ffn)",
-                         "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak,
-                         "peak_source": f"{peak_src} bf16_tflops_sustained",
-                         "traffic": NCU_TRAFFIC_BYTES.get(w.name)},
+                         **roof},
             "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
                     "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},

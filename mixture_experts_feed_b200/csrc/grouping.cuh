@@ -8,9 +8,14 @@
 // weights are slice s of the shared weight tensor, outputs go to rows
 // s * T + t of output 1.
 //
-// Tiles are numbered group by group; inside a group, n-tile by n-tile, and
-// inside an n-tile, m-tile by m-tile (consecutive tiles share one weight
-// strip, so CTAs running together reuse it from L2).
+// Tiles are numbered group by group.  Inside a group the longer of its two
+// tile dimensions is the outer one: with no more m-tiles than n-tiles, tiles
+// run n-tile by n-tile and m-tile by m-tile inside (consecutive tiles share
+// one weight strip); with more m-tiles than n-tiles, m-tile by m-tile and
+// n-tile by n-tile inside (consecutive tiles share one block of rows).  CTAs
+// running together then reuse the shared operand from L2, and the group's
+// other operand (the n-tile strips, or the row blocks) is the smaller one to
+// keep in L2 from one wave of tiles to the next.
 //
 // A group's rows split into mt = ceil(rows / bm) m-tiles of bm rows.  A
 // launch covers them in one of three ways (TileSet):
@@ -144,8 +149,14 @@ __device__ __forceinline__ void decode_tile(int tile, const int* s_tile, int G, 
   const int rows = g < E ? (s_off[g + 1] - s_off[g]) : static_cast<int>(T);
   const int mt = tiles_of_rows(rows, set, bm);
   const int local = tile - s_tile[g];
-  n = local / mt;
-  m = local - n * mt;
+  const int nt = (s_tile[g + 1] - s_tile[g]) / mt;
+  if (mt > nt) {
+    m = local / nt;
+    n = local - m * nt;
+  } else {
+    n = local / mt;
+    m = local - n * mt;
+  }
 }
 
 }  // namespace moe
