@@ -39,7 +39,8 @@ from typing import Dict, Optional
 import torch
 
 __all__ = ["Workload", "WORKLOADS", "by_name", "generate", "slice_seed",
-           "expert_slice", "zipf_bias", "flops", "tiny"]
+           "expert_slice", "zipf_bias", "flops", "tiny", "DenseWorkload",
+           "DENSE_WORKLOADS", "dense_by_name", "generate_dense", "dense_flops"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -114,7 +115,8 @@ def flops(w: Workload, tokens: Optional[int] = None) -> Dict[str, float]:
 
 # ---------------------------------------------------------------- generator
 _TENSOR_IDS = {"x": 1, "w_router": 2, "corr_bias": 3, "w_gate_up": 4,
-               "w_down": 5, "ws_gate_up": 6, "ws_down": 7}
+               "w_down": 5, "ws_gate_up": 6, "ws_down": 7,
+               "dense_gate_up": 8, "dense_down": 9}
 
 
 def slice_seed(seed: int, tensor: str, index: int = 0) -> int:
@@ -225,3 +227,114 @@ def weight_bytes(w: Workload) -> int:
     el = 4 if w.dtype == "f32" else 2
     return el * (w.E + w.S) * 3 * w.H * w.I + 4 * (w.E + w.S) * w.H + 4 * w.E
 
+
+
+# ------------------------------------------------------------ dense layers
+# The dense feed-forward layer of the model (``InklingDenseMLP`` on the
+# ``layers`` page; ``dense_mlp_idx`` picks which decoder layer has it).  Its
+# width is ``dense_intermediate_size`` when set, else ``intermediate_size``
+# (24576 by default, ``InklingTextConfig``).  Weights in ``[out, in]`` form:
+#
+#   x          [T, H]    activations, N(0, 1)
+#   gate_up    [2I, H]   fused projection, row 2j = gate_j, row 2j+1 = up_j,
+#                        N(0, 0.02^2) (``InklingDenseMLP.init_weights``)
+#   down       [H, I]    N(0, 0.02^2)
+#
+# The projections are drawn in slices of 256 rows, each from its own seed,
+# so they can be drawn in parallel with identical results.
+
+@dataclasses.dataclass(frozen=True)
+class DenseWorkload:
+    """One dense-MLP layer shape with its value distributions and seed."""
+
+    name: str
+    T: int
+    H: int
+    I: int
+    dtype: str        # "f32" or "bf16"
+    global_scale: float
+    seed: int
+    init_std: float = 0.02
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    def replace(self, **kw) -> "DenseWorkload":
+        return dataclasses.replace(self, **kw)
+
+
+DENSE_WORKLOADS: Dict[str, DenseWorkload] = {w.name: w for w in [
+    # the dense layer at the model's sizes (hidden 6144, intermediate 24576)
+    DenseWorkload("dense-bf16-T8192-H6144-I24576", 8192, 6144, 24576, "bf16", 1.0, seed=5),
+    # one decode step of the same layer: weight-streaming bound
+    DenseWorkload("dense-decode-bf16-T32-H6144-I24576", 32, 6144, 24576, "bf16", 1.0, seed=6),
+    # small cases the oracle finishes in seconds (ragged T, several tiles)
+    DenseWorkload("dense-bf16-T300-H512-I640", 300, 512, 640, "bf16", 1.0, seed=7),
+    DenseWorkload("dense-f32-T96-H128-I192", 96, 128, 192, "f32", 1.0, seed=8),
+]}
+
+
+def dense_by_name(name: str) -> DenseWorkload:
+    if name in DENSE_WORKLOADS:
+        return DENSE_WORKLOADS[name]
+    raise KeyError(f"unknown dense workload {name!r}; known: {list(DENSE_WORKLOADS)}")
+
+
+def dense_tiny(T=24, H=64, I=96, dtype="f32", global_scale=1.0, seed=21) -> DenseWorkload:
+    """A small ad-hoc dense workload for unit tests."""
+    return DenseWorkload(f"dense-adhoc-T{T}-H{H}-I{I}-{dtype}", T, H, I, dtype, global_scale, seed)
+
+
+_DENSE_SLICE = 256
+
+
+def _fill_rows(w: DenseWorkload, tensor: str, rows: int, cols: int, threads: int) -> torch.Tensor:
+    out = torch.empty((rows, cols), dtype=w.torch_dtype)
+    n = (rows + _DENSE_SLICE - 1) // _DENSE_SLICE
+
+    def one(i):
+        r0 = i * _DENSE_SLICE
+        r1 = min(rows, r0 + _DENSE_SLICE)
+        out[r0:r1].copy_(_normal((r1 - r0, cols), w.init_std, slice_seed(w.seed, tensor, i)))
+        return i
+
+    if threads <= 1:
+        for i in range(n):
+            one(i)
+    else:
+        with _cf.ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(one, range(n)))
+    return out
+
+
+def generate_dense(w: DenseWorkload, pin_memory: bool = False,
+                   threads: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """Inputs of one dense layer as CPU tensors: ``x``, ``w_gate_up``, ``w_down``."""
+    if threads is None:
+        threads = max(1, min(16, len(os.sched_getaffinity(0))))
+    torch_threads = torch.get_num_threads()
+    torch.set_num_threads(1 if threads > 1 else torch_threads)
+    try:
+        d = {"x": _normal((w.T, w.H), 1.0, slice_seed(w.seed, "x")).to(w.torch_dtype),
+             "w_gate_up": _fill_rows(w, "dense_gate_up", 2 * w.I, w.H, threads),
+             "w_down": _fill_rows(w, "dense_down", w.H, w.I, threads)}
+    finally:
+        torch.set_num_threads(torch_threads)
+    if pin_memory:
+        d = {k: v.pin_memory() for k, v in d.items()}
+    return d
+
+
+def dense_flops(w: DenseWorkload, tokens: Optional[int] = None) -> float:
+    """Algorithmic flops of one dense layer (2 per multiply-add)."""
+    T = w.T if tokens is None else tokens
+    return 6.0 * T * w.H * w.I
+
+
+def dense_token_sample(w: DenseWorkload, n: int, seed_offset: int = 0) -> torch.Tensor:
+    """A fixed, sorted, seeded subset of token indices of a dense workload."""
+    n = min(n, w.T)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed * 31 + 977 + seed_offset)
+    return torch.randperm(w.T, generator=g)[:n].sort().values

@@ -26,6 +26,10 @@ What it computes, step by step, from the NeMo AutoModel Inkling pages
    (``InklingMoE.forward``).
 7. ``permute``: the reference token order for grouped dispatch, rows ordered
    by (expert, token).
+8. ``dense_mlp``: the dense feed-forward layer (``InklingDenseMLP.forward``):
+   fused interleaved gate/up projection, SwiGLU, down projection, times the
+   layer's ``global_scale`` (the pages leave where it applies unstated; the
+   output is scaled, which in exact arithmetic equals scaling h).
 
 Readings taken where the pages are silent (each one is listed in the design doc):
 log-sigmoid applies to the whole concatenated vector, shared logits included;
@@ -33,12 +37,15 @@ the gammas are scaled like the routed weights; ties in the selection score go
 to the lower expert index and the k chosen experts are returned in descending
 score order; weights are stored ``[out, in]`` (the checkpoint form that needs
 no more than a transposed view); the router has no norm; padded tokens take no routed
-rows but still receive the shared experts.
+rows but still receive the shared experts; the dense layer's global_scale
+multiplies its output.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (brute-force selection, closed-form weights, the sum invariant, the textbook
 SwiGLU MLP special case, a library sort for the permutation, and a hand-worked
-two-token example under ``tests/golden/``).
+two-token example under ``tests/golden/``; for ``dense_mlp`` a textbook
+SwiGLU MLP from separate gate and up matrices and a hand-worked closed-form
+example).
 """
 from __future__ import annotations
 
@@ -243,3 +250,24 @@ def permute(topk_idx: torch.Tensor, n_routed: int,
 
 def default_threads() -> int:
     return max(1, len(os.sched_getaffinity(0)))
+
+
+# ------------------------------------------------------------- dense layer
+def dense_mlp(x: torch.Tensor, w_gate_up: torch.Tensor, w_down: torch.Tensor,
+              global_scale: float = 1.0, tokens: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """``InklingDenseMLP.forward`` (``layers`` page): ``x`` of shape ``[..., H]``
+    (any leading dims) through the fused interleaved projection ``w_gate_up``
+    ``[2I, H]`` (row 2j gate_j, row 2j+1 up_j), SwiGLU (``inkling_swiglu`` with
+    weight 1), the down projection ``w_down`` ``[H, I]``, times
+    ``global_scale``.  Returns float64 of shape ``[..., H]``; with ``tokens``
+    (indices into the flattened leading dims) only those rows, ``[n, H]``."""
+    H = x.shape[-1]
+    x64 = _f64(x).reshape(-1, H)
+    if tokens is not None:
+        x64 = x64[tokens]
+    G = x64 @ _f64(w_gate_up).T
+    h = swiglu_interleaved(G, torch.ones(G.shape[0], 1, dtype=F64))
+    out = float(global_scale) * (h @ _f64(w_down).T)
+    if tokens is not None:
+        return out
+    return out.reshape(*x.shape[:-1], H)

@@ -360,3 +360,88 @@ def test_planted_transposed_down_is_caught(monkeypatch):
         Wd = w_down.reshape(w_down.shape[1], w_down.shape[0])   # wrong orientation, same size
         return h @ Wd
     _expect_pin_failure(monkeypatch, "expert_mlp", bad, [check_interleave, check_two_token])
+
+
+# ------------------------------------------------------------- dense layer
+DENSE_GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "dense_mlp_example.json")
+
+
+def check_dense_example():
+    g = json.load(open(DENSE_GOLDEN))
+    a = math.log(3.0)
+    x = (torch.tensor(g["inputs"]["x_coeff_a"], dtype=F64) * a
+         + torch.tensor(g["inputs"]["x_coeff_1"], dtype=F64))
+    out = oracle.dense_mlp(x, torch.tensor(g["inputs"]["w_gate_up"], dtype=F64),
+                           torch.tensor(g["inputs"]["w_down"], dtype=F64),
+                           g["sizes"]["global_scale"])
+    want = frac(g["expected"]["out_coeff_a"]) * a + frac(g["expected"]["out_coeff_a2"]) * a * a
+    np.testing.assert_allclose(out.numpy(), want, rtol=0, atol=1e-14)
+
+
+def check_dense_textbook(seed=5, gs=1.7):
+    g = torch.Generator().manual_seed(seed)
+    H, I = 10, 6
+    A = torch.randn(I, H, generator=g, dtype=F64)
+    B = torch.randn(I, H, generator=g, dtype=F64)
+    D = torch.randn(H, I, generator=g, dtype=F64)
+    x = torch.randn(2, 3, H, generator=g, dtype=F64)     # leading dims kept
+    got = oracle.dense_mlp(x, interleave_rows(A, B), D, gs)
+    assert got.shape == (2, 3, H)
+    want = gs * textbook_swiglu_mlp(x.reshape(-1, H), A, B, D)
+    np.testing.assert_allclose(got.reshape(-1, H).numpy(), want.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_dense_example():
+    check_dense_example()
+
+
+def test_dense_is_textbook_swiglu_mlp_times_global_scale():
+    check_dense_textbook()
+
+
+def test_dense_token_subset_equals_full_rows():
+    w = mw.dense_tiny(T=20, H=64, I=64)
+    d = mw.generate_dense(w)
+    full = oracle.dense_mlp(d["x"], d["w_gate_up"], d["w_down"], 0.5)
+    idx = torch.tensor([0, 7, 19])
+    sub = oracle.dense_mlp(d["x"], d["w_gate_up"], d["w_down"], 0.5, tokens=idx)
+    # same rows; the library matmul may block a 3-row product differently
+    np.testing.assert_allclose(sub.numpy(), full[idx].numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_dense_generator_slices_are_reproducible():
+    w = mw.dense_tiny(T=4, H=64, I=300)     # 600 gate/up rows: three 256-row slices
+    a = mw.generate_dense(w, threads=1)
+    b = mw.generate_dense(w, threads=4)
+    for k in a:
+        assert torch.equal(a[k], b[k])
+    assert a["w_gate_up"].shape == (600, 64) and a["w_down"].shape == (64, 300)
+
+
+def test_planted_dense_swapped_gate_up_is_caught(monkeypatch):
+    def bad(G, w):
+        g, u = G[..., 1::2], G[..., 0::2]
+        return w * (g * torch.sigmoid(g)) * u
+    _expect_pin_failure(monkeypatch, "swiglu_interleaved", bad, [check_dense_example])
+
+
+def test_planted_dense_missing_global_scale_is_caught(monkeypatch):
+    real = oracle.dense_mlp
+
+    def bad(x, wgu, wd, global_scale=1.0, tokens=None):
+        return real(x, wgu, wd, 1.0, tokens)
+    monkeypatch.setattr(oracle, "dense_mlp", bad)
+    for pin in (check_dense_example, check_dense_textbook):
+        with pytest.raises(AssertionError):
+            pin()
+
+
+def test_planted_dense_transposed_down_is_caught(monkeypatch):
+    real_mlp = oracle.dense_mlp
+
+    def bad(x, wgu, wd, global_scale=1.0, tokens=None):
+        return real_mlp(x, wgu, wd.T.contiguous().reshape(wd.shape), global_scale, tokens)
+    monkeypatch.setattr(oracle, "dense_mlp", bad)
+    for pin in (check_dense_example, check_dense_textbook):
+        with pytest.raises(AssertionError):
+            pin()
