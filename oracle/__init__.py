@@ -26,6 +26,10 @@ What it computes, step by step, from the NeMo AutoModel Inkling pages
    (``InklingMoE.forward``).
 7. ``permute``: the reference token order for grouped dispatch, rows ordered
    by (expert, token).
+9. ``rmsnorm``: the feed-forward block's input norm (``InklingRMSNorm`` on
+   the ``text`` page, the decoder layer's ``post_attention_layernorm``):
+   ``x / sqrt(mean(x^2) + eps) * weight`` over the hidden axis, in float64,
+   rounded once (round to nearest, ties to even) to the input's dtype.
 8. ``dense_mlp``: the dense feed-forward layer (``InklingDenseMLP.forward``):
    fused interleaved gate/up projection, SwiGLU, down projection, times the
    layer's ``global_scale`` (the pages leave where it applies unstated; the
@@ -271,3 +275,40 @@ def dense_mlp(x: torch.Tensor, w_gate_up: torch.Tensor, w_down: torch.Tensor,
     if tokens is not None:
         return out
     return out.reshape(*x.shape[:-1], H)
+
+
+# ------------------------------------------------------------------ RMSNorm
+def round_to_bf16(y: torch.Tensor) -> torch.Tensor:
+    """Round float64 values once to the nearest bfloat16 (ties to even),
+    returned as float64 holding bfloat16 values.  Normal range: keep the top
+    7 fraction bits of the float64 pattern, rounding on the dropped 45 bits
+    (adding 2^44 - 1 plus the kept last bit carries exactly when the dropped
+    part is above half, or exactly half with an odd last bit).  Below 2^-126
+    bfloat16 spacing is 2^-133: round y * 2^133 to an integer, ties to even.
+    (A float64 -> float32 -> bfloat16 cast rounds twice and can differ.)"""
+    a = y.detach().to("cpu", F64).numpy().copy()
+    bits = a.view(np.uint64)
+    lsb = (bits >> np.uint64(45)) & np.uint64(1)
+    rb = ((bits + np.uint64((1 << 44) - 1) + lsb) >> np.uint64(45)) << np.uint64(45)
+    r = rb.view(np.float64).copy()
+    tiny = np.abs(a) < 2.0 ** -126
+    r[tiny] = np.rint(a[tiny] * 2.0 ** 133) * 2.0 ** -133
+    return torch.from_numpy(r)
+
+
+def rmsnorm(x: torch.Tensor, weight: torch.Tensor, eps: float,
+            out_dtype: Optional[torch.dtype] = None) -> torch.Tensor:
+    """``InklingRMSNorm.forward``: each row of the last axis divided by its
+    root mean square (with ``eps`` added to the mean square), times the
+    learned ``weight``; float64.  With ``out_dtype`` (the module returns the
+    input's dtype) the float64 result is rounded once to it and returned in
+    that dtype."""
+    x64 = _f64(x)
+    y = x64 / torch.sqrt((x64 * x64).mean(-1, keepdim=True) + float(eps)) * _f64(weight)
+    if out_dtype is None:
+        return y
+    if out_dtype == torch.bfloat16:
+        return round_to_bf16(y).reshape(y.shape).to(torch.float32).to(torch.bfloat16)
+    if out_dtype == torch.float32:
+        return torch.from_numpy(y.numpy().astype(np.float32))
+    return y.to(out_dtype)

@@ -445,3 +445,99 @@ def test_planted_dense_transposed_down_is_caught(monkeypatch):
     for pin in (check_dense_example, check_dense_textbook):
         with pytest.raises(AssertionError):
             pin()
+
+
+# ------------------------------------------------------------------ RMSNorm
+RMS_GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "rmsnorm_example.json")
+
+
+def check_rmsnorm_example():
+    g = json.load(open(RMS_GOLDEN))
+    for c in g["cases"]:
+        y = oracle.rmsnorm(torch.tensor([c["x"]], dtype=F64), torch.tensor(c["weight"], dtype=F64),
+                           c["eps"])
+        np.testing.assert_allclose(y[0].numpy(), np.array(c["expected_over_sqrt2"]) * math.sqrt(2.0),
+                                   rtol=0, atol=1e-15)
+
+
+def check_rounding_cases():
+    vals = [1 + 2 ** -8, 1 + 3 * 2 ** -8, 1 + 2 ** -8 + 2 ** -30, -(1 + 2 ** -8 + 2 ** -30),
+            1.5 * 2.0 ** -133, 2.5 * 2.0 ** -133]
+    want = [1.0, 1 + 2 ** -6, 1 + 2 ** -7, -(1 + 2 ** -7), 2.0 ** -132, 2.0 ** -132]
+    got = oracle.round_to_bf16(torch.tensor(vals, dtype=F64)).tolist()
+    assert got == want
+
+
+def check_rounding_matches_single_rounding_from_float32(seed=9):
+    # float32 inputs: the library's float32 -> bfloat16 conversion rounds once
+    g = torch.Generator().manual_seed(seed)
+    a = torch.randn(20000, generator=g, dtype=torch.float32) * 3
+    ties = (torch.randint(-200, 200, (2000,), generator=g).float() + 0.5) * 2.0 ** -7  # exact ties
+    a = torch.cat([a, ties.float(), -ties.float()])
+    want = a.to(torch.bfloat16).double()
+    got = oracle.round_to_bf16(a.double())
+    assert torch.equal(got, want)
+
+
+def check_rmsnorm_library_and_invariants(seed=4):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(5, 3, 48, generator=g, dtype=F64)
+    w = torch.rand(48, generator=g, dtype=F64) + 0.5
+    eps = 1e-6
+    want = F.rms_norm(x, (48,), weight=w, eps=eps)     # library routine
+    np.testing.assert_allclose(oracle.rmsnorm(x, w, eps).numpy(), want.numpy(), rtol=1e-13, atol=1e-14)
+    ones = torch.ones(48, dtype=F64)
+    y = oracle.rmsnorm(x, ones, 0.0)
+    np.testing.assert_allclose(y.pow(2).mean(-1).numpy(), 1.0, rtol=1e-14)   # unit RMS
+    np.testing.assert_allclose(oracle.rmsnorm(7.5 * x, ones, 0.0).numpy(), y.numpy(), rtol=1e-14)
+
+
+def test_rmsnorm_example():
+    check_rmsnorm_example()
+
+
+def test_round_to_bf16_cases():
+    check_rounding_cases()
+    check_rounding_matches_single_rounding_from_float32()
+
+
+def test_rmsnorm_library_and_invariants():
+    check_rmsnorm_library_and_invariants()
+
+
+def test_rmsnorm_rounds_once_into_the_input_dtype():
+    g = torch.Generator().manual_seed(2)
+    x = torch.randn(4, 64, generator=g).to(torch.bfloat16)
+    w = (torch.rand(64, generator=g) + 0.5).to(torch.bfloat16)
+    y = oracle.rmsnorm(x, w, 1e-6, out_dtype=torch.bfloat16)
+    assert y.dtype == torch.bfloat16
+    assert torch.equal(y.double(), oracle.round_to_bf16(oracle.rmsnorm(x, w, 1e-6)).reshape(4, 64))
+    y32 = oracle.rmsnorm(x.float(), w.float(), 1e-6, out_dtype=torch.float32)
+    assert y32.dtype == torch.float32
+
+
+def test_planted_eps_outside_sqrt_is_caught(monkeypatch):
+    def bad(x, weight, eps, out_dtype=None):
+        x64 = x.double()
+        return x64 / (torch.sqrt((x64 * x64).mean(-1, keepdim=True)) + eps) * weight.double()
+    _expect_pin_failure(monkeypatch, "rmsnorm", bad, [check_rmsnorm_example])
+
+
+def test_planted_norm_over_wrong_axis_is_caught(monkeypatch):
+    def bad(x, weight, eps, out_dtype=None):
+        x64 = x.double()
+        return x64 / torch.sqrt((x64 * x64).mean(0, keepdim=True) + eps) * weight.double()
+    _expect_pin_failure(monkeypatch, "rmsnorm", bad, [check_rmsnorm_library_and_invariants])
+
+
+def test_planted_missing_norm_weight_is_caught(monkeypatch):
+    def bad(x, weight, eps, out_dtype=None):
+        x64 = x.double()
+        return x64 / torch.sqrt((x64 * x64).mean(-1, keepdim=True) + eps)
+    _expect_pin_failure(monkeypatch, "rmsnorm", bad, [check_rmsnorm_example])
+
+
+def test_planted_double_rounding_is_caught(monkeypatch):
+    monkeypatch.setattr(oracle, "round_to_bf16", lambda y: y.to(torch.bfloat16).double())
+    with pytest.raises(AssertionError):
+        check_rounding_cases()
