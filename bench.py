@@ -15,6 +15,10 @@ taken on the device with CUDA events and reduced as the max over ranks.
 
 ``--impl reference`` times the CPU fp64 oracle instead, on a bounded token
 sample per step, on rank 0 only.
+
+``--workload dense-...`` times the model's dense feed-forward layer
+(InklingDenseMLP, ``moe_dense_mlp``) the same way: a step is one forward pass
+of that layer over T tokens.
 """
 from __future__ import annotations
 
@@ -242,16 +246,25 @@ def gpu_arm(args, world, rank, local):
     wsgu = d.get("ws_gate_up") if S else None
     wsd = d.get("ws_down") if S else None
 
+    # --prenorm: the block's RMSNorm first (its own timed op), the layer on its output
+    nw = mw.norm_weight(H, seed=w.seed, dtype=L.dtype).to(dev) if args.prenorm else None
+    xn = torch.empty_like(d["x"]) if args.prenorm else None
+    xin = xn if args.prenorm else d["x"]
+
     def step(ev=None):
+        if args.prenorm:
+            if ev is not None:
+                ev[5].record(stream)
+            moe.moe_rmsnorm(d["x"], nw, xn, mw.RMS_NORM_EPS, stream)
         if ev is not None:
             ev[0].record(stream)
-        moe.moe_route(L, d["x"], d["w_router"], d["corr_bias"], tw, ti, sg, ws, stream)
+        moe.moe_route(L, xin, d["w_router"], d["corr_bias"], tw, ti, sg, ws, stream)
         if ev is not None:
             ev[1].record(stream)
-        moe.moe_permute(L, ti, None, d["x"], off, ps, ip, xp, ws, stream)
+        moe.moe_permute(L, ti, None, xin, off, ps, ip, xp, ws, stream)
         if ev is not None:
             ev[2].record(stream)
-        moe.moe_expert_ffn(L, d["x"], xp, off, ps, tw, sg, d["w_gate_up"], d["w_down"], wsgu, wsd,
+        moe.moe_expert_ffn(L, xin, xp, off, ps, tw, sg, d["w_gate_up"], d["w_down"], wsgu, wsd,
                            yr, ys, ws, stream)
         if ev is not None:
             ev[3].record(stream)
@@ -266,7 +279,7 @@ def gpu_arm(args, world, rank, local):
 
     # ---- timed region: K steps, inputs (weights 9.7 GB at the default
     # workload) far larger than the 126 MB L2, so no flush is needed between steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize(dev)
@@ -276,8 +289,10 @@ def gpu_arm(args, world, rank, local):
         barrier(world)
     clocks = clk.summary()
     moe.read_device_status(ws, stream)
-    total_ms = evs[0][0].elapsed_time(evs[-1][4])
+    first = 5 if args.prenorm else 0
+    total_ms = evs[0][first].elapsed_time(evs[-1][4])
     op_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(4)]
+    norm_ms = (sum(e[5].elapsed_time(e[0]) for e in evs) / args.steps) if args.prenorm else None
     ms_step = max_over_ranks(total_ms / args.steps, world)
 
     # ---- end to end through the public one-call API with host buffers: every
@@ -302,8 +317,13 @@ def gpu_arm(args, world, rank, local):
             stream.wait_event(ev["h2d"][b])
             if i >= 2:
                 stream.wait_event(ev["d2h"][b])                       # out_dev[b] read back
-            moe.moe_forward(L, x_dev[b], d["w_router"], d["corr_bias"], d["w_gate_up"],
-                            d["w_down"], wsgu, wsd, out_dev[b], ws, stream=stream)
+            if args.prenorm:
+                moe.moe_forward_prenorm(L, x_dev[b], nw, mw.RMS_NORM_EPS, d["w_router"],
+                                        d["corr_bias"], d["w_gate_up"], d["w_down"], wsgu, wsd,
+                                        out_dev[b], ws, stream=stream)
+            else:
+                moe.moe_forward(L, x_dev[b], d["w_router"], d["corr_bias"], d["w_gate_up"],
+                                d["w_down"], wsgu, wsd, out_dev[b], ws, stream=stream)
             ev["comp"][b].record(stream)
             with torch.cuda.stream(d2h_s):
                 d2h_s.wait_event(ev["comp"][b])
@@ -370,11 +390,193 @@ def gpu_arm(args, world, rank, local):
             "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
                     "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
-            "gpu_launches": moe.forward_kernel_count(L) * args.steps,
+            "gpu_launches": (moe.forward_prenorm_kernel_count(L) if args.prenorm
+                             else moe.forward_kernel_count(L)) * args.steps,
+            "clocks": clocks,
+        }
+        if args.prenorm:
+            # the block: post_attention_layernorm, then the layer
+            el_x = 2 if w.dtype == "bf16" else 4
+            nb = 2 * T * H * el_x
+            line["config"]["block"] = "rmsnorm prologue + layer"
+            line["op_ms"]["rmsnorm"] = norm_ms
+            line["rmsnorm_roofline"] = {"bound": "hbm", "achieved": nb / (norm_ms / 1e3) / 1e9,
+                                        "peak": hbm_peak, "unit": "GB/s",
+                                        "frac": nb / (norm_ms / 1e3) / 1e9 / hbm_peak,
+                                        "algorithmic_bytes": nb}
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, inputs)
+        print(json.dumps(line), flush=True)
+    finish(world)
+
+
+# ------------------------------------------------------------- dense layer
+DENSE_METRIC = "Inkling dense-MLP layer tokens/s and TFLOP/s (% of B200 bf16 peak / % HBM BW), 1 GPU"
+
+
+def dense_oracle_run(w, inputs, tokens_per_step: int, steps: int, warmup: int, threads: int):
+    import oracle
+    torch.set_num_threads(threads)
+    n_done, t_total = 0, 0.0
+    for i in range(warmup + steps):
+        tok = mw.dense_token_sample(w, tokens_per_step, seed_offset=1000 + i)
+        t0 = time.perf_counter()
+        oracle.dense_mlp(inputs["x"], inputs["w_gate_up"], inputs["w_down"], w.global_scale,
+                         tokens=tok)
+        dt = time.perf_counter() - t0
+        if i >= warmup:
+            n_done += tok.numel()
+            t_total += dt
+    return n_done / t_total, n_done, t_total
+
+
+def dense_reference_arm(args, world, rank):
+    w = mw.dense_by_name(args.workload)
+    if rank != 0:
+        return
+    inputs = mw.generate_dense(w)
+    threads = len(os.sched_getaffinity(0))
+    tokens_per_step = int(max(1, min(64, 480 // max(1, args.steps + args.warmup))))
+    tps, done, secs = dense_oracle_run(w, inputs, tokens_per_step, args.steps, args.warmup, threads)
+    line = {
+        "impl": "reference", "metric": DENSE_METRIC, "value": tps, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "H": w.H, "I": w.I,
+                   "tokens_per_step": tokens_per_step},
+        "tflops": tps * mw.dense_flops(w, 1) / 1e12,
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{tokens_per_step} seeded tokens per step of {w.name}"},
+        "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def dense_gpu_arm(args, world, rank, local):
+    import mixture_experts_feed_b200 as moe
+
+    w = mw.dense_by_name(args.workload)
+    inputs = mw.generate_dense(w)
+    if rank > 0:
+        g = torch.Generator().manual_seed(10_000 + rank)
+        inputs["x"] = torch.randn(w.T, w.H, generator=g).to(w.torch_dtype)
+    L = moe.DenseLayer.from_workload(w)
+    dev = torch.device("cuda", local)
+    d = {k: v.to(dev).contiguous() for k, v in inputs.items()}
+    stream = torch.cuda.current_stream(dev)
+    ws = moe.new_dense_workspace(L, device=dev)
+    out = torch.empty(w.T, w.H, dtype=w.torch_dtype, device=dev)
+
+    def step():
+        moe.moe_dense_mlp(L, d["x"], d["w_gate_up"], d["w_down"], out, ws, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    moe.read_device_status(ws, stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    clocks = clk.summary()
+    moe.read_device_status(ws, stream)
+    ms_step = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+
+    # end to end through the same call with host buffers (double-buffered as
+    # in the MoE arm: each step uploads its x and downloads its output)
+    x_host = inputs["x"].pin_memory()
+    out_host = [torch.empty(w.T, w.H, dtype=w.torch_dtype).pin_memory() for _ in range(2)]
+    x_dev = [d["x"], torch.empty_like(d["x"])]
+    out_dev = [out, torch.empty_like(out)]
+    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = {n: [torch.cuda.Event() for _ in range(2)] for n in ("h2d", "comp", "d2h")}
+
+    def e2e_steps(n):
+        for i in range(n):
+            b = i & 1
+            with torch.cuda.stream(h2d_s):
+                if i >= 2:
+                    h2d_s.wait_event(ev["comp"][b])
+                x_dev[b].copy_(x_host, non_blocking=True)
+                ev["h2d"][b].record(h2d_s)
+            stream.wait_event(ev["h2d"][b])
+            if i >= 2:
+                stream.wait_event(ev["d2h"][b])
+            moe.moe_dense_mlp(L, x_dev[b], d["w_gate_up"], d["w_down"], out_dev[b], ws, stream)
+            ev["comp"][b].record(stream)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(ev["comp"][b])
+                out_host[b].copy_(out_dev[b], non_blocking=True)
+                ev["d2h"][b].record(d2h_s)
+
+    e2e_steps(max(2, args.warmup // 2))
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    h2d_s.wait_event(e0)
+    e2e_steps(args.steps)
+    stream.wait_stream(d2h_s)
+    stream.wait_stream(h2d_s)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    moe.read_device_status(ws, stream)
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        el = 2 if w.dtype == "bf16" else 4
+        flops = mw.dense_flops(w)
+        # weights once; x read, h written and read, y (fp32) written and read,
+        # out written
+        nbytes = 3 * w.H * w.I * el + w.T * (w.H * el + 2 * w.I * el + 8 * w.H + w.H * el)
+        peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        s_step = ms_step / 1e3
+        if flops / nbytes >= peak * 1e12 / (hbm_peak * 1e9):
+            roof = {"bound": "tensor", "achieved": flops / s_step / 1e12, "peak": peak,
+                    "unit": "TFLOP/s", "peak_source": f"{peak_src} bf16_tflops_sustained"}
+        else:
+            roof = {"bound": "hbm", "achieved": nbytes / s_step / 1e9, "peak": hbm_peak,
+                    "unit": "GB/s", "peak_source": f"{peak_src} hbm_gbs"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["traffic"] = NCU_TRAFFIC_BYTES.get(w.name)
+        roof["algorithmic_bytes"] = nbytes
+        roof["algorithmic_flops"] = flops
+        line = {
+            "metric": DENSE_METRIC, "value": world * w.T / s_step, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32",
+            "data": "synthetic (seeded N(0,1) activations, N(0,0.02^2) weights, random init)",
+            "config": {"workload": w.name, "T": w.T, "H": w.H, "I": w.I,
+                       "global_scale": w.global_scale, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (weights %.2f GB)" % (3 * w.H * w.I * el / 1e9)},
+            "tflops": world * flops / s_step / 1e12,
+            "roofline": {"kernel": "dense gate_up + down GEMM launches of moe_dense_mlp (whole call timed)",
+                         **roof},
+            "e2e": {"value": world * w.T / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+                    "d2h_bytes_per_step": out_host[0].numel() * out_host[0].element_size()},
+            "gpu_launches": moe.dense_kernel_count(L) * args.steps,
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(w, inputs)
+            threads = len(os.sched_getaffinity(0))
+            n = int(max(4, min(w.T, 64)))
+            tps, done, secs = dense_oracle_run(w, inputs, n, 1, 0, threads)
+            line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": threads,
+                                    "kind": "oracle",
+                                    "sample": f"{done} seeded tokens of {w.name} (oracle fp64, {secs:.1f} s)"}
         print(json.dumps(line), flush=True)
     finish(world)
 
@@ -387,13 +589,17 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prenorm", action="store_true",
+                    help="time the feed-forward block: the RMSNorm prologue, then the MoE layer")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least three untimed warm-up steps
+    dense = args.workload in mw.DENSE_WORKLOADS
     if args.impl == "reference":
-        reference_arm(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+        arm = dense_reference_arm if dense else reference_arm
+        arm(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
         return
     world, rank, local = dist_setup(args)
-    gpu_arm(args, world, rank, local)
+    (dense_gpu_arm if dense else gpu_arm)(args, world, rank, local)
 
 
 if __name__ == "__main__":

@@ -213,6 +213,90 @@ moe_status_t moe_selftest_wait_timeout(void* workspace, size_t workspace_bytes, 
 /* Number of kernels moe_forward launches for this layer (for launch accounting). */
 int32_t moe_forward_kernel_count(const moe_layer_desc_t* desc);
 
+/* ------------------------------------------------------------------------
+ * The feed-forward block's input norm (InklingRMSNorm, "text" page; the
+ * decoder layer's post_attention_layernorm):
+ *   out[t, :] = x[t, :] / sqrt(mean_h x[t, h]^2 + eps) * weight
+ * over rows of H elements, rounded once (to nearest, ties to even) to
+ * `dtype`.  The page states fp32 variance accumulation; this library
+ * computes in fp64 and rounds once, so that the rounding (which decides the
+ * top-k selection downstream) equals the exact value's rounding except within
+ * ~1e-16 of a tie.  weight [H] has `dtype`; eps >= 0 (rms_norm_eps, 1e-6 by
+ * default).  x, out [T, H]; out may equal x.  H % 64 == 0.  T = 0 launches
+ * nothing.  Asynchronous on `stream`; no workspace.
+ * ---------------------------------------------------------------------- */
+moe_status_t moe_rmsnorm(int64_t num_tokens, int32_t hidden, moe_dtype_t dtype, float eps,
+                         const void* x, const void* weight, void* out, void* stream);
+
+/*
+ * moe_forward_prenorm — the block's norm followed by the MoE layer:
+ * moe_rmsnorm(x) into the workspace, then moe_forward on it.  Arguments as
+ * moe_forward plus norm_weight [H] (dtype) and norm_eps.  The residual add of
+ * the decoder block is not part of it.
+ */
+moe_status_t moe_forward_prenorm(const moe_layer_desc_t* desc, const void* x,
+                                 const void* norm_weight, float norm_eps, const float* w_router,
+                                 const float* corr_bias, const void* w_gate_up, const void* w_down,
+                                 const void* ws_gate_up, const void* ws_down,
+                                 const uint8_t* padding_mask, void* out, float* topk_w,
+                                 int32_t* topk_idx, float* shared_gamma, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/* Number of kernels moe_forward_prenorm launches (moe_forward's + 1). */
+int32_t moe_forward_prenorm_kernel_count(const moe_layer_desc_t* desc);
+
+/* ------------------------------------------------------------------------
+ * The dense feed-forward layer (InklingDenseMLP, "layers" page): the model's
+ * decoder layer that has a plain MLP instead of experts (dense_mlp_idx).  It
+ * keeps the checkpoint's fused interleaved gate/up projection:
+ *   out = global_scale * ( (silu(g) * u) @ w_down^T ),
+ *   [g_j, u_j] = rows 2j, 2j+1 of x @ w_gate_up^T
+ *   w_gate_up [2I, H] (row 2j = gate_j, row 2j+1 = up_j), w_down [H, I],
+ *   x and out [T, H] (leading dims flattened by the caller), all in `dtype`.
+ * I is dense_intermediate_size, else intermediate_size (InklingTextConfig).
+ * The pages hold global_scale as a parameter of the module without saying
+ * where it applies; it scales the output (in exact arithmetic the same as
+ * scaling silu(g) * u, which is where the kernels apply it).
+ * Same conventions as above; limits: H % 64 == 0, I % 64 == 0, T < 2^26.
+ * T = 0 returns MOE_OK without reading any pointer.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int64_t num_tokens;    /* T */
+  int32_t hidden;        /* H: hidden_size */
+  int32_t intermediate;  /* I */
+  moe_dtype_t dtype;     /* x, weights, out */
+  float global_scale;    /* finite */
+} moe_dense_desc_t;
+
+/* Workspace bytes for moe_dense_mlp(_prenorm): status word, h [T, I] in dtype,
+ * y [T, H] fp32, the normalised input [T, H] in dtype. */
+moe_status_t moe_dense_workspace_size(const moe_dense_desc_t* desc, size_t* bytes);
+
+/*
+ * moe_dense_mlp — InklingDenseMLP.forward.  bf16 layers run both projections
+ * on the tcgen05 tensor cores (bf16 operands, fp32 accumulation; h rounded
+ * to bf16, y kept fp32 and rounded once into out); fp32 layers run them in
+ * fp32 on the CUDA cores.  Workspace as for the MoE layer: initialise its
+ * status word once with moe_workspace_init().
+ */
+moe_status_t moe_dense_mlp(const moe_dense_desc_t* desc, const void* x, const void* w_gate_up,
+                           const void* w_down, void* out, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/* Number of kernels moe_dense_mlp launches for this layer. */
+int32_t moe_dense_kernel_count(const moe_dense_desc_t* desc);
+
+/* moe_dense_mlp_prenorm — moe_rmsnorm(x) into the workspace, then
+ * moe_dense_mlp on it (the dense layer's feed-forward block without its
+ * residual add).  norm_weight [H] in dtype, norm_eps >= 0. */
+moe_status_t moe_dense_mlp_prenorm(const moe_dense_desc_t* desc, const void* x,
+                                   const void* norm_weight, float norm_eps, const void* w_gate_up,
+                                   const void* w_down, void* out, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/* Number of kernels moe_dense_mlp_prenorm launches (moe_dense_mlp's + 1). */
+int32_t moe_dense_prenorm_kernel_count(const moe_dense_desc_t* desc);
+
 const char* moe_status_string(moe_status_t status);
 int32_t moe_version(void);
 

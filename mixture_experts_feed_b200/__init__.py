@@ -42,6 +42,13 @@ class LayerDesc(ctypes.Structure):
                 ("global_scale", ctypes.c_float)]
 
 
+class DenseDesc(ctypes.Structure):
+    """``moe_dense_desc_t``."""
+    _fields_ = [("num_tokens", ctypes.c_int64), ("hidden", ctypes.c_int32),
+                ("intermediate", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("global_scale", ctypes.c_float)]
+
+
 class MoEError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -66,9 +73,24 @@ LIB.moe_expert_ffn.argtypes = [_DESC] + [_P] * 13 + [ctypes.c_size_t, _P]
 LIB.moe_combine.argtypes = [_DESC, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 LIB.moe_forward.argtypes = [_DESC] + [_P] * 13 + [ctypes.c_size_t, _P]
 LIB.moe_selftest_wait_timeout.argtypes = [_P, ctypes.c_size_t, ctypes.c_uint32, _P]
+_DDESC = ctypes.POINTER(DenseDesc)
+LIB.moe_dense_workspace_size.argtypes = [_DDESC, ctypes.POINTER(ctypes.c_size_t)]
+LIB.moe_dense_mlp.argtypes = [_DDESC, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+LIB.moe_dense_kernel_count.restype = ctypes.c_int32
+LIB.moe_dense_kernel_count.argtypes = [_DDESC]
+LIB.moe_rmsnorm.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
+                            _P, _P, _P, _P]
+LIB.moe_forward_prenorm.argtypes = [_DESC, _P, _P, ctypes.c_float] + [_P] * 12 + [ctypes.c_size_t, _P]
+LIB.moe_dense_mlp_prenorm.argtypes = [_DDESC, _P, _P, ctypes.c_float, _P, _P, _P, _P,
+                                      ctypes.c_size_t, _P]
+LIB.moe_forward_prenorm_kernel_count.restype = ctypes.c_int32
+LIB.moe_forward_prenorm_kernel_count.argtypes = [_DESC]
+LIB.moe_dense_prenorm_kernel_count.restype = ctypes.c_int32
+LIB.moe_dense_prenorm_kernel_count.argtypes = [_DDESC]
 for _f in ("moe_workspace_size", "moe_workspace_init", "moe_read_device_status", "moe_route",
            "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_combine", "moe_forward",
-           "moe_selftest_wait_timeout"):
+           "moe_selftest_wait_timeout", "moe_dense_workspace_size", "moe_dense_mlp",
+           "moe_rmsnorm", "moe_forward_prenorm", "moe_dense_mlp_prenorm"):
     getattr(LIB, _f).restype = ctypes.c_int
 
 
@@ -95,6 +117,26 @@ class Layer:
     @staticmethod
     def from_workload(w) -> "Layer":
         return Layer(w.T, w.H, w.E, w.k, w.S, w.I, w.torch_dtype, w.route_scale, w.global_scale)
+
+
+@dataclass(frozen=True)
+class DenseLayer:
+    """Sizes of the dense feed-forward layer (``InklingDenseMLP``)."""
+    T: int
+    H: int
+    I: int
+    dtype: torch.dtype = torch.bfloat16
+    global_scale: float = 1.0
+
+    def desc(self) -> DenseDesc:
+        code = {torch.float32: MOE_F32, torch.bfloat16: MOE_BF16}.get(self.dtype)
+        if code is None:
+            raise ValueError(f"unsupported dtype {self.dtype}")
+        return DenseDesc(self.T, self.H, self.I, code, self.global_scale)
+
+    @staticmethod
+    def from_workload(w) -> "DenseLayer":
+        return DenseLayer(w.T, w.H, w.I, w.torch_dtype, w.global_scale)
 
 
 def _check(status: int, where: str) -> None:
@@ -254,6 +296,70 @@ def moe_forward(layer: Layer, x, w_router, corr_bias, w_gate_up, w_down, ws_gate
            "moe_forward")
 
 
+def _dtype_code(dtype: torch.dtype) -> int:
+    code = {torch.float32: MOE_F32, torch.bfloat16: MOE_BF16}.get(dtype)
+    if code is None:
+        raise ValueError(f"unsupported dtype {dtype}")
+    return code
+
+
+def moe_rmsnorm(x, weight, out, eps: float = 1e-6, stream=None):
+    """``InklingRMSNorm``: ``x`` [T, H] -> ``out`` [T, H] (may be ``x``)."""
+    if x.dim() != 2:
+        raise ValueError("x must be [T, H]")
+    T, H = x.shape
+    _expect(x, "x", (T, H), x.dtype)
+    _expect(weight, "weight", (H,), x.dtype)
+    _expect(out, "out", (T, H), x.dtype)
+    _check(LIB.moe_rmsnorm(T, H, _dtype_code(x.dtype), eps, _ptr(x), _ptr(weight), _ptr(out),
+                           _stream(stream)), "moe_rmsnorm")
+
+
+def moe_forward_prenorm(layer: Layer, x, norm_weight, norm_eps, w_router, corr_bias, w_gate_up,
+                        w_down, ws_gate_up, ws_down, out, ws, padding_mask=None, topk_w=None,
+                        topk_idx=None, shared_gamma=None, stream=None):
+    L = layer
+    _expect(norm_weight, "norm_weight", (L.H,), L.dtype)
+    _expect(x, "x", (L.T, L.H), L.dtype)
+    _expect(w_router, "w_router", (L.E + L.S, L.H), torch.float32)
+    _expect(corr_bias, "corr_bias", (L.E,), torch.float32)
+    _expect(w_gate_up, "w_gate_up", (L.E, 2 * L.I, L.H), L.dtype)
+    _expect(w_down, "w_down", (L.E, L.H, L.I), L.dtype)
+    _expect(ws_gate_up, "ws_gate_up", (L.S, 2 * L.I, L.H), L.dtype, allow_none=L.S == 0)
+    _expect(ws_down, "ws_down", (L.S, L.H, L.I), L.dtype, allow_none=L.S == 0)
+    _expect(out, "out", (L.T, L.H), L.dtype)
+    _expect(padding_mask, "padding_mask", (L.T,), torch.uint8, allow_none=True)
+    _expect(topk_w, "topk_w", (L.T, L.k), torch.float32, allow_none=True)
+    _expect(topk_idx, "topk_idx", (L.T, L.k), torch.int32, allow_none=True)
+    _expect(shared_gamma, "shared_gamma", (L.T, L.S), torch.float32, allow_none=True)
+    _check(LIB.moe_forward_prenorm(ctypes.byref(L.desc()), _ptr(x), _ptr(norm_weight), norm_eps,
+                                   _ptr(w_router), _ptr(corr_bias), _ptr(w_gate_up), _ptr(w_down),
+                                   _ptr(ws_gate_up), _ptr(ws_down), _ptr(padding_mask), _ptr(out),
+                                   _ptr(topk_w), _ptr(topk_idx), _ptr(shared_gamma), ws.data_ptr(),
+                                   ws.numel(), _stream(stream)), "moe_forward_prenorm")
+
+
+def moe_dense_mlp_prenorm(layer: "DenseLayer", x, norm_weight, norm_eps, w_gate_up, w_down, out,
+                          ws, stream=None):
+    L = layer
+    _expect(norm_weight, "norm_weight", (L.H,), L.dtype)
+    _expect(x, "x", (L.T, L.H), L.dtype)
+    _expect(w_gate_up, "w_gate_up", (2 * L.I, L.H), L.dtype)
+    _expect(w_down, "w_down", (L.H, L.I), L.dtype)
+    _expect(out, "out", (L.T, L.H), L.dtype)
+    _check(LIB.moe_dense_mlp_prenorm(ctypes.byref(L.desc()), _ptr(x), _ptr(norm_weight), norm_eps,
+                                     _ptr(w_gate_up), _ptr(w_down), _ptr(out), ws.data_ptr(),
+                                     ws.numel(), _stream(stream)), "moe_dense_mlp_prenorm")
+
+
+def forward_prenorm_kernel_count(layer: Layer) -> int:
+    return int(LIB.moe_forward_prenorm_kernel_count(ctypes.byref(layer.desc())))
+
+
+def dense_prenorm_kernel_count(layer: "DenseLayer") -> int:
+    return int(LIB.moe_dense_prenorm_kernel_count(ctypes.byref(layer.desc())))
+
+
 def selftest_wait_timeout(ws: torch.Tensor, limit_ms: int = 1000, stream=None) -> None:
     """Launch the stall-detection self-test (see the header); the next
     read_device_status() raises MoEError with MOE_ERR_TIMEOUT."""
@@ -265,14 +371,46 @@ def forward_kernel_count(layer: Layer) -> int:
     return int(LIB.moe_forward_kernel_count(ctypes.byref(layer.desc())))
 
 
+def dense_workspace_size(layer: DenseLayer) -> int:
+    n = ctypes.c_size_t(0)
+    _check(LIB.moe_dense_workspace_size(ctypes.byref(layer.desc()), ctypes.byref(n)),
+           "moe_dense_workspace_size")
+    return n.value
+
+
+def new_dense_workspace(layer: DenseLayer, device=None, stream=None) -> torch.Tensor:
+    """Allocate (with torch) and initialise a workspace for the dense ``layer``."""
+    ws = torch.empty(dense_workspace_size(layer), dtype=torch.uint8, device=device or "cuda")
+    _check(LIB.moe_workspace_init(ws.data_ptr(), ws.numel(), _stream(stream)), "moe_workspace_init")
+    return ws
+
+
+def moe_dense_mlp(layer: DenseLayer, x, w_gate_up, w_down, out, ws, stream=None):
+    L = layer
+    _expect(x, "x", (L.T, L.H), L.dtype)
+    _expect(w_gate_up, "w_gate_up", (2 * L.I, L.H), L.dtype)
+    _expect(w_down, "w_down", (L.H, L.I), L.dtype)
+    _expect(out, "out", (L.T, L.H), L.dtype)
+    _check(LIB.moe_dense_mlp(ctypes.byref(L.desc()), _ptr(x), _ptr(w_gate_up), _ptr(w_down),
+                             _ptr(out), ws.data_ptr(), ws.numel(), _stream(stream)),
+           "moe_dense_mlp")
+
+
+def dense_kernel_count(layer: DenseLayer) -> int:
+    return int(LIB.moe_dense_kernel_count(ctypes.byref(layer.desc())))
+
+
 class InklingMoE:
     """Device-resident weights of one layer plus its workspace; ``__call__``
     runs ``moe_forward`` on ``x`` of shape ``[..., H]`` (leading dims are
     flattened to tokens, as ``InklingMoE.forward`` does)."""
 
     def __init__(self, weights: dict, E: int, k: int, S: int, route_scale: float,
-                 global_scale: float = 1.0, device="cuda"):
+                 global_scale: float = 1.0, device="cuda", norm_weight=None, norm_eps: float = 1e-6):
         self.w = {n: t.to(device).contiguous() for n, t in weights.items() if n != "x"}
+        # optional post_attention_layernorm run first (moe_forward_prenorm)
+        self.norm_weight = None if norm_weight is None else norm_weight.to(device).contiguous()
+        self.norm_eps = norm_eps
         self.E, self.k, self.S = E, k, S
         self.H = self.w["w_router"].shape[1]
         self.I = self.w["w_down"].shape[2]
@@ -299,7 +437,52 @@ class InklingMoE:
         if padding_mask is not None:
             pm = padding_mask.reshape(-1).to(device=xt.device, dtype=torch.uint8).contiguous()
         w = self.w
-        moe_forward(L, xt, w["w_router"], w["corr_bias"], w["w_gate_up"], w["w_down"],
-                    w.get("ws_gate_up") if self.S else None, w.get("ws_down") if self.S else None,
-                    out, self._ws, padding_mask=pm, stream=stream)
+        wsgu = w.get("ws_gate_up") if self.S else None
+        wsd = w.get("ws_down") if self.S else None
+        if self.norm_weight is None:
+            moe_forward(L, xt, w["w_router"], w["corr_bias"], w["w_gate_up"], w["w_down"], wsgu,
+                        wsd, out, self._ws, padding_mask=pm, stream=stream)
+        else:
+            moe_forward_prenorm(L, xt, self.norm_weight, self.norm_eps, w["w_router"],
+                                w["corr_bias"], w["w_gate_up"], w["w_down"], wsgu, wsd, out,
+                                self._ws, padding_mask=pm, stream=stream)
+        return out.reshape(*lead, self.H)
+
+
+class InklingDenseMLP:
+    """Device-resident weights of the dense feed-forward layer plus its
+    workspace; ``__call__`` runs ``moe_dense_mlp`` on ``x`` of shape
+    ``[..., H]`` (leading dims flattened to tokens)."""
+
+    def __init__(self, w_gate_up: torch.Tensor, w_down: torch.Tensor, global_scale: float = 1.0,
+                 device="cuda", norm_weight=None, norm_eps: float = 1e-6):
+        # optional post_attention_layernorm run first (moe_dense_mlp_prenorm)
+        self.norm_weight = None if norm_weight is None else norm_weight.to(device).contiguous()
+        self.norm_eps = norm_eps
+        self.w_gate_up = w_gate_up.to(device).contiguous()
+        self.w_down = w_down.to(device).contiguous()
+        self.H = self.w_gate_up.shape[1]
+        self.I = self.w_down.shape[1]
+        self.dtype = self.w_gate_up.dtype
+        self.global_scale = global_scale
+        self.device = device
+        self._ws = None
+        self._ws_T = -1
+
+    def layer(self, T: int) -> DenseLayer:
+        return DenseLayer(T, self.H, self.I, self.dtype, self.global_scale)
+
+    def __call__(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+        lead = x.shape[:-1]
+        xt = x.reshape(-1, self.H).contiguous()
+        L = self.layer(xt.shape[0])
+        if self._ws is None or self._ws_T < L.T:
+            self._ws = new_dense_workspace(L, device=self.device, stream=stream)
+            self._ws_T = L.T
+        out = torch.empty_like(xt)
+        if self.norm_weight is None:
+            moe_dense_mlp(L, xt, self.w_gate_up, self.w_down, out, self._ws, stream=stream)
+        else:
+            moe_dense_mlp_prenorm(L, xt, self.norm_weight, self.norm_eps, self.w_gate_up,
+                                  self.w_down, out, self._ws, stream=stream)
         return out.reshape(*lead, self.H)

@@ -22,7 +22,8 @@ struct SimtParams {
   const int32_t* offsets;
   const int32_t* perm_slot;
   const float* topk_w;
-  const float* gamma;
+  const float* gamma;   // null: every shared row gets uniform_w (the dense layer)
+  float uniform_w;
   int32_t* status;
   int64_t T, a1_base, a1_stride;
   int E, S, K, N, ld_out, rows_cap;
@@ -101,7 +102,7 @@ __global__ void __launch_bounds__(SB_THREADS) grouped_gemm_simt_kernel(const Sim
               w = 0.0f;
             }
           } else {
-            w = p.gamma[static_cast<int64_t>(r) * p.S + gi.s];
+            w = p.gamma != nullptr ? p.gamma[static_cast<int64_t>(r) * p.S + gi.s] : p.uniform_w;
           }
           float2 hv;
           hv.x = w * (acc[i][0] / (1.0f + expf(-acc[i][0]))) * acc[i][1];
@@ -137,6 +138,7 @@ cudaError_t launch_expert_ffn_f32(const Layer& L, const void* x, const void* x_p
   g.out[0] = hf;
   g.out[1] = hf + Rk * L.I;
   g.offsets = offsets; g.perm_slot = perm_slot; g.topk_w = topk_w; g.gamma = gamma;
+  g.uniform_w = L.global_scale;
   g.status = status;
   g.T = L.T; g.a1_base = 0; g.a1_stride = 0;
   g.E = L.E; g.S = L.S; g.K = L.H; g.N = 2 * L.I; g.ld_out = L.I;
@@ -153,6 +155,7 @@ cudaError_t launch_expert_ffn_f32(const Layer& L, const void* x, const void* x_p
   d.out[0] = static_cast<float*>(y_routed);
   d.out[1] = static_cast<float*>(y_shared);
   d.offsets = offsets; d.perm_slot = perm_slot; d.topk_w = topk_w; d.gamma = gamma;
+  d.uniform_w = L.global_scale;
   d.status = status;
   d.T = L.T; d.a1_base = Rk; d.a1_stride = L.T;
   d.E = L.E; d.S = L.S; d.K = L.I; d.N = L.H; d.ld_out = L.H;

@@ -7,7 +7,9 @@
 //            ([g0, u0, g1, u1, ...], the fused gate_up_proj layout of the
 //            Inkling layers page, inkling_swiglu); the epilogue writes
 //            h = w * silu(g) * u in bf16, w the row's routing weight (routed
-//            rows: topk_w of the row's slot; shared rows: the token's gamma).
+//            rows: topk_w of the row's slot; shared rows: the token's gamma,
+//            or one uniform weight when no gamma is given: the dense layer,
+//            run as a single shared group, passes its global_scale).
 //   kDown:   the epilogue writes D in fp32 (the down projection); the rows
 //            stay fp32 until the recombination rounds the layer output once
 //            (rounding them to bf16 as well would put a correct pipeline at
@@ -86,7 +88,8 @@ struct alignas(64) GemmParams {
   const int32_t* offsets;     // [E+1]
   const int32_t* perm_slot;   // [rows] slot of each permuted row (kGateUp weights)
   const float* topk_w;        // [T*k]
-  const float* gamma;         // [T*S]
+  const float* gamma;         // [T*S], or null: every shared row gets uniform_w
+  float uniform_w;
   void* out[2];               // output of routed (0) and shared (1) groups
   int32_t* status;
   int64_t T;
@@ -426,7 +429,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             w = 0.0f;
           }
         } else {
-          w = p.gamma[static_cast<int64_t>(r) * p.S + gi.s];
+          w = p.gamma != nullptr ? p.gamma[static_cast<int64_t>(r) * p.S + gi.s] : p.uniform_w;
         }
       }
       const uint32_t t_row = t_lane + static_cast<uint32_t>(acc * BN);
@@ -574,13 +577,19 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   __nv_bfloat16* hb = static_cast<__nv_bfloat16*>(h);
 
   // ---------------- gate_up: [rows, H] x [2I, H]^T -> SwiGLU -> h [rows, I]
+  // With no routed rows (E == 0: the dense layer) the routed maps are never
+  // read; they are encoded over the shared operands so that every map is valid.
+  const bool routed = L.E > 0 && Rk > 0;
   GemmParams g{};
-  bool ok = encode_a(&g.tmA[0], x_perm, Rk, L.H) && encode_a(&g.tmA[1], x, L.T, L.H) &&
-            encode_b(&g.tmB[0], w_gate_up, L.E, 2 * L.I, L.H, BROWS);
+  bool ok = encode_a(&g.tmA[0], routed ? x_perm : x, routed ? Rk : L.T, L.H) &&
+            encode_a(&g.tmA[1], x, L.T, L.H);
+  if (ok && L.E > 0) ok = encode_b(&g.tmB[0], w_gate_up, L.E, 2 * L.I, L.H, BROWS);
   if (ok && L.S > 0) ok = encode_b(&g.tmB[1], ws_gate_up, L.S, 2 * L.I, L.H, BROWS);
-  else g.tmB[1] = g.tmB[0];
+  if (L.E == 0) g.tmB[0] = g.tmB[1];
+  if (L.S == 0) g.tmB[1] = g.tmB[0];
   if (!ok) { *map_error = true; return cudaErrorInvalidValue; }
   g.offsets = offsets; g.perm_slot = perm_slot; g.topk_w = topk_w; g.gamma = gamma;
+  g.uniform_w = L.global_scale;
   g.out[0] = hb;
   g.out[1] = hb + Rk * L.I;
   g.status = status;
@@ -597,12 +606,15 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
 
   // ---------------- down: h [rows, I] x [H, I]^T -> y [rows, H] (fp32)
   GemmParams d{};
-  ok = encode_a(&d.tmA[0], h, Rh, L.I) && encode_b(&d.tmB[0], w_down, L.E, L.H, L.I, BROWS);
+  ok = encode_a(&d.tmA[0], h, Rh, L.I);
+  if (ok && L.E > 0) ok = encode_b(&d.tmB[0], w_down, L.E, L.H, L.I, BROWS);
   d.tmA[1] = d.tmA[0];
   if (ok && L.S > 0) ok = encode_b(&d.tmB[1], ws_down, L.S, L.H, L.I, BROWS);
-  else d.tmB[1] = d.tmB[0];
+  if (L.E == 0) d.tmB[0] = d.tmB[1];
+  if (L.S == 0) d.tmB[1] = d.tmB[0];
   if (!ok) { *map_error = true; return cudaErrorInvalidValue; }
   d.offsets = offsets; d.perm_slot = perm_slot; d.topk_w = topk_w; d.gamma = gamma;
+  d.uniform_w = L.global_scale;
   d.out[0] = y_routed;
   d.out[1] = y_shared;
   d.status = status;

@@ -57,6 +57,10 @@ cudaError_t launch_expert_ffn_f32(const Layer& L, const void* x, const void* x_p
                                   void* h, void* y_routed, void* y_shared, int32_t* status,
                                   int num_sms, cudaStream_t stream);
 
+// rmsnorm.cu (out may alias x)
+cudaError_t launch_rmsnorm(int64_t T, int H, int dtype, float eps, const void* x,
+                           const void* weight, void* out, int num_sms, cudaStream_t stream);
+
 // combine.cu
 cudaError_t launch_combine(const Layer& L, const void* y_routed, const void* y_shared,
                            const int32_t* inv_perm, void* out, int32_t* status, int num_sms,

@@ -21,7 +21,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct WsLayout {
   size_t status, logits, wparts, counts, topk_w, topk_idx, gamma, offsets, perm_slot, inv_perm, x_perm,
-      h, y_routed, y_shared, total;
+      h, y_routed, y_shared, x_norm, total;
 };
 
 // Row stride of the router logits: E+S rounded up to 32 (whole 32-column
@@ -66,6 +66,7 @@ WsLayout ws_layout(const Layer& L) {
   w.h = take(Rh * L.I * elt);
   w.y_routed = take(Rk * L.H * 4);   // expert output rows stay fp32
   w.y_shared = take(T * L.S * L.H * 4);
+  w.x_norm = take(T * L.H * elt);    // moe_forward_prenorm: the normalised input
   w.total = off;
   return w;
 }
@@ -190,6 +191,128 @@ moe_status_t ffn_impl(const Layer& L, const void* x, const void* x_perm, const i
                                            num_sms(), stream));
 }
 
+// moe_forward with an optional RMSNorm prologue (norm_weight != null): the
+// normalised input goes to the workspace and feeds every later step.
+moe_status_t forward_checked(const moe_layer_desc_t* desc, const void* x, const void* norm_weight,
+                             float norm_eps, const float* w_router, const float* corr_bias,
+                             const void* w_gate_up, const void* w_down, const void* ws_gate_up,
+                             const void* ws_down, const uint8_t* padding_mask, void* out,
+                             float* topk_w, int32_t* topk_idx, float* shared_gamma,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  Layer L;
+  MOE_TRY(check_desc(desc, &L));
+  if (!aligned16(x) || !aligned16(w_router) || corr_bias == nullptr || !aligned16(w_gate_up) ||
+      !aligned16(w_down) || !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
+  if (L.S > 0 && (!aligned16(ws_gate_up) || !aligned16(ws_down))) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(L, workspace, workspace_bytes));
+  if (L.T == 0) return MOE_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const WsLayout w = ws_layout(L);
+  if (norm_weight != nullptr) {
+    void* xn = region<void>(workspace, w.x_norm);
+    MOE_TRY(cuda_status(launch_rmsnorm(L.T, L.H, L.dtype, norm_eps, x, norm_weight, xn, num_sms(), s)));
+    x = xn;
+  }
+  float* tw = topk_w ? topk_w : region<float>(workspace, w.topk_w);
+  int32_t* ti = topk_idx ? topk_idx : region<int32_t>(workspace, w.topk_idx);
+  float* sg = shared_gamma ? shared_gamma : region<float>(workspace, w.gamma);
+  int32_t* offsets = region<int32_t>(workspace, w.offsets);
+  int32_t* perm_slot = region<int32_t>(workspace, w.perm_slot);
+  int32_t* inv_perm = region<int32_t>(workspace, w.inv_perm);
+  void* x_perm = region<void>(workspace, w.x_perm);
+  void* y_routed = region<void>(workspace, w.y_routed);
+  void* y_shared = region<void>(workspace, w.y_shared);
+  MOE_TRY(route_impl(L, x, w_router, corr_bias, tw, ti, sg, workspace, s));
+  MOE_TRY(permute_impl(L, ti, padding_mask, x, offsets, perm_slot, inv_perm, x_perm, workspace, s));
+  MOE_TRY(ffn_impl(L, x, x_perm, offsets, perm_slot, tw, sg, w_gate_up, w_down, ws_gate_up,
+                   ws_down, y_routed, y_shared, workspace, s));
+  return cuda_status(launch_combine(L, y_routed, y_shared, inv_perm, out,
+                                    region<int32_t>(workspace, w.status), num_sms(), s));
+}
+
+// ------------------------------------------------------------ dense layer
+// InklingDenseMLP runs through the expert GEMMs as one shared group over all
+// T tokens (E = 0, S = 1) whose per-token weight is global_scale, then the
+// recombination with k = 0 rounds y into out.
+struct DenseWs {
+  size_t status, h, y, x_norm, total;
+};
+
+moe_status_t check_dense(const moe_dense_desc_t* d, Layer* L) {
+  if (d == nullptr) return MOE_ERR_INVALID_ARG;
+  if (d->num_tokens < 0 || d->hidden <= 0 || d->intermediate <= 0) return MOE_ERR_INVALID_ARG;
+  if (d->dtype != MOE_F32 && d->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (!isfinite(d->global_scale)) return MOE_ERR_INVALID_ARG;
+  if (d->hidden % 64 != 0 || d->intermediate % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  if (d->num_tokens >= (int64_t{1} << 26)) return MOE_ERR_UNSUPPORTED;
+  L->T = d->num_tokens;
+  L->H = d->hidden;
+  L->E = 0;
+  L->k = 0;
+  L->S = 1;
+  L->I = d->intermediate;
+  L->dtype = d->dtype;
+  L->route_scale = 1.0f;
+  L->global_scale = d->global_scale;
+  return MOE_OK;
+}
+
+DenseWs dense_ws_layout(const Layer& L) {
+  DenseWs w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes > 0 ? bytes : 1, kRegionAlign);
+    return o;
+  };
+  const size_t elt = L.dtype == MOE_BF16 ? 2 : 4;
+  const size_t T = static_cast<size_t>(L.T);
+  w.status = take(kStatusBytes);
+  w.h = take(T * L.I * elt);
+  w.y = take(T * L.H * 4);
+  w.x_norm = take(T * L.H * elt);    // moe_dense_mlp_prenorm: the normalised input
+  w.total = off;
+  return w;
+}
+
+moe_status_t dense_checked(const moe_dense_desc_t* desc, const void* x, const void* norm_weight,
+                           float norm_eps, const void* w_gate_up, const void* w_down, void* out,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  Layer L;
+  MOE_TRY(check_dense(desc, &L));
+  if (L.T == 0) return MOE_OK;   // nothing to read or write
+  if (!aligned16(x) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255) != 0)
+    return MOE_ERR_INVALID_ARG;
+  const DenseWs w = dense_ws_layout(L);
+  if (workspace_bytes < w.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* status = region<int32_t>(workspace, w.status);
+  void* h = region<void>(workspace, w.h);
+  float* y = region<float>(workspace, w.y);
+  if (norm_weight != nullptr) {
+    void* xn = region<void>(workspace, w.x_norm);
+    MOE_TRY(cuda_status(launch_rmsnorm(L.T, L.H, L.dtype, norm_eps, x, norm_weight, xn, num_sms(), s)));
+    x = xn;
+  }
+  // one shared group: the routed operands are never read (E = 0, k = 0)
+  if (L.dtype == MOE_BF16) {
+    bool map_error = false;
+    const cudaError_t e = launch_expert_ffn_bf16(L, x, x, nullptr, nullptr, nullptr, nullptr,
+                                                 nullptr, nullptr, w_gate_up, w_down, h, y, y,
+                                                 status, num_sms(), s, &map_error);
+    if (map_error) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(cuda_status(e));
+  } else {
+    MOE_TRY(cuda_status(launch_expert_ffn_f32(L, x, x, nullptr, nullptr, nullptr, nullptr,
+                                              nullptr, nullptr, w_gate_up, w_down, h, y, y,
+                                              status, num_sms(), s)));
+  }
+  return cuda_status(launch_combine(L, y, y, nullptr, out, status, num_sms(), s));
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -297,31 +420,34 @@ moe_status_t moe_forward(const moe_layer_desc_t* desc, const void* x, const floa
                          const void* ws_gate_up, const void* ws_down, const uint8_t* padding_mask,
                          void* out, float* topk_w, int32_t* topk_idx, float* shared_gamma,
                          void* workspace, size_t workspace_bytes, void* stream) {
-  Layer L;
-  MOE_TRY(check_desc(desc, &L));
-  if (!aligned16(x) || !aligned16(w_router) || corr_bias == nullptr || !aligned16(w_gate_up) ||
-      !aligned16(w_down) || !aligned16(out))
+  return forward_checked(desc, x, nullptr, 0.0f, w_router, corr_bias, w_gate_up, w_down,
+                         ws_gate_up, ws_down, padding_mask, out, topk_w, topk_idx, shared_gamma,
+                         workspace, workspace_bytes, stream);
+}
+
+moe_status_t moe_forward_prenorm(const moe_layer_desc_t* desc, const void* x,
+                                 const void* norm_weight, float norm_eps, const float* w_router,
+                                 const float* corr_bias, const void* w_gate_up, const void* w_down,
+                                 const void* ws_gate_up, const void* ws_down,
+                                 const uint8_t* padding_mask, void* out, float* topk_w,
+                                 int32_t* topk_idx, float* shared_gamma, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (!aligned16(norm_weight) || !isfinite(norm_eps) || norm_eps < 0.0f) return MOE_ERR_INVALID_ARG;
+  return forward_checked(desc, x, norm_weight, norm_eps, w_router, corr_bias, w_gate_up, w_down,
+                         ws_gate_up, ws_down, padding_mask, out, topk_w, topk_idx, shared_gamma,
+                         workspace, workspace_bytes, stream);
+}
+
+moe_status_t moe_rmsnorm(int64_t num_tokens, int32_t hidden, moe_dtype_t dtype, float eps,
+                         const void* x, const void* weight, void* out, void* stream) {
+  if (num_tokens < 0 || hidden <= 0 || (dtype != MOE_F32 && dtype != MOE_BF16) ||
+      !isfinite(eps) || eps < 0.0f)
     return MOE_ERR_INVALID_ARG;
-  if (L.S > 0 && (!aligned16(ws_gate_up) || !aligned16(ws_down))) return MOE_ERR_INVALID_ARG;
-  MOE_TRY(check_ws(L, workspace, workspace_bytes));
-  if (L.T == 0) return MOE_OK;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const WsLayout w = ws_layout(L);
-  float* tw = topk_w ? topk_w : region<float>(workspace, w.topk_w);
-  int32_t* ti = topk_idx ? topk_idx : region<int32_t>(workspace, w.topk_idx);
-  float* sg = shared_gamma ? shared_gamma : region<float>(workspace, w.gamma);
-  int32_t* offsets = region<int32_t>(workspace, w.offsets);
-  int32_t* perm_slot = region<int32_t>(workspace, w.perm_slot);
-  int32_t* inv_perm = region<int32_t>(workspace, w.inv_perm);
-  void* x_perm = region<void>(workspace, w.x_perm);
-  void* y_routed = region<void>(workspace, w.y_routed);
-  void* y_shared = region<void>(workspace, w.y_shared);
-  MOE_TRY(route_impl(L, x, w_router, corr_bias, tw, ti, sg, workspace, s));
-  MOE_TRY(permute_impl(L, ti, padding_mask, x, offsets, perm_slot, inv_perm, x_perm, workspace, s));
-  MOE_TRY(ffn_impl(L, x, x_perm, offsets, perm_slot, tw, sg, w_gate_up, w_down, ws_gate_up,
-                   ws_down, y_routed, y_shared, workspace, s));
-  return cuda_status(launch_combine(L, y_routed, y_shared, inv_perm, out,
-                                    region<int32_t>(workspace, w.status), num_sms(), s));
+  if (hidden % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return MOE_OK;
+  if (!aligned16(x) || !aligned16(weight) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_rmsnorm(num_tokens, hidden, dtype, eps, x, weight, out, num_sms(),
+                                    static_cast<cudaStream_t>(stream)));
 }
 
 int32_t moe_forward_kernel_count(const moe_layer_desc_t* desc) {
@@ -332,6 +458,49 @@ int32_t moe_forward_kernel_count(const moe_layer_desc_t* desc) {
   // T > 128: CTA-pair launch + single-CTA launch each); combine.
   const int experts = L.dtype == MOE_BF16 ? (L.T > 128 ? 4 : 2) : 2;
   return (L.dtype == MOE_BF16 ? 3 : 2) + 4 + experts + 1;
+}
+
+moe_status_t moe_dense_workspace_size(const moe_dense_desc_t* desc, size_t* bytes) {
+  Layer L;
+  MOE_TRY(check_dense(desc, &L));
+  if (bytes == nullptr) return MOE_ERR_INVALID_ARG;
+  *bytes = dense_ws_layout(L).total;
+  return MOE_OK;
+}
+
+moe_status_t moe_dense_mlp(const moe_dense_desc_t* desc, const void* x, const void* w_gate_up,
+                           const void* w_down, void* out, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  return dense_checked(desc, x, nullptr, 0.0f, w_gate_up, w_down, out, workspace, workspace_bytes,
+                       stream);
+}
+
+moe_status_t moe_dense_mlp_prenorm(const moe_dense_desc_t* desc, const void* x,
+                                   const void* norm_weight, float norm_eps, const void* w_gate_up,
+                                   const void* w_down, void* out, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  if (!aligned16(norm_weight) || !isfinite(norm_eps) || norm_eps < 0.0f) return MOE_ERR_INVALID_ARG;
+  return dense_checked(desc, x, norm_weight, norm_eps, w_gate_up, w_down, out, workspace,
+                       workspace_bytes, stream);
+}
+
+int32_t moe_dense_kernel_count(const moe_dense_desc_t* desc) {
+  Layer L;
+  if (check_dense(desc, &L) != MOE_OK || L.T == 0) return 0;
+  // gate_up + down (bf16 with T > 128: CTA-pair launch + single-CTA launch
+  // each), then the rounding pass
+  const int gemms = L.dtype == MOE_BF16 ? (L.T > 128 ? 4 : 2) : 2;
+  return gemms + 1;
+}
+
+int32_t moe_dense_prenorm_kernel_count(const moe_dense_desc_t* desc) {
+  const int32_t n = moe_dense_kernel_count(desc);
+  return n > 0 ? n + 1 : 0;   // + the RMSNorm prologue
+}
+
+int32_t moe_forward_prenorm_kernel_count(const moe_layer_desc_t* desc) {
+  const int32_t n = moe_forward_kernel_count(desc);
+  return n > 0 ? n + 1 : 0;   // + the RMSNorm prologue
 }
 
 const char* moe_status_string(moe_status_t status) {

@@ -338,3 +338,17 @@ def dense_token_sample(w: DenseWorkload, n: int, seed_offset: int = 0) -> torch.
     g = torch.Generator(device="cpu")
     g.manual_seed(w.seed * 31 + 977 + seed_offset)
     return torch.randperm(w.T, generator=g)[:n].sort().values
+
+
+# ----------------------------------------------------------- norm weights
+def norm_weight(H: int, seed: int, dtype: torch.dtype = torch.bfloat16,
+                spread: float = 0.1) -> torch.Tensor:
+    """A learned-looking RMSNorm scale: 1 + spread * N(0, 1) per channel (the
+    module initialises it to ones; a spread keeps a missing weight visible)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed * 7919 + 17)
+    return (1.0 + spread * torch.randn(H, generator=g, dtype=torch.float32)).to(dtype)
+
+
+# rms_norm_eps of InklingTextConfig (1e-6), as the float32 the C ABI receives
+RMS_NORM_EPS = float(torch.tensor(1e-6, dtype=torch.float32))

@@ -118,3 +118,68 @@ def test_binding_checks_shapes_on_host():
     x = torch.zeros(4, 64)   # wrong H, on CPU: rejected before the C call
     with pytest.raises(ValueError):
         moe.moe_combine(L, x, x, torch.zeros(8, dtype=torch.int32), x, torch.zeros(16, dtype=torch.uint8))
+
+
+# ------------------------------------------------------------- dense layer
+def test_dense_desc_layout_and_sizes():
+    assert ctypes.sizeof(moe.DenseDesc) == 24     # int64 + 3 x int32 + float
+    assert moe.DenseDesc.global_scale.offset == 20
+    for w in mw.DENSE_WORKLOADS.values():
+        L = moe.DenseLayer.from_workload(w)
+        el = 4 if w.dtype == "f32" else 2
+        assert moe.dense_workspace_size(L) >= el * w.T * w.I + 4 * w.T * w.H
+        gemms = (4 if w.T > 128 else 2) if w.dtype == "bf16" else 2
+        assert moe.dense_kernel_count(L) == gemms + 1
+
+
+def _dense_status(T=8, H=64, I=64, dtype=moe.MOE_BF16, gs=1.0, ws_bytes=None, ptr=256):
+    d = moe.DenseDesc(T, H, I, dtype, gs)
+    if ws_bytes is None:
+        ws_bytes = 1 << 40     # large enough for any valid desc; argument checks come first
+    # aligned fake pointers: every call below returns on the host before any
+    # CUDA call, so nothing is dereferenced
+    return moe.LIB.moe_dense_mlp(ctypes.byref(d), ptr, ptr, ptr, ptr, 4096, ws_bytes, None)
+
+
+def test_dense_host_checks():
+    assert _dense_status(H=100) == 2                      # H % 64
+    assert _dense_status(I=96) == 2                       # I % 64
+    assert _dense_status(T=-1) == 1
+    assert _dense_status(gs=float("nan")) == 1
+    assert _dense_status(dtype=7) == 1
+    assert _dense_status(ws_bytes=100) == 3               # workspace too small
+    assert _dense_status(ptr=8) == 1                      # misaligned operand
+    assert _dense_status(T=0, ptr=0) == 0                 # T = 0: nothing read
+    assert moe.LIB.moe_dense_workspace_size(None, None) == 1
+
+
+def test_dense_binding_checks_shapes():
+    L = moe.DenseLayer(4, 64, 64)
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        moe.moe_dense_mlp(L, x, torch.zeros(64, 64, dtype=torch.bfloat16),     # not [2I, H]
+                          torch.zeros(64, 64, dtype=torch.bfloat16), x, None)
+
+
+def declared_arity():
+    """Parameter count of every function the header declares."""
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for name, params in re.findall(r"\b(moe_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", src):
+        params = params.strip()
+        out[name] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argtypes_match_the_header():
+    """Every ctypes prototype the binding sets has the header's parameter
+    count (a missing argument shifts the rest, which ctypes does not catch)."""
+    arity = declared_arity()
+    assert len(arity) == len(declared_functions())
+    for name, n in arity.items():
+        fn = getattr(moe.LIB, name)
+        if fn.argtypes is None:
+            assert n == 0, f"{name}: no ctypes prototype for {n} parameters"
+        else:
+            assert len(fn.argtypes) == n, f"{name}: {len(fn.argtypes)} argtypes, header has {n}"

@@ -1,0 +1,101 @@
+"""GPU parity of the dense feed-forward layer (InklingDenseMLP) through the
+C ABI (moe_dense_mlp) against the CPU fp64 oracle (oracle.dense_mlp).
+
+Bars as for the MoE layer: max|gpu - oracle| <= 2e-2 x RMS (bf16) or
+1e-4 x RMS (fp32), element by element; small shapes span several tiles with
+ragged tails; the model-sized layer runs at full size with the oracle on a
+seeded token sample.
+"""
+from __future__ import annotations
+
+import pytest
+import torch
+
+import moe_workloads as mw
+import oracle
+from moe_gpu_helpers import check_output, to_device
+
+pytestmark = pytest.mark.gpu
+
+try:
+    import mixture_experts_feed_b200 as moe
+except ImportError:   # collected on CPU-only machines too; the gpu marker deselects
+    moe = None
+
+
+def run_dense(w, inputs, d=None):
+    L = moe.DenseLayer.from_workload(w)
+    d = d or to_device(inputs)
+    ws = moe.new_dense_workspace(L)
+    out = torch.empty(w.T, w.H, dtype=w.torch_dtype, device="cuda")
+    moe.moe_dense_mlp(L, d["x"], d["w_gate_up"], d["w_down"], out, ws)
+    torch.cuda.synchronize()
+    moe.read_device_status(ws)
+    return out.cpu()
+
+
+SMALL = [
+    # T, H, I, dtype, global_scale      what it covers
+    (300, 512, 640, "bf16", 1.0),       # ragged T (3 m-tiles: single CTAs), gate_up N = 1280
+    (517, 384, 320, "bf16", 0.5),       # 5 m-tiles, down N = 384 (1.5 tiles), scale 0.5
+    (1024, 256, 512, "bf16", 2.0),      # 8 m-tiles: CTA pairs
+    (1, 128, 64, "bf16", 1.0),          # a single token
+    (129, 128, 192, "bf16", 1.0),       # 2 m-tiles, the second one row
+    (96, 128, 192, "f32", 1.0),         # fp32 layer (CUDA cores)
+    (77, 192, 128, "f32", 1.5),
+]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=[f"T{s[0]}-H{s[1]}-I{s[2]}-{s[3]}-gs{s[4]}" for s in SMALL])
+def test_dense_small_shapes(shape):
+    T, H, I, dtype, gs = shape
+    w = mw.dense_tiny(T=T, H=H, I=I, dtype=dtype, global_scale=gs, seed=31 + T)
+    inputs = mw.generate_dense(w, threads=4)
+    out = run_dense(w, inputs)
+    ref = oracle.dense_mlp(inputs["x"], inputs["w_gate_up"], inputs["w_down"], gs)
+    check_output(out, ref, w.torch_dtype, "dense out", strict=False)
+
+
+@pytest.mark.parametrize("name", list(mw.DENSE_WORKLOADS))
+def test_dense_workloads(name):
+    w = mw.dense_by_name(name)
+    inputs = mw.generate_dense(w)
+    d = to_device(inputs)
+    out = run_dense(w, inputs, d)
+    tokens = None
+    if w.T > 1024:   # a seeded token sample (the full fp64 layer would take minutes)
+        tokens = torch.cat([torch.tensor([0, w.T - 1]), mw.dense_token_sample(w, 30)]).unique()
+    ref = oracle.dense_mlp(inputs["x"], inputs["w_gate_up"], inputs["w_down"], w.global_scale,
+                           tokens=tokens)
+    got = out if tokens is None else out[tokens]
+    # the plain 2e-2 x RMS bound at the model's sizes; the small shapes get half
+    # a bf16 ulp of the exact value on top (their outputs reach 5 x RMS, where
+    # the final rounding alone costs 2^-8 x 5 = 2% of RMS)
+    rel = check_output(got, ref, w.torch_dtype, f"{name} out", strict=w.H >= 2048)
+    print(f"{name}: max|err|/RMS = {rel:.4f}")
+
+
+def test_dense_module_leading_dims_and_determinism():
+    w = mw.dense_tiny(T=300, H=256, I=320, dtype="bf16", seed=77)
+    inputs = mw.generate_dense(w)
+    mlp = moe.InklingDenseMLP(inputs["w_gate_up"], inputs["w_down"], global_scale=1.0)
+    x = inputs["x"].cuda()
+    flat = mlp(x)
+    shaped = mlp(x.reshape(3, 100, w.H))
+    assert shaped.shape == (3, 100, w.H)
+    assert torch.equal(shaped.reshape(-1, w.H), flat)
+    assert torch.equal(mlp(x), flat)            # same inputs, same bits
+    ref = oracle.dense_mlp(inputs["x"].reshape(3, 100, w.H), inputs["w_gate_up"],
+                           inputs["w_down"], 1.0)
+    check_output(shaped.cpu(), ref, torch.bfloat16, "module out", strict=False)
+
+
+def test_dense_empty_batch():
+    L = moe.DenseLayer(0, 256, 320)
+    ws = moe.new_dense_workspace(L)
+    x = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
+    wgu = torch.zeros(640, 256, dtype=torch.bfloat16, device="cuda")
+    wd = torch.zeros(256, 320, dtype=torch.bfloat16, device="cuda")
+    moe.moe_dense_mlp(L, x, wgu, wd, torch.empty_like(x), ws)
+    torch.cuda.synchronize()
+    moe.read_device_status(ws)
