@@ -3,18 +3,29 @@
 //   out[t, :] = x[t, :] / sqrt(mean_h x[t, h]^2 + eps) * weight
 // rounded once to the input dtype.  The arithmetic is fp64: squares of bf16
 // or fp32 values are exact in fp64, the row sum carries ~1e-16 relative
-// error, and fp64 square root and division are correctly rounded, so the
-// rounded result is the exact value's rounding except within ~1e-16 of a
-// tie.  (The page states fp32 variance accumulation; fp64 is at least that,
-// and it makes the bf16 rounding, which decides the top-k selection
-// downstream, reproducible.)  The rounding to bf16 is done here on the fp64
-// bit pattern, round to nearest with ties to even, in one step.
+// error, and the row's 1/sqrt(mean + eps) is one correctly rounded fp64
+// square root and division, so the rounded result is the exact value's
+// rounding except within ~1e-16 of a tie.  (The page states fp32 variance
+// accumulation; fp64 is at least that, and it makes the bf16 rounding, which
+// decides the top-k selection downstream, reproducible.)  The rounding to
+// bf16 is done here on the fp64 bit pattern, round to nearest with ties to
+// even, in one step.
 //
-// One block of 256 threads per token row, 16-byte vectors along the row:
-// pass 1 sums the squares (warp shuffles, then the 8 warp sums in a fixed
-// order), pass 2 re-reads the row (L1/L2) and writes the result.  HBM-bound:
-// 2 x dtype bytes per element.  `out` may alias `x` (each thread reads a
-// vector in pass 2 before it writes the same vector).
+// One warp per token row, 16-byte vectors along the row: pass 1 streams
+// the row and sums the squares in fp64 (a lane's own elements in order, then
+// a butterfly across the warp, which leaves the same sum in every lane),
+// pass 2 streams it again (from L1/L2) and writes the result.  No block-wide
+// barrier, so every resident warp keeps a row in flight.  Each element is
+// scaled by the row's 1/s, s = sqrt(mean + eps), computed once per row in
+// fp64.  bf16 layers: x * weight is exact in fp32 (two 8-bit significands);
+// y32 = (x * weight) * fp32(1/s) is within 2^-23 |y| (under 2 fp32 ulps) of
+// the exact y, so when y32 is at least 3 ulps from a bf16 rounding tie it
+// rounds like y, and it is rounded directly; otherwise (about 1 element in
+// 8000) y is formed in fp64 and rounded from there.  fp32 layers multiply in
+// fp64.  Against x / s * weight in fp64 the result differs only within
+// ~1e-16 of a tie.  HBM-bound: 2 x dtype bytes per element.  `out` may alias
+// `x` (a lane writes a vector only after reading it, and pass 1 of a row
+// ends before its pass 2 starts).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -50,73 +61,80 @@ __device__ __forceinline__ uint16_t bf16_bits_rne(double y) {
 struct Bf16Row {
   using Vec = uint4;                      // 8 bf16
   static constexpr int V = 8;
-  __device__ static void unpack(const Vec& q, double (&d)[V]) {
+  __device__ static double sumsq(const Vec& q) {
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    double acc = 0.0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      d[2 * i] = static_cast<double>(__uint_as_float(w[i] << 16));
-      d[2 * i + 1] = static_cast<double>(__uint_as_float(w[i] & 0xFFFF0000u));
+      const double a = __uint_as_float(w[i] << 16), b = __uint_as_float(w[i] & 0xFFFF0000u);
+      acc = fma(a, a, acc);              // squares of bf16 values are exact
+      acc = fma(b, b, acc);
     }
+    return acc;
   }
-  __device__ static Vec pack(const double (&y)[V]) {
-    uint32_t w[4];
+  // bf16 bits of p * inv (p = x * weight, exact in fp32)
+  __device__ static uint32_t one(float p, float inv32, double inv) {
+    const float y32 = p * inv32;
+    const uint32_t b = __float_as_uint(y32);
+    const int from_tie = static_cast<int>(b & 0xFFFFu) - 0x8000;
+    if ((from_tie >= -3 && from_tie <= 3) || fabsf(y32) < 0x1p-120f)
+      return bf16_bits_rne(static_cast<double>(p) * inv);
+    return (b + 0x8000u) >> 16;          // not a tie: round to nearest
+  }
+  __device__ static Vec scale(const Vec& q, const Vec& g, float inv32, double inv) {
+    const uint32_t xw[4] = {q.x, q.y, q.z, q.w}, gw[4] = {g.x, g.y, g.z, g.w};
+    uint32_t o[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      w[i] = static_cast<uint32_t>(bf16_bits_rne(y[2 * i])) |
-             (static_cast<uint32_t>(bf16_bits_rne(y[2 * i + 1])) << 16);
-    return make_uint4(w[0], w[1], w[2], w[3]);
+    for (int i = 0; i < 4; ++i) {
+      const float lo = __uint_as_float(xw[i] << 16) * __uint_as_float(gw[i] << 16);
+      const float hi = __uint_as_float(xw[i] & 0xFFFF0000u) * __uint_as_float(gw[i] & 0xFFFF0000u);
+      o[i] = one(lo, inv32, inv) | (one(hi, inv32, inv) << 16);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
   }
 };
 
 struct F32Row {
   using Vec = float4;
   static constexpr int V = 4;
-  __device__ static void unpack(const Vec& q, double (&d)[V]) {
-    d[0] = q.x; d[1] = q.y; d[2] = q.z; d[3] = q.w;
+  __device__ static double sumsq(const Vec& q) {
+    double acc = static_cast<double>(q.x) * q.x;   // squares of fp32 values are exact in fp64
+    acc = fma(static_cast<double>(q.y), q.y, acc);
+    acc = fma(static_cast<double>(q.z), q.z, acc);
+    return fma(static_cast<double>(q.w), q.w, acc);
   }
-  __device__ static Vec pack(const double (&y)[V]) {
-    return make_float4(__double2float_rn(y[0]), __double2float_rn(y[1]),
-                       __double2float_rn(y[2]), __double2float_rn(y[3]));
+  __device__ static Vec scale(const Vec& q, const Vec& g, float, double inv) {
+    return make_float4(__double2float_rn(static_cast<double>(q.x) * g.x * inv),
+                       __double2float_rn(static_cast<double>(q.y) * g.y * inv),
+                       __double2float_rn(static_cast<double>(q.z) * g.z * inv),
+                       __double2float_rn(static_cast<double>(q.w) * g.w * inv));
   }
 };
 
 template <typename R>
 __global__ void __launch_bounds__(kThreads)
-    rmsnorm_kernel(const void* __restrict__ x_, const void* __restrict__ w_, void* out_, int64_t T,
-                   int H, double eps) {
+    rmsnorm_kernel(const void* x_, const void* __restrict__ w_, void* out_, int64_t T, int H,
+                   double eps) {
   using Vec = typename R::Vec;
   const Vec* x = static_cast<const Vec*>(x_);
   const Vec* w = static_cast<const Vec*>(w_);
   Vec* out = static_cast<Vec*>(out_);
   const int nv = H / R::V;
-  __shared__ double s_warp[kThreads / 32];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5); t < T;
+       t += warps) {
     const Vec* row = x + t * nv;
     double acc = 0.0;
-    for (int v = threadIdx.x; v < nv; v += kThreads) {
-      double d[R::V];
-      R::unpack(row[v], d);
-#pragma unroll
-      for (int i = 0; i < R::V; ++i) acc = fma(d[i], d[i], acc);   // d*d exact
-    }
+#pragma unroll 4
+    for (int v = lane; v < nv; v += 32) acc += R::sumsq(row[v]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) s_warp[warp] = acc;
-    __syncthreads();
-    double ss = 0.0;
-#pragma unroll
-    for (int i = 0; i < kThreads / 32; ++i) ss += s_warp[i];      // same order in every thread
-    const double s = sqrt(ss / H + eps);
-    for (int v = threadIdx.x; v < nv; v += kThreads) {
-      double d[R::V], g[R::V], y[R::V];
-      R::unpack(row[v], d);
-      R::unpack(w[v], g);
-#pragma unroll
-      for (int i = 0; i < R::V; ++i) y[i] = d[i] / s * g[i];
-      out[t * nv + v] = R::pack(y);
-    }
-    __syncthreads();   // s_warp is rewritten for the next row
+    const double inv = 1.0 / sqrt(acc / H + eps);
+    const float inv32 = __double2float_rn(inv);
+    Vec* orow = out + t * nv;
+#pragma unroll 4
+    for (int v = lane; v < nv; v += 32) orow[v] = R::scale(row[v], w[v], inv32, inv);
   }
 }
 
@@ -125,7 +143,9 @@ __global__ void __launch_bounds__(kThreads)
 cudaError_t launch_rmsnorm(int64_t T, int H, int dtype, float eps, const void* x,
                            const void* weight, void* out, int num_sms, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(T, static_cast<int64_t>(num_sms) * 8));
+  // one warp per row, 8 rows per block, up to 8 blocks per SM
+  const int64_t blocks = (T + kThreads / 32 - 1) / (kThreads / 32);
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(blocks, static_cast<int64_t>(num_sms) * 8));
   if (dtype == MOE_BF16)
     rmsnorm_kernel<Bf16Row><<<grid, kThreads, 0, stream>>>(x, weight, out, T, H, eps);
   else
