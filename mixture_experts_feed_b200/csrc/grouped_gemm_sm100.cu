@@ -97,7 +97,8 @@ struct alignas(64) GemmParams {
   int E, S, K, N;
   int ld_out;                 // output row length in elements
   int rows_cap;               // rows of the routed A operand (bound of offsets)
-  int ksplit;                 // kRouter: K-range splits (each writes its own partial)
+  int ksplit;                 // kRouter, kDown: K-range splits (each writes its own partial)
+  int bn;                     // single-CTA expert launches: n-tile width (32..256, multiple of 32)
   int64_t split_stride;       // kRouter: elements between partial outputs
 };
 
@@ -177,9 +178,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   const int G = p.E + p.S;
-  // kRouter folds its K splits into the n-tile index: nv = n * ksplit + ks
-  const int ksplit = MODE == kRouter ? p.ksplit : 1;
-  const int n_tiles = (p.N + BN - 1) / BN * ksplit;
+  // kRouter and kDown fold their K splits into the n-tile index: nv = n * ksplit + ks
+  const int ksplit = MODE == kGateUp ? 1 : p.ksplit;
+  // n-tile width: the MMA's full N, except single-CTA expert launches, which
+  // may use narrower tiles (more tiles for layers with few rows)
+  const int bn = (PAIR || MODE == kRouter) ? BN : p.bn;
+  const int n_tiles = (p.N + bn - 1) / bn * ksplit;
   const int k_blocks = p.K / BK;                               // per weight part
   const int k_total = MODE == kRouter ? 3 * k_blocks : k_blocks;
   // K-block range [kt_begin(ks), kt_begin(ks + 1)) of split ks
@@ -243,8 +247,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int a_row = static_cast<int>(gi.a_row0) + tile_first_row(m, gi.rows, SET, BM) +
                         static_cast<int>(rank) * BM;
       // pairs: this CTA's half of the tile's (possibly narrowed) N range
-      const int n_pad = (min(BN, p.N - n * BN) + 31) & ~31;
-      const int b_row = n * BN + (PAIR ? static_cast<int>(rank) * (n_pad >> 1) : 0);
+      const int n_pad = (min(bn, p.N - n * bn) + 31) & ~31;
+      const int b_row = n * bn + (PAIR ? static_cast<int>(rank) * (n_pad >> 1) : 0);
+      // single-CTA expert tiles load only the 128-row boxes the tile covers
+      const int b_loads = (PAIR || MODE == kRouter) ? TL::B_LOADS : (n_pad + TL::B_BOX - 1) / TL::B_BOX;
       bool ok = true;
       for (int kt = kt_begin(ks); kt < kt_begin(ks + 1); ++kt) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, s_abort, p.status)) { ok = false; break; }
@@ -258,10 +264,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tma_load_2d_pair(sA + stage * A_BYTES, tmA, bar0, kb * BK, a_row);
           tma_load_3d_pair(sB + stage * TL::B_BYTES, tmB, bar0, kb * BK, b_row, slice);
         } else {
-          mbar_arrive_expect_tx(&full[stage], A_BYTES + TL::B_BYTES);
+          mbar_arrive_expect_tx(&full[stage], A_BYTES + b_loads * (TL::B_BOX * BK * 2));
           tma_load_2d(sA + stage * A_BYTES, tmA, &full[stage], kb * BK, a_row);
-#pragma unroll
-          for (int i = 0; i < TL::B_LOADS; ++i)
+          for (int i = 0; i < b_loads; ++i)
             tma_load_3d(sB + stage * TL::B_BYTES + i * (TL::B_BOX * BK * 2), tmB, &full[stage],
                         kb * BK, b_row + i * TL::B_BOX, slice);
         }
@@ -291,8 +296,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int g, m, nv;
       decode_tile(tile, s_tile, G, s_off, p.E, p.T, SET, BM, g, m, nv);
       const int n = nv / ksplit, ks = nv - n * ksplit;
-      // the last n-tile of a ragged N runs a narrower MMA (N multiple of 32)
-      const int n_here = min(BN, p.N - n * BN);
+      // a narrow or ragged last n-tile runs a narrower MMA (N multiple of 32)
+      const int n_here = min(bn, p.N - n * bn);
       const uint32_t idesc = n_here >= BN ? TL::IDESC : idesc_bf16_f32(TL::TILE_M, (n_here + 31) & ~31);
       if (MODE != kRouter) {
         const int acc = it & 1;
@@ -318,7 +323,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kk = 0; kk < BK / 16; ++kk) {
           // +32 bytes per K=16 step inside the 128-byte swizzle atom
           // router: a fresh sum per chain; experts: accumulate over the tile
-          const bool accumulate = MODE == kRouter ? (!chain_start || kk != 0) : ((kb | kk) != 0);
+          const bool accumulate = MODE == kRouter ? (!chain_start || kk != 0) : (((kb - kb0) | kk) != 0);
           if (PAIR)
             mma_bf16_ss_pair(d_tmem, adesc + static_cast<uint64_t>(2 * kk),
                              bdesc + static_cast<uint64_t>(2 * kk), idesc, accumulate ? 1u : 0u);
@@ -433,10 +438,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       const uint32_t t_row = t_lane + static_cast<uint32_t>(acc * BN);
+      const int n_here = min(bn, p.N - n * bn);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
-        const int col0 = n * BN + c * 32;
-        if (col0 >= p.N) break;                    // warp-uniform
+        const int col0 = n * bn + c * 32;
+        if (c * 32 >= n_here) break;               // warp-uniform
         uint32_t v[32];
         tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * 32), v);
         tmem_ld_wait();
@@ -458,7 +464,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
           dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
         } else {
-          store_rows_f32(st, v, lane, static_cast<float*>(p.out[gi.src]),
+          // kDown with K splits: split ks writes its own partial rows
+          store_rows_f32(st, v, lane, static_cast<float*>(p.out[gi.src]) + ks * p.split_stride,
                          gi.out_row0 + row0 + quarter * 32, rows_left, p.ld_out, col0);
         }
       }
@@ -566,7 +573,7 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
                                    const void* w_down, const void* ws_gate_up,
                                    const void* ws_down, void* h, void* y_routed, void* y_shared,
                                    int32_t* status, int num_sms, cudaStream_t stream,
-                                   bool* map_error) {
+                                   bool* map_error, const FfnTiling& tiling) {
   using namespace sm100;
   // B maps: box of 128 rows = the half of a 256-row n-tile one CTA of a pair
   // loads; the single-CTA odd-tile launch loads both halves (two boxes)
@@ -597,6 +604,7 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   g.E = L.E; g.S = L.S; g.K = L.H; g.N = 2 * L.I; g.ld_out = L.I;
   g.rows_cap = static_cast<int>(Rk);
   g.ksplit = 1;
+  g.bn = tiling.gate_up_bn;
   // paired groups on CTA pairs, the rest on single CTAs (grouping.cuh); with
   // T <= 128 every group has one m-tile and the pair launch is skipped
   const bool pairs = L.T > BM;
@@ -621,7 +629,9 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   d.T = L.T; d.a1_base = Rk; d.a1_stride = L.T;
   d.E = L.E; d.S = L.S; d.K = L.I; d.N = L.H; d.ld_out = L.H;
   d.rows_cap = static_cast<int>(Rk);
-  d.ksplit = 1;
+  d.ksplit = tiling.down_ksplit;
+  d.split_stride = L.T * static_cast<int64_t>(L.H);   // partial rows of the shared groups
+  d.bn = 256;
   e = pairs ? launch_mode<kDown, true>(d, num_sms, stream) : cudaSuccess;
   if (e == cudaSuccess) e = launch_mode<kDown, false>(d, num_sms, stream);
   return e;
@@ -652,6 +662,7 @@ cudaError_t launch_router_logits_sm100(const Layer& L, const void* x, const void
   r.rows_cap = 0;
   r.ksplit = ksplit;
   r.split_stride = L.T * static_cast<int64_t>(ld_z);
+  r.bn = Tile<kRouter, false>::BN;
   return launch_mode<kRouter, false>(r, num_sms, stream);
 }
 

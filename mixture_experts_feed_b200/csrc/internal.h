@@ -37,13 +37,21 @@ cudaError_t launch_permute(const Layer& L, const int32_t* topk_idx, const uint8_
                            cudaStream_t stream);
 
 // grouped_gemm_sm100.cu (bf16, tcgen05)
+// Tile shape choices of one expert-FFN call: the n-tile width of the
+// single-CTA gate_up launch (256 or 128) and the K splits of the down
+// projection (its split s writes partial rows at y_shared + s * T * H; the
+// caller sums them).  The MoE layer uses the defaults.
+struct FfnTiling {
+  int gate_up_bn = 256;
+  int down_ksplit = 1;
+};
 cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_perm,
                                    const int32_t* offsets, const int32_t* perm_slot,
                                    const float* topk_w, const float* gamma, const void* w_gate_up,
                                    const void* w_down, const void* ws_gate_up,
                                    const void* ws_down, void* h, void* y_routed, void* y_shared,
                                    int32_t* status, int num_sms, cudaStream_t stream,
-                                   bool* map_error);
+                                   bool* map_error, const FfnTiling& tiling = FfnTiling());
 int sm100_gemm_max_smem(int E, int S);
 cudaError_t launch_router_logits_sm100(const Layer& L, const void* x, const void* w_parts,
                                        float* logits, int ld_z, int ksplit, int32_t* status,

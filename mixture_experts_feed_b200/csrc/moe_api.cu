@@ -239,6 +239,36 @@ struct DenseWs {
   size_t status, h, y, x_norm, total;
 };
 
+// Tile choices of the dense layer on the tensor cores (functions of the
+// shape only, so every device computes the same partial sums).  With few
+// token rows (decode) the layer streams its weights: the single-CTA gate_up
+// launch takes 128-wide n-tiles when that fills the 148 SMs better, and the
+// down projection splits K until its tiles reach about 148.
+constexpr int kTilingSms = 148;
+
+FfnTiling dense_tiling(const Layer& L) {
+  FfnTiling t;
+  if (L.dtype != MOE_BF16 || L.T <= 0) return t;
+  const int64_t mt = (L.T + 127) / 128;
+  auto waves_eff = [](int64_t tiles) {
+    const int64_t waves = (tiles + kTilingSms - 1) / kTilingSms;
+    return static_cast<double>(tiles) / static_cast<double>(waves * kTilingSms);
+  };
+  if (L.T <= 128) {   // every tile on the single-CTA launch
+    const int64_t t256 = mt * ((2 * L.I + 255) / 256), t128 = mt * ((2 * L.I + 127) / 128);
+    if (t256 < 4 * kTilingSms && waves_eff(t128) > waves_eff(t256) + 0.05) t.gate_up_bn = 128;
+  }
+  const int64_t down_tiles = mt * ((L.H + 255) / 256);   // m-tiles x n-tiles (either launch)
+  if (down_tiles < kTilingSms) {
+    int64_t ks = kTilingSms / down_tiles;
+    const int64_t kmax = L.I / 64 / 4;                     // at least 4 K blocks per split
+    if (ks > kmax) ks = kmax;
+    if (ks > 16) ks = 16;
+    t.down_ksplit = static_cast<int>(ks < 1 ? 1 : ks);
+  }
+  return t;
+}
+
 moe_status_t check_dense(const moe_dense_desc_t* d, Layer* L) {
   if (d == nullptr) return MOE_ERR_INVALID_ARG;
   if (d->num_tokens < 0 || d->hidden <= 0 || d->intermediate <= 0) return MOE_ERR_INVALID_ARG;
@@ -270,7 +300,7 @@ DenseWs dense_ws_layout(const Layer& L) {
   const size_t T = static_cast<size_t>(L.T);
   w.status = take(kStatusBytes);
   w.h = take(T * L.I * elt);
-  w.y = take(T * L.H * 4);
+  w.y = take(T * L.H * 4 * dense_tiling(L).down_ksplit);   // one partial per K split
   w.x_norm = take(T * L.H * elt);    // moe_dense_mlp_prenorm: the normalised input
   w.total = off;
   return w;
@@ -298,11 +328,12 @@ moe_status_t dense_checked(const moe_dense_desc_t* desc, const void* x, const vo
     x = xn;
   }
   // one shared group: the routed operands are never read (E = 0, k = 0)
+  const FfnTiling tiling = dense_tiling(L);
   if (L.dtype == MOE_BF16) {
     bool map_error = false;
     const cudaError_t e = launch_expert_ffn_bf16(L, x, x, nullptr, nullptr, nullptr, nullptr,
                                                  nullptr, nullptr, w_gate_up, w_down, h, y, y,
-                                                 status, num_sms(), s, &map_error);
+                                                 status, num_sms(), s, &map_error, tiling);
     if (map_error) return MOE_ERR_INVALID_ARG;
     MOE_TRY(cuda_status(e));
   } else {
@@ -310,7 +341,10 @@ moe_status_t dense_checked(const moe_dense_desc_t* desc, const void* x, const vo
                                               nullptr, nullptr, w_gate_up, w_down, h, y, y,
                                               status, num_sms(), s)));
   }
-  return cuda_status(launch_combine(L, y, y, nullptr, out, status, num_sms(), s));
+  // the recombination sums the K-split partials in split order (S of them)
+  Layer Lc = L;
+  Lc.S = tiling.down_ksplit;
+  return cuda_status(launch_combine(Lc, y, y, nullptr, out, status, num_sms(), s));
 }
 
 }  // namespace

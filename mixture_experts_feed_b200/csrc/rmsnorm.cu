@@ -11,21 +11,24 @@
 // bf16 is done here on the fp64 bit pattern, round to nearest with ties to
 // even, in one step.
 //
-// One warp per token row, 16-byte vectors along the row: pass 1 streams
-// the row and sums the squares in fp64 (a lane's own elements in order, then
-// a butterfly across the warp, which leaves the same sum in every lane),
-// pass 2 streams it again (from L1/L2) and writes the result.  No block-wide
-// barrier, so every resident warp keeps a row in flight.  Each element is
+// One warp per token row, 16-byte vectors along the row, streamed twice:
+// pass 1 sums the squares, pass 2 re-reads the row (from L1: a few blocks
+// per SM keep their rows there) and writes the result.  Both passes load
+// their vectors in explicit batches (RMS_BATCH vectors a lane in registers
+// before any is used), so each warp keeps RMS_BATCH x 512 bytes in flight,
+// and pass 1 adds into one fp64 partial sum per element position of a
+// vector (8 short chains instead of one long one); the partials are added in
+// a fixed order, then across the warp by a butterfly, which leaves the same
+// sum in every lane.  Each element is
 // scaled by the row's 1/s, s = sqrt(mean + eps), computed once per row in
 // fp64.  bf16 layers: x * weight is exact in fp32 (two 8-bit significands);
 // y32 = (x * weight) * fp32(1/s) is within 2^-23 |y| (under 2 fp32 ulps) of
-// the exact y, so when y32 is at least 3 ulps from a bf16 rounding tie it
+// the exact y, so when y32 is at least 4 ulps from a bf16 rounding tie it
 // rounds like y, and it is rounded directly; otherwise (about 1 element in
 // 8000) y is formed in fp64 and rounded from there.  fp32 layers multiply in
 // fp64.  Against x / s * weight in fp64 the result differs only within
 // ~1e-16 of a tie.  HBM-bound: 2 x dtype bytes per element.  `out` may alias
-// `x` (a lane writes a vector only after reading it, and pass 1 of a row
-// ends before its pass 2 starts).
+// `x` (a lane writes only vectors it has read).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -58,19 +61,25 @@ __device__ __forceinline__ uint16_t bf16_bits_rne(double y) {
   return static_cast<uint16_t>(__float_as_uint(__double2float_rn(r)) >> 16);
 }
 
+#ifndef RMS_BATCH
+#define RMS_BATCH 4
+#endif
+#ifndef RMS_BLOCKS_PER_SM
+#define RMS_BLOCKS_PER_SM 4
+#endif
+
 struct Bf16Row {
   using Vec = uint4;                      // 8 bf16
   static constexpr int V = 8;
-  __device__ static double sumsq(const Vec& q) {
+  // acc[i] += square of element i (squares of bf16 values are exact)
+  __device__ static void sumsq(const Vec& q, double (&acc)[V]) {
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    double acc = 0.0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const double a = __uint_as_float(w[i] << 16), b = __uint_as_float(w[i] & 0xFFFF0000u);
-      acc = fma(a, a, acc);              // squares of bf16 values are exact
-      acc = fma(b, b, acc);
+      acc[2 * i] = fma(a, a, acc[2 * i]);
+      acc[2 * i + 1] = fma(b, b, acc[2 * i + 1]);
     }
-    return acc;
   }
   // bf16 bits of p * inv (p = x * weight, exact in fp32)
   __device__ static uint32_t one(float p, float inv32, double inv) {
@@ -97,11 +106,12 @@ struct Bf16Row {
 struct F32Row {
   using Vec = float4;
   static constexpr int V = 4;
-  __device__ static double sumsq(const Vec& q) {
-    double acc = static_cast<double>(q.x) * q.x;   // squares of fp32 values are exact in fp64
-    acc = fma(static_cast<double>(q.y), q.y, acc);
-    acc = fma(static_cast<double>(q.z), q.z, acc);
-    return fma(static_cast<double>(q.w), q.w, acc);
+  // squares of fp32 values are exact in fp64
+  __device__ static void sumsq(const Vec& q, double (&acc)[V]) {
+    acc[0] = fma(static_cast<double>(q.x), q.x, acc[0]);
+    acc[1] = fma(static_cast<double>(q.y), q.y, acc[1]);
+    acc[2] = fma(static_cast<double>(q.z), q.z, acc[2]);
+    acc[3] = fma(static_cast<double>(q.w), q.w, acc[3]);
   }
   __device__ static Vec scale(const Vec& q, const Vec& g, float, double inv) {
     return make_float4(__double2float_rn(static_cast<double>(q.x) * g.x * inv),
@@ -116,6 +126,7 @@ __global__ void __launch_bounds__(kThreads)
     rmsnorm_kernel(const void* x_, const void* __restrict__ w_, void* out_, int64_t T, int H,
                    double eps) {
   using Vec = typename R::Vec;
+  constexpr int B = RMS_BATCH;
   const Vec* x = static_cast<const Vec*>(x_);
   const Vec* w = static_cast<const Vec*>(w_);
   Vec* out = static_cast<Vec*>(out_);
@@ -125,16 +136,38 @@ __global__ void __launch_bounds__(kThreads)
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5); t < T;
        t += warps) {
     const Vec* row = x + t * nv;
+    Vec* orow = out + t * nv;
+    double part[R::V];
+#pragma unroll
+    for (int i = 0; i < R::V; ++i) part[i] = 0.0;
+    for (int v0 = lane; v0 < nv; v0 += 32 * B) {
+      Vec buf[B];
+#pragma unroll
+      for (int j = 0; j < B; ++j)
+        if (v0 + 32 * j < nv) buf[j] = row[v0 + 32 * j];
+#pragma unroll
+      for (int j = 0; j < B; ++j)
+        if (v0 + 32 * j < nv) R::sumsq(buf[j], part);
+    }
     double acc = 0.0;
-#pragma unroll 4
-    for (int v = lane; v < nv; v += 32) acc += R::sumsq(row[v]);
+#pragma unroll
+    for (int i = 0; i < R::V; ++i) acc += part[i];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     const double inv = 1.0 / sqrt(acc / H + eps);
     const float inv32 = __double2float_rn(inv);
-    Vec* orow = out + t * nv;
-#pragma unroll 4
-    for (int v = lane; v < nv; v += 32) orow[v] = R::scale(row[v], w[v], inv32, inv);
+    for (int v0 = lane; v0 < nv; v0 += 32 * B) {
+      Vec buf[B], gw[B];
+#pragma unroll
+      for (int j = 0; j < B; ++j)
+        if (v0 + 32 * j < nv) {
+          buf[j] = row[v0 + 32 * j];
+          gw[j] = w[v0 + 32 * j];
+        }
+#pragma unroll
+      for (int j = 0; j < B; ++j)
+        if (v0 + 32 * j < nv) orow[v0 + 32 * j] = R::scale(buf[j], gw[j], inv32, inv);
+    }
   }
 }
 
@@ -143,9 +176,10 @@ __global__ void __launch_bounds__(kThreads)
 cudaError_t launch_rmsnorm(int64_t T, int H, int dtype, float eps, const void* x,
                            const void* weight, void* out, int num_sms, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  // one warp per row, 8 rows per block, up to 8 blocks per SM
+  // one warp per row, 8 rows per block, a few blocks per SM (rows re-read from L1)
   const int64_t blocks = (T + kThreads / 32 - 1) / (kThreads / 32);
-  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(blocks, static_cast<int64_t>(num_sms) * 8));
+  const unsigned grid = static_cast<unsigned>(
+      std::min<int64_t>(blocks, static_cast<int64_t>(num_sms) * RMS_BLOCKS_PER_SM));
   if (dtype == MOE_BF16)
     rmsnorm_kernel<Bf16Row><<<grid, kThreads, 0, stream>>>(x, weight, out, T, H, eps);
   else

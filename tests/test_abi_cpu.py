@@ -130,6 +130,10 @@ def test_dense_desc_layout_and_sizes():
         assert moe.dense_workspace_size(L) >= el * w.T * w.I + 4 * w.T * w.H
         gemms = (4 if w.T > 128 else 2) if w.dtype == "bf16" else 2
         assert moe.dense_kernel_count(L) == gemms + 1
+    for T in (0, 1, 32, 129):              # host-side tiling choices at the edges
+        for dt in (torch.bfloat16, torch.float32):
+            assert moe.dense_workspace_size(moe.DenseLayer(T, 128, 64, dt)) > 0
+    assert moe.dense_kernel_count(moe.DenseLayer(0, 128, 64)) == 0
 
 
 def _dense_status(T=8, H=64, I=64, dtype=moe.MOE_BF16, gs=1.0, ws_bytes=None, ptr=256):

@@ -36,11 +36,12 @@ def run_dense(w, inputs, d=None):
 
 SMALL = [
     # T, H, I, dtype, global_scale      what it covers
-    (300, 512, 640, "bf16", 1.0),       # ragged T (3 m-tiles: single CTAs), gate_up N = 1280
+    (300, 512, 640, "bf16", 1.0),       # ragged T (3 m-tiles: single CTAs), down split 2 ways
     (517, 384, 320, "bf16", 0.5),       # 5 m-tiles, down N = 384 (1.5 tiles), scale 0.5
-    (1024, 256, 512, "bf16", 2.0),      # 8 m-tiles: CTA pairs
+    (1024, 256, 512, "bf16", 2.0),      # 8 m-tiles: CTA pairs, down split 2 ways
     (1, 128, 64, "bf16", 1.0),          # a single token
     (129, 128, 192, "bf16", 1.0),       # 2 m-tiles, the second one row
+    (64, 256, 1024, "bf16", 1.0),       # decode-shaped: 128-wide gate_up tiles, down split 4 ways
     (96, 128, 192, "f32", 1.0),         # fp32 layer (CUDA cores)
     (77, 192, 128, "f32", 1.5),
 ]
