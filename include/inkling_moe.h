@@ -61,7 +61,7 @@ extern "C" {
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned buffer */
-  MOE_ERR_UNSUPPORTED = 2,   /* valid layer outside this build's limits */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid layer outside this library's limits */
   MOE_ERR_WORKSPACE = 3,     /* workspace smaller than moe_workspace_size() */
   MOE_ERR_CUDA = 4,          /* the CUDA runtime reported an error */
   MOE_ERR_DEVICE_CHECK = 5,  /* a kernel saw an out-of-range index */

@@ -69,8 +69,9 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-# The five workloads: sizes from the task's configuration table; the default
-# hidden size 6144 of the last three is the pages' InklingTextConfig.hidden_size.
+# The five MoE workloads: a small fp32 layer, a mid-sized bf16 layer, and three
+# layers at InklingTextConfig's hidden size 6144 (prefill, one decode step, and
+# a Zipf-skewed router).
 WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
     Workload("tiny-f32-T64-H128-E8k2S1-I64", 64, 128, 8, 2, 1, 64,
              "f32", 1.0, 1.0, seed=0),

@@ -35,7 +35,7 @@ What it computes, step by step, from the NeMo AutoModel Inkling pages
    layer's ``global_scale`` (the pages leave where it applies unstated; the
    output is scaled, which in exact arithmetic equals scaling h).
 
-Readings taken where the pages are silent (each one is listed in the design doc):
+Readings taken where the pages are silent:
 log-sigmoid applies to the whole concatenated vector, shared logits included;
 the gammas are scaled like the routed weights; ties in the selection score go
 to the lower expert index and the k chosen experts are returned in descending
