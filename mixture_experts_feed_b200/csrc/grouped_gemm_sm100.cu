@@ -607,9 +607,12 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   g.bn = tiling.gate_up_bn;
   // paired groups on CTA pairs, the rest on single CTAs (grouping.cuh); with
   // T <= 128 every group has one m-tile and the pair launch is skipped
-  const bool pairs = L.T > BM;
+  // (E == 0, the dense layer: the host knows the one group's m-tiles and
+  // launches only the kind of CTA that has tiles)
+  const bool pairs = L.T > BM && (L.E > 0 || group_paired(static_cast<int>((L.T + BM - 1) / BM)));
+  const bool singles = L.E > 0 || !pairs;
   cudaError_t e = pairs ? launch_mode<kGateUp, true>(g, num_sms, stream) : cudaSuccess;
-  if (e == cudaSuccess) e = launch_mode<kGateUp, false>(g, num_sms, stream);
+  if (e == cudaSuccess && singles) e = launch_mode<kGateUp, false>(g, num_sms, stream);
   if (e != cudaSuccess) return e;
 
   // ---------------- down: h [rows, I] x [H, I]^T -> y [rows, H] (fp32)
@@ -633,7 +636,7 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   d.split_stride = L.T * static_cast<int64_t>(L.H);   // partial rows of the shared groups
   d.bn = 256;
   e = pairs ? launch_mode<kDown, true>(d, num_sms, stream) : cudaSuccess;
-  if (e == cudaSuccess) e = launch_mode<kDown, false>(d, num_sms, stream);
+  if (e == cudaSuccess && singles) e = launch_mode<kDown, false>(d, num_sms, stream);
   return e;
 }
 

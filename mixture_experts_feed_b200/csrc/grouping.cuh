@@ -67,7 +67,7 @@ __device__ __forceinline__ GroupInfo group_info(int g, const int* s_off, int E, 
 
 enum TileSet { kAllTiles = 0, kPairs = 1, kSingles = 2 };
 
-__device__ __forceinline__ bool group_paired(int mt) {
+__host__ __device__ __forceinline__ bool group_paired(int mt) {
   return mt >= 2 && ((mt & 1) == 0 || mt >= 7);
 }
 

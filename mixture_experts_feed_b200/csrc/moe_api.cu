@@ -521,10 +521,9 @@ moe_status_t moe_dense_mlp_prenorm(const moe_dense_desc_t* desc, const void* x,
 int32_t moe_dense_kernel_count(const moe_dense_desc_t* desc) {
   Layer L;
   if (check_dense(desc, &L) != MOE_OK || L.T == 0) return 0;
-  // gate_up + down (bf16 with T > 128: CTA-pair launch + single-CTA launch
-  // each), then the rounding pass
-  const int gemms = L.dtype == MOE_BF16 ? (L.T > 128 ? 4 : 2) : 2;
-  return gemms + 1;
+  // gate_up + down (one launch each: the one group's tiles are all CTA-pair
+  // or all single-CTA tiles), then the rounding pass
+  return 3;
 }
 
 int32_t moe_dense_prenorm_kernel_count(const moe_dense_desc_t* desc) {

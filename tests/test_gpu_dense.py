@@ -100,3 +100,23 @@ def test_dense_empty_batch():
     moe.moe_dense_mlp(L, x, wgu, wd, torch.empty_like(x), ws)
     torch.cuda.synchronize()
     moe.read_device_status(ws)
+
+
+def _random_dense(n, seed):
+    g = torch.Generator().manual_seed(seed)
+    r = lambda lo, hi: int(torch.randint(lo, hi + 1, (1,), generator=g))
+    return [(r(1, 1100), 64 * r(1, 12), 64 * r(1, 16), "f32" if r(0, 3) == 0 else "bf16",
+             0.25 * r(1, 8)) for _ in range(n)]
+
+
+RANDOM = _random_dense(8, seed=77)
+
+
+@pytest.mark.parametrize("shape", RANDOM, ids=[f"T{s[0]}-H{s[1]}-I{s[2]}-{s[3]}-gs{s[4]}" for s in RANDOM])
+def test_dense_random_shapes(shape):
+    T, H, I, dtype, gs = shape
+    w = mw.dense_tiny(T=T, H=H, I=I, dtype=dtype, global_scale=gs, seed=T + H + I)
+    inputs = mw.generate_dense(w, threads=4)
+    out = run_dense(w, inputs)
+    ref = oracle.dense_mlp(inputs["x"], inputs["w_gate_up"], inputs["w_down"], gs)
+    check_output(out, ref, w.torch_dtype, "dense out", strict=False)

@@ -223,3 +223,27 @@ def test_stalled_wait_times_out_and_context_survives():
     assert 0.9 < elapsed < 30.0
     r = run_forward(L, to_device(inputs), ws=ws)     # the context is still usable
     assert torch.isfinite(r["out"].float()).all()
+
+
+def _random_shapes(n, seed):
+    g = torch.Generator().manual_seed(seed)
+    out = []
+    for _ in range(n):
+        r = lambda lo, hi: int(torch.randint(lo, hi + 1, (1,), generator=g))
+        E = r(1, 300)
+        k = r(1, min(8, E))
+        dtype = "f32" if r(0, 3) == 0 else "bf16"
+        out.append((r(1, 600), 64 * r(1, 12), E, k, r(0, 3), 64 * r(1, 6), dtype))
+    return out
+
+
+RANDOM = _random_shapes(16, seed=2024)
+
+
+@pytest.mark.parametrize("shape", RANDOM, ids=[f"T{s[0]}-H{s[1]}-E{s[2]}k{s[3]}S{s[4]}-I{s[5]}-{s[6]}" for s in RANDOM])
+def test_random_shapes(shape):
+    """Seeded random layer shapes (T, H, E, k, S, I, dtype) through the one-call path."""
+    w, inputs = small_case(*shape, seed=sum(shape[:6]))
+    L = moe.Layer.from_workload(w)
+    r = run_forward(L, to_device(inputs))
+    check_all(w, inputs, r)
