@@ -15,7 +15,12 @@
 // n-tile by n-tile inside (consecutive tiles share one block of rows).  CTAs
 // running together then reuse the shared operand from L2, and the group's
 // other operand (the n-tile strips, or the row blocks) is the smaller one to
-// keep in L2 from one wave of tiles to the next.
+// keep in L2 from one wave of tiles to the next.  A group long in both
+// dimensions (more than kBandTiles m-tiles and more than kNarrowStrips
+// n-tiles: a dense layer) runs in bands of kBandTiles m-tiles, n-tile by
+// n-tile inside a band: a wave covers a near-square block of tiles, the
+// band's rows stay in L2 while its strips stream past, and each strip is
+// shared by the band's tiles running together.
 //
 // A group's rows split into mt = ceil(rows / bm) m-tiles of bm rows.  A
 // launch covers them in one of three ways (TileSet):
@@ -66,6 +71,9 @@ __device__ __forceinline__ GroupInfo group_info(int g, const int* s_off, int E, 
 }
 
 enum TileSet { kAllTiles = 0, kPairs = 1, kSingles = 2 };
+
+constexpr int kBandTiles = 8;      // m-tiles per band (tile order, below)
+constexpr int kNarrowStrips = 16;  // groups with at most this many n-tiles keep every strip in L2
 
 __host__ __device__ __forceinline__ bool group_paired(int mt) {
   return mt >= 2 && ((mt & 1) == 0 || mt >= 7);
@@ -150,7 +158,15 @@ __device__ __forceinline__ void decode_tile(int tile, const int* s_tile, int G, 
   const int mt = tiles_of_rows(rows, set, bm);
   const int local = tile - s_tile[g];
   const int nt = (s_tile[g + 1] - s_tile[g]) / mt;
-  if (mt > nt) {
+  if (mt > kBandTiles && nt > kNarrowStrips) {
+    // banded: kBandTiles m-tiles at a time, n-tile by n-tile inside a band
+    const int band_tiles = kBandTiles * nt;
+    const int band = local / band_tiles;
+    const int in_band = local - band * band_tiles;
+    const int rows = min(kBandTiles, mt - band * kBandTiles);   // m-tiles in this band
+    n = in_band / rows;
+    m = band * kBandTiles + (in_band - n * rows);
+  } else if (mt > nt) {
     m = local / nt;
     n = local - m * nt;
   } else {
