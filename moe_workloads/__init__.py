@@ -69,9 +69,9 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-# The five MoE workloads: a small fp32 layer, a mid-sized bf16 layer, and three
-# layers at InklingTextConfig's hidden size 6144 (prefill, one decode step, and
-# a Zipf-skewed router).
+# The MoE workloads: a small fp32 layer, a mid-sized bf16 layer, three layers
+# at InklingTextConfig's hidden size 6144 (prefill, one decode step, and a
+# Zipf-skewed router), and the layer at InklingTextConfig's own MoE defaults.
 WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
     Workload("tiny-f32-T64-H128-E8k2S1-I64", 64, 128, 8, 2, 1, 64,
              "f32", 1.0, 1.0, seed=0),
@@ -83,6 +83,11 @@ WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
              "bf16", 2.5, 1.0, seed=3),
     Workload("zipf-bf16-T16384-H6144-E256k8S1-I1024", 16384, 6144, 256, 8, 1, 1024,
              "bf16", 2.5, 1.0, seed=4, bias="zipf"),
+    # InklingTextConfig's own MoE defaults (hidden_size 6144, n_routed_experts
+    # 256, num_experts_per_tok 6, n_shared_experts 2, moe_intermediate_size
+    # 3072, route_scale 8.0) on a 4096-token batch: 29 GB of expert weights
+    Workload("model-bf16-T4096-H6144-E256k6S2-I3072", 4096, 6144, 256, 6, 2, 3072,
+             "bf16", 8.0, 1.0, seed=9),
 ]}
 
 ORDERED = list(WORKLOADS.values())
@@ -91,7 +96,7 @@ ORDERED = list(WORKLOADS.values())
 def by_name(name: str) -> Workload:
     if name in WORKLOADS:
         return WORKLOADS[name]
-    # allow 1-based position as a short name ("1".."5")
+    # allow 1-based position as a short name ("1".."6")
     if name.isdigit() and 1 <= int(name) <= len(ORDERED):
         return ORDERED[int(name) - 1]
     raise KeyError(f"unknown workload {name!r}; known: {list(WORKLOADS)}")
