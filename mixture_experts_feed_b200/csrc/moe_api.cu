@@ -487,11 +487,12 @@ moe_status_t moe_rmsnorm(int64_t num_tokens, int32_t hidden, moe_dtype_t dtype, 
 int32_t moe_forward_kernel_count(const moe_layer_desc_t* desc) {
   Layer L;
   if (check_desc(desc, &L) != MOE_OK || L.T == 0) return 0;
-  // router: (bf16: split + tensor-core logits | fp32: logits) + top-k;
-  // permute: count, scan, compact, gather; experts: gate_up + down (bf16 with
-  // T > 128: CTA-pair launch + single-CTA launch each); combine.
+  // router: (bf16: split + tensor-core logits | fp32: logits) + top-k (plus
+  // a partial-logit sum when K is split 4 or more ways); permute: count,
+  // scan, compact, gather; experts: gate_up + down (bf16 with T > 128:
+  // CTA-pair launch + single-CTA launch each); combine.
   const int experts = L.dtype == MOE_BF16 ? (L.T > 128 ? 4 : 2) : 2;
-  return (L.dtype == MOE_BF16 ? 3 : 2) + 4 + experts + 1;
+  return (L.dtype == MOE_BF16 ? 2 : 1) + router_topk_launches(router_ksplit(L)) + 4 + experts + 1;
 }
 
 moe_status_t moe_dense_workspace_size(const moe_dense_desc_t* desc, size_t* bytes) {

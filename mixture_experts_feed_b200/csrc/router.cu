@@ -11,6 +11,8 @@
 //                         fp32 FFMA, tiled 64 tokens x 64 rows x 32 K.
 //   Both give fp32 logits for all E routed + S shared rows of the gate bank
 //   (the gate runs in fp32: gate_precision=torch.float32).
+//   router_sum_splits_kernel  (many K splits only) partial logits summed in
+//                         split order, one thread per logit
 //   router_topk_kernel    one warp per token: selection score
 //                         sigmoid(z) + bias over the routed rows, k rounds of
 //                         a warp-shuffle argmax (ties to the lower expert id),
@@ -136,8 +138,29 @@ __global__ void __launch_bounds__(RL_THREADS)
 __device__ __forceinline__ float sigmoidf_(float v) { return 1.0f / (1.0f + expf(-v)); }
 
 constexpr int TK_WARPS = 8;
+// From this many K splits on, a separate kernel sums the partial logits first.
+constexpr int kSumSplitsFrom = 4;
 
 // PL: routed scores held per lane (E <= 32 * PL).
+// Sum the K-split partial logits into split 0, in split order, one thread
+// per logit over the whole grid (the same additions, in the same order, as
+// the top-k kernel makes when it reads the partials itself).  Used when the
+// split count is large (few tokens): there the top-k kernel has few warps.
+__global__ void router_sum_splits_kernel(float* __restrict__ z, int ld, int ksplit, int64_t T,
+                                         int NE) {
+  const int64_t split = T * static_cast<int64_t>(ld);
+  const int64_t n = T * static_cast<int64_t>(NE);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const int64_t t = i / NE;
+    const int e = static_cast<int>(i - t * NE);
+    float* zt = z + t * ld + e;
+    float v = zt[0];
+    for (int s2 = 1; s2 < ksplit; ++s2) v += zt[s2 * split];
+    zt[0] = v;
+  }
+}
+
 template <int PL>
 __global__ void __launch_bounds__(TK_WARPS * 32)
     router_topk_kernel(const float* __restrict__ z, int ld, int ksplit,
@@ -231,9 +254,21 @@ cudaError_t launch_router_logits(const Layer& L, const void* x, const float* w_r
   return cudaGetLastError();
 }
 
+int router_topk_launches(int ksplit) { return ksplit >= kSumSplitsFrom ? 2 : 1; }
+
 cudaError_t launch_router_topk(const Layer& L, const float* logits, int ld, int ksplit,
                                const float* corr_bias, float* topk_w, int32_t* topk_idx,
                                float* shared_gamma, cudaStream_t stream) {
+  if (router_topk_launches(ksplit) == 2) {
+    const int NE = L.E + L.S;
+    const int64_t n = L.T * static_cast<int64_t>(NE);
+    const unsigned sgrid = static_cast<unsigned>(std::min<int64_t>(ceil_div(n, 256), 148 * 8));
+    router_sum_splits_kernel<<<sgrid, 256, 0, stream>>>(const_cast<float*>(logits), ld, ksplit,
+                                                        L.T, NE);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    ksplit = 1;
+  }
   const unsigned grid = static_cast<unsigned>(ceil_div(L.T, TK_WARPS));
   const float scale = L.route_scale * L.global_scale;
   const int pl = static_cast<int>(ceil_div(L.E, 32));
