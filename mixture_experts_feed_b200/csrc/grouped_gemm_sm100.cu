@@ -85,6 +85,7 @@ template <int MODE, bool PAIR_> struct Tile {
 struct alignas(64) GemmParams {
   CUtensorMap tmA[2];   // A operand of routed (0) and shared (1) groups: 2-D [rows, K]
   CUtensorMap tmB[2];   // weights of routed (0) and shared (1) groups: 3-D [G][N][K]
+  CUtensorMap tmY[2];   // kDown: fp32 output rows of routed (0) and shared (1) groups, box 32 x 32
   const int32_t* offsets;     // [E+1]
   const int32_t* perm_slot;   // [rows] slot of each permuted row (kGateUp weights)
   const float* topk_w;        // [T*k]
@@ -105,7 +106,9 @@ struct alignas(64) GemmParams {
 // Per epilogue warp, a 32 x 32 fp32 staging tile (row stride 36 floats:
 // 16-byte aligned, and each quarter-warp's 16-byte accesses hit distinct banks).
 constexpr int STAGE_LD = 36;
-constexpr int STAGE_WARP_BYTES = 32 * STAGE_LD * 4;
+// 5120 bytes a warp (the padded tile needs 4608): every warp's region starts
+// on a 1024-byte boundary, as a 128-byte-swizzled TMA box requires
+constexpr int STAGE_WARP_BYTES = 5120;
 
 template <int MODE, bool PAIR> struct SmemLayout {
   static constexpr int STAGES = Tile<MODE, PAIR>::STAGES;
@@ -464,9 +467,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
           dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
         } else {
-          // kDown with K splits: split ks writes its own partial rows
-          store_rows_f32(st, v, lane, static_cast<float*>(p.out[gi.src]) + ks * p.split_stride,
-                         gi.out_row0 + row0 + quarter * 32, rows_left, p.ld_out, col0);
+          if (rows_left >= 32) {
+            // a full 32-row slab: the 32 x 32 fp32 chunk goes through a
+            // 128-byte-swizzled staging box (chunk j of row r at 16-byte slot
+            // j ^ (r & 7): conflict-free) and one TMA store; only the buffer
+            // reuse waits, for the previous store to have read it.  K split
+            // ks writes the partial rows at row offset ks * T.
+            if (lane == 0) bulk_wait_group_read0();
+            __syncwarp();
+            uint8_t* box = reinterpret_cast<uint8_t*>(st);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ (lane & 7)) * 16)) =
+                  make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&p.tmY[gi.src], box, col0,
+                           static_cast<int32_t>(ks * p.T + gi.out_row0 + row0 + quarter * 32));
+              bulk_commit_group();
+            }
+          } else {
+            // the group's last rows: coalesced stores of the valid rows only
+            // (a box would write into the next group's rows)
+            if (lane == 0) bulk_wait_group_read0();
+            __syncwarp();
+            store_rows_f32(st, v, lane, static_cast<float*>(p.out[gi.src]) + ks * p.split_stride,
+                           gi.out_row0 + row0 + quarter * 32, rows_left, p.ld_out, col0);
+          }
         }
       }
       tc_fence_before();
@@ -477,6 +505,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       ++it;
     }
+    // the warp's TMA stores complete before the block (and its shared memory) goes
+    if (MODE == kDown && lane == 0) bulk_wait_group0();
   }
 
   tc_fence_before();
@@ -514,6 +544,20 @@ static bool encode_a(CUtensorMap* m, const void* base, int64_t rows, int K) {
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D fp32 map over [rows, H] (H contiguous), box [32 rows, 32 columns],
+// 128B swizzle: the down projection's output rows, written by TMA stores.
+static bool encode_y(CUtensorMap* m, void* base, int64_t rows, int H) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(H) * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 3-D bf16 map over [G][N][K] (K contiguous), box [1][bn][BK], 128B swizzle.
@@ -623,6 +667,13 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   if (ok && L.S > 0) ok = encode_b(&d.tmB[1], ws_down, L.S, L.H, L.I, BROWS);
   if (L.E == 0) d.tmB[0] = d.tmB[1];
   if (L.S == 0) d.tmB[1] = d.tmB[0];
+  // output maps: routed rows [T*k, H]; shared rows [S*T, H], or one partial
+  // [T, H] per K split when the down projection splits K (the dense layer)
+  const int64_t shared_rows = L.T * static_cast<int64_t>(L.S > tiling.down_ksplit ? L.S : tiling.down_ksplit);
+  if (ok && L.S > 0) ok = encode_y(&d.tmY[1], y_shared, shared_rows, L.H);
+  if (ok && routed) ok = encode_y(&d.tmY[0], y_routed, Rk, L.H);
+  if (!routed) d.tmY[0] = d.tmY[1];
+  if (L.S == 0) d.tmY[1] = d.tmY[0];
   if (!ok) { *map_error = true; return cudaErrorInvalidValue; }
   d.offsets = offsets; d.perm_slot = perm_slot; d.topk_w = topk_w; d.gamma = gamma;
   d.uniform_w = L.global_scale;
