@@ -45,9 +45,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # this workload, measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum,
 # one pass, first warm-up step); absent until captured for the current build.
 NCU_TRAFFIC_BYTES = {
-    "bf16-T8192-H6144-E128k8S1-I2048": 14288097280,
-    "zipf-bf16-T16384-H6144-E256k8S1-I1024": 8143021056,
-    "dense-bf16-T8192-H6144-I24576": 6509459712,
+    "bf16-T8192-H6144-E128k8S1-I2048": 14133757696,
+    "zipf-bf16-T16384-H6144-E256k8S1-I1024": 8011068160,
+    "dense-bf16-T8192-H6144-I24576": 6732003328,
+    "model-bf16-T4096-H6144-E256k6S2-I3072": 22748480000,
 }
 
 
