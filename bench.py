@@ -253,31 +253,53 @@ def gpu_arm(args, world, rank, local):
     xn = torch.empty_like(d["x"]) if args.prenorm else None
     xin = xn if args.prenorm else d["x"]
 
-    def step(ev=None):
+    def step(ev=None, st=None):
+        st = stream if st is None else st      # the stream to launch on (a capture stream too)
         if args.prenorm:
             if ev is not None:
-                ev[5].record(stream)
-            moe.moe_rmsnorm(d["x"], nw, xn, mw.RMS_NORM_EPS, stream)
+                ev[5].record(st)
+            moe.moe_rmsnorm(d["x"], nw, xn, mw.RMS_NORM_EPS, st)
         if ev is not None:
-            ev[0].record(stream)
-        moe.moe_route(L, xin, d["w_router"], d["corr_bias"], tw, ti, sg, ws, stream)
+            ev[0].record(st)
+        moe.moe_route(L, xin, d["w_router"], d["corr_bias"], tw, ti, sg, ws, st)
         if ev is not None:
-            ev[1].record(stream)
-        moe.moe_permute(L, ti, None, xin, off, ps, ip, xp, ws, stream)
+            ev[1].record(st)
+        moe.moe_permute(L, ti, None, xin, off, ps, ip, xp, ws, st)
         if ev is not None:
-            ev[2].record(stream)
+            ev[2].record(st)
         moe.moe_expert_ffn(L, xin, xp, off, ps, tw, sg, d["w_gate_up"], d["w_down"], wsgu, wsd,
-                           yr, ys, ws, stream)
+                           yr, ys, ws, st)
         if ev is not None:
-            ev[3].record(stream)
-        moe.moe_combine(L, yr, ys, ip, out, ws, stream)
+            ev[3].record(st)
+        moe.moe_combine(L, yr, ys, ip, out, ws, st)
         if ev is not None:
-            ev[4].record(stream)
+            ev[4].record(st)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
     moe.read_device_status(ws, stream)
+    graph = None
+    if args.graph:
+        # the whole op chain of one step captured once and replayed (the
+        # per-op events stay outside: op_ms then has only the total)
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.graph(graph, stream=cap):
+            step(st=cap)
+        torch.cuda.synchronize(dev)
+        # the replay must do the step's work: from a zeroed output it gives the
+        # eager step's bits
+        out.zero_()
+        graph.replay()
+        torch.cuda.synchronize(dev)
+        replayed = out.clone()
+        out.zero_()
+        step()
+        torch.cuda.synchronize(dev)
+        if not (torch.equal(replayed, out) and bool(replayed.abs().sum() > 0)):
+            raise RuntimeError("the captured graph does not reproduce the eager step")
 
     # ---- timed region: K steps, inputs (weights 9.7 GB at the default
     # workload) far larger than the 126 MB L2, so no flush is needed between steps
@@ -286,15 +308,24 @@ def gpu_arm(args, world, rank, local):
         barrier(world)
         torch.cuda.synchronize(dev)
         for i in range(args.steps):
-            step(evs[i])
+            if graph is None:
+                step(evs[i])
+            else:
+                evs[i][5 if args.prenorm else 0].record(stream)
+                graph.replay()
+                evs[i][4].record(stream)
         torch.cuda.synchronize(dev)
         barrier(world)
     clocks = clk.summary()
     moe.read_device_status(ws, stream)
     first = 5 if args.prenorm else 0
     total_ms = evs[0][first].elapsed_time(evs[-1][4])
-    op_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(4)]
-    norm_ms = (sum(e[5].elapsed_time(e[0]) for e in evs) / args.steps) if args.prenorm else None
+    if graph is None:
+        op_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(4)]
+        norm_ms = (sum(e[5].elapsed_time(e[0]) for e in evs) / args.steps) if args.prenorm else None
+    else:
+        op_ms = [float("nan")] * 4
+        norm_ms = float("nan") if args.prenorm else None
     ms_step = max_over_ranks(total_ms / args.steps, world)
 
     # ---- end to end through the public one-call API with host buffers: every
@@ -352,7 +383,9 @@ def gpu_arm(args, world, rank, local):
         peaks, peak_src = load_peaks()
         fl = mw.flops(w)
         ffn_flops = fl["routed"] + fl["shared"]
-        ffn_s = op_ms[2] / 1e3
+        # per-op times need the events between ops; a graph replay has only the
+        # step's: the roofline then charges the expert flops with the whole step
+        ffn_s = (op_ms[2] if graph is None else ms_step) / 1e3
         # algorithmic bytes of moe_expert_ffn: the weights of every group with
         # rows (routed experts with a nonzero count, every shared expert) once,
         # x_perm / x rows read once, h written and read once in the dtype, the
@@ -387,7 +420,8 @@ def gpu_arm(args, world, rank, local):
                        "l2": "inputs larger than L2 (expert weights %.1f GB)" % (mw.weight_bytes(w) / 1e9)},
             "tflops": world * fl["total"] / (ms_step / 1e3) / 1e12,
             "op_ms": {"route": op_ms[0], "permute": op_ms[1], "expert_ffn": op_ms[2], "combine": op_ms[3]},
-            "roofline": {"kernel": "grouped expert GEMMs (gate_up + down launches of moe_expert_ffn)",
+            "roofline": {"kernel": ("grouped expert GEMMs (gate_up + down launches of moe_expert_ffn)"
+                                    if graph is None else "whole step (one CUDA graph replay)"),
                          **roof},
             "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
@@ -396,16 +430,20 @@ def gpu_arm(args, world, rank, local):
                              else moe.forward_kernel_count(L)) * args.steps,
             "clocks": clocks,
         }
+        if graph is not None:
+            line["config"]["graph"] = True
+            del line["op_ms"]
         if args.prenorm:
             # the block: post_attention_layernorm, then the layer
             el_x = 2 if w.dtype == "bf16" else 4
             nb = 2 * T * H * el_x
             line["config"]["block"] = "rmsnorm prologue + layer"
-            line["op_ms"]["rmsnorm"] = norm_ms
-            line["rmsnorm_roofline"] = {"bound": "hbm", "achieved": nb / (norm_ms / 1e3) / 1e9,
-                                        "peak": hbm_peak, "unit": "GB/s",
-                                        "frac": nb / (norm_ms / 1e3) / 1e9 / hbm_peak,
-                                        "algorithmic_bytes": nb}
+            if graph is None:
+                line["op_ms"]["rmsnorm"] = norm_ms
+                line["rmsnorm_roofline"] = {"bound": "hbm", "achieved": nb / (norm_ms / 1e3) / 1e9,
+                                            "peak": hbm_peak, "unit": "GB/s",
+                                            "frac": nb / (norm_ms / 1e3) / 1e9 / hbm_peak,
+                                            "algorithmic_bytes": nb}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, inputs)
         print(json.dumps(line), flush=True)
@@ -593,6 +631,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prenorm", action="store_true",
                     help="time the feed-forward block: the RMSNorm prologue, then the MoE layer")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay each step's op chain as one captured CUDA graph")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least three untimed warm-up steps
     dense = args.workload in mw.DENSE_WORKLOADS

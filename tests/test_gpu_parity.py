@@ -247,3 +247,42 @@ def test_random_shapes(shape):
     L = moe.Layer.from_workload(w)
     r = run_forward(L, to_device(inputs))
     check_all(w, inputs, r)
+
+
+@pytest.mark.parametrize("shape", [(32, 512, 16, 4, 1, 256, "bf16"), (300, 256, 12, 3, 2, 320, "bf16")],
+                         ids=["decode-T32", "T300"])
+def test_forward_in_cuda_graph(shape):
+    """moe_forward captured once in a CUDA graph and replayed on new inputs
+    gives the eager call's bits (the call path syncs and reads nothing on the
+    host, so a serving loop can replay it)."""
+    w, inputs = small_case(*shape)
+    L = moe.Layer.from_workload(w)
+    d = to_device(inputs)
+    ws = moe.new_workspace(L)
+    x_static = d["x"].clone()
+    out = torch.empty_like(x_static)
+    wsgu, wsd = (d["ws_gate_up"], d["ws_down"]) if w.S else (None, None)
+
+    def call(x, o):
+        moe.moe_forward(L, x, d["w_router"], d["corr_bias"], d["w_gate_up"], d["w_down"], wsgu, wsd,
+                        o, ws)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        call(x_static, out)            # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call(x_static, out)
+    gen = torch.Generator().manual_seed(123)
+    for _ in range(3):
+        x_new = torch.randn(w.T, w.H, generator=gen).to(w.torch_dtype).cuda()
+        x_static.copy_(x_new)
+        g.replay()
+        eager = torch.empty_like(out)
+        call(x_new, eager)
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager)
+    assert moe.read_device_status(ws) == 0
