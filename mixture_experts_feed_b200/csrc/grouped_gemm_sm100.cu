@@ -720,6 +720,5 @@ cudaError_t launch_router_logits_sm100(const Layer& L, const void* x, const void
   return launch_mode<kRouter, false>(r, num_sms, stream);
 }
 
-int sm100_gemm_max_smem(int E, int S) { return sm100::smem_bytes<sm100::kGateUp, true>(E, S); }
 
 }  // namespace moe

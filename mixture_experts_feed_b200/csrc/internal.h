@@ -54,7 +54,6 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
                                    const void* ws_down, void* h, void* y_routed, void* y_shared,
                                    int32_t* status, int num_sms, cudaStream_t stream,
                                    bool* map_error, const FfnTiling& tiling = FfnTiling());
-int sm100_gemm_max_smem(int E, int S);
 cudaError_t launch_router_logits_sm100(const Layer& L, const void* x, const void* w_parts,
                                        float* logits, int ld_z, int ksplit, int32_t* status,
                                        int num_sms, cudaStream_t stream, bool* map_error);
