@@ -87,12 +87,26 @@ def check_routing(gpu_idx: torch.Tensor, gpu_w: torch.Tensor, gpu_gamma: Optiona
     idx_g = gpu_idx.to(torch.int64)
     idx_o = ref["topk_idx"]
     gap = ref["gap"]
+    scores = ref["scores"]
+    # The chosen set is unique where the k-th and (k+1)-th scores are more
+    # than DELTA apart; its order is unique where, in addition, every pair of
+    # neighbours among the k chosen is.  Closer neighbours inside the set are
+    # ordered by a decision below fp32 resolution: there the order is checked
+    # for validity only.
     sure = gap > DELTA
-    diff_sure = (idx_g[sure] != idx_o[sure]).any(dim=1)
+    ranked = torch.sort(scores, dim=1, descending=True).values[:, :L.k]
+    inner = (ranked[:, :-1] - ranked[:, 1:]).min(dim=1).values if L.k > 1 else torch.full_like(gap, float("inf"))
+    order_sure = sure & (inner > DELTA)
+    diff_sure = (idx_g[order_sure] != idx_o[order_sure]).any(dim=1)
     assert not bool(diff_sure.any()), (
         f"{int(diff_sure.sum())} certified tokens select differently; first "
-        f"{torch.nonzero(sure).flatten()[diff_sure][:5].tolist()}")
-    scores = ref["scores"]
+        f"{torch.nonzero(order_sure).flatten()[diff_sure][:5].tolist()}")
+    set_only = sure & ~order_sure
+    same_set = (torch.sort(idx_g[set_only], 1).values == torch.sort(idx_o[set_only], 1).values).all(1)
+    assert bool(same_set.all()), f"{int((~same_set).sum())} certified tokens choose a different set"
+    for t in torch.nonzero(set_only).flatten().tolist():
+        cs = scores[t][idx_g[t]]
+        assert bool((cs[1:] <= cs[:-1] + DELTA).all()), f"token {t}: order broken"
     near = torch.nonzero(~sure).flatten()
     for t in near.tolist():
         s = scores[t]
@@ -110,7 +124,7 @@ def check_routing(gpu_idx: torch.Tensor, gpu_w: torch.Tensor, gpu_gamma: Optiona
         np.testing.assert_allclose(gpu_gamma.double().numpy(), g_ref.numpy(), rtol=WEIGHT_RTOL, atol=1e-7)
     total = gpu_w.double().sum(1) + (gpu_gamma.double().sum(1) if L.S else 0)
     np.testing.assert_allclose(total.numpy(), L.route_scale * L.global_scale, rtol=1e-5)
-    return {"near_ties": int(near.numel()),
+    return {"near_ties": int(near.numel()), "order_near_ties": int(set_only.sum()),
             "differ": int((idx_g != idx_o).any(dim=1).sum()),
             "min_gap": float(gap.min()) if gap.numel() else float("inf")}
 
