@@ -286,3 +286,13 @@ def test_forward_in_cuda_graph(shape):
         torch.cuda.synchronize()
         assert torch.equal(out, eager)
     assert moe.read_device_status(ws) == 0
+
+
+def test_maximum_limits():
+    """E = 1024, k = 16, S = 8: the largest layer the header allows (32 scores
+    per lane in the top-k, 1024 compaction blocks, 24 rows summed per token)."""
+    w, inputs = small_case(256, 128, 1024, 16, 8, 64, seed=17)
+    L = moe.Layer.from_workload(w)
+    r = run_chain(L, to_device(inputs))
+    stats, _ = check_all(w, inputs, r)
+    print(f"max limits: {stats}")
