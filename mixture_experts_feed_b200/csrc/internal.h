@@ -35,8 +35,13 @@ cudaError_t launch_router_topk(const Layer& L, const float* logits, int ld, int 
 // permute.cu
 cudaError_t launch_permute(const Layer& L, const int32_t* topk_idx, const uint8_t* padding_mask,
                            const void* x, int32_t* offsets, int32_t* perm_slot, int32_t* inv_perm,
-                           void* x_perm, int32_t* counts, int32_t* status, int num_sms,
-                           cudaStream_t stream);
+                           void* x_perm, int32_t* counts, int32_t* chunk, int32_t* status,
+                           int num_sms, cudaStream_t stream);
+// Chunks of slots the workspace path splits T*k slots into (at most 2048),
+// and the slots per chunk; `chunk` holds E * permute_chunks(T*k) int32.
+// chunk == nullptr selects the workspace-free path (one block per expert).
+int64_t permute_chunk_slots(int64_t slots);
+int64_t permute_chunks(int64_t slots);
 
 // grouped_gemm_sm100.cu (bf16, tcgen05)
 // Tile shape choices of one expert-FFN call: the n-tile width of the

@@ -20,7 +20,7 @@ constexpr size_t kRegionAlign = 1024;
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct WsLayout {
-  size_t status, logits, wparts, counts, topk_w, topk_idx, gamma, offsets, perm_slot, inv_perm, x_perm,
+  size_t status, logits, wparts, counts, chunk, topk_w, topk_idx, gamma, offsets, perm_slot, inv_perm, x_perm,
       h, y_routed, y_shared, x_norm, total;
 };
 
@@ -56,6 +56,7 @@ WsLayout ws_layout(const Layer& L) {
   w.logits = take(T * logits_ld(L) * 4 * router_ksplit(L));
   w.wparts = take(L.dtype == MOE_BF16 ? 3 * static_cast<size_t>(L.E + L.S) * L.H * 2 : 0);
   w.counts = take(static_cast<size_t>(L.E) * 4);
+  w.chunk = take(static_cast<size_t>(L.E) * permute_chunks(Rk) * 4);   // per-chunk expert counts
   w.topk_w = take(Rk * 4);
   w.topk_idx = take(Rk * 4);
   w.gamma = take(T * L.S * 4);
@@ -167,7 +168,8 @@ moe_status_t permute_impl(const Layer& L, const int32_t* topk_idx, const uint8_t
                           void* x_perm, void* ws, cudaStream_t stream) {
   const WsLayout w = ws_layout(L);
   return cuda_status(launch_permute(L, topk_idx, pad, x, offsets, perm_slot, inv_perm, x_perm,
-                                    region<int32_t>(ws, w.counts), region<int32_t>(ws, w.status),
+                                    region<int32_t>(ws, w.counts), region<int32_t>(ws, w.chunk),
+                                    region<int32_t>(ws, w.status),
                                     num_sms(), stream));
 }
 

@@ -81,7 +81,8 @@ extern "C" moe_status_t moe_permute_noalloc(const moe_layer_desc_t* desc, const 
   // workspace there is no status word: an out-of-range expert id is skipped
   // (its slot gets inv_perm = -1) without being reported.
   const cudaError_t e = launch_permute(L, topk_idx, padding_mask, x, expert_offsets, perm_slot,
-                                       inv_perm, x_perm, counts, /*status=*/nullptr,
+                                       inv_perm, x_perm, counts, /*chunk=*/nullptr,
+                                       /*status=*/nullptr,
                                        device_sm_count(), s);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
