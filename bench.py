@@ -45,10 +45,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # this workload, measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum,
 # one pass, first warm-up step); absent until captured for the current build.
 NCU_TRAFFIC_BYTES = {
-    "bf16-T8192-H6144-E128k8S1-I2048": 14133757696,
-    "zipf-bf16-T16384-H6144-E256k8S1-I1024": 8011068160,
-    "dense-bf16-T8192-H6144-I24576": 6732003328,
-    "model-bf16-T4096-H6144-E256k6S2-I3072": 22748480000,
+    "bf16-T8192-H6144-E128k8S1-I2048": 14786637568,
+    "zipf-bf16-T16384-H6144-E256k8S1-I1024": 8327614720,
+    "dense-bf16-T8192-H6144-I24576": 7101638656,
+    "model-bf16-T4096-H6144-E256k6S2-I3072": 22768929536,
 }
 
 
@@ -240,7 +240,9 @@ def gpu_arm(args, world, rank, local):
     off = torch.empty(E + 1, dtype=torch.int32, device=dev)
     ps = torch.empty(T * k, dtype=torch.int32, device=dev)
     ip = torch.empty(T * k, dtype=torch.int32, device=dev)
-    xp = torch.empty(T * k, H, dtype=L.dtype, device=dev)
+    # the permuted copy of x, as moe_forward makes it (--gather-rows: none;
+    # the gate_up GEMM then gathers the routed rows of x itself)
+    xp = None if args.gather_rows else torch.empty(T * k, H, dtype=L.dtype, device=dev)
     yr = torch.empty(T * k, H, dtype=torch.float32, device=dev)
     ys = torch.empty(S * T, H, dtype=torch.float32, device=dev) if S else None
     out = torch.empty(T, H, dtype=L.dtype, device=dev)
@@ -433,6 +435,9 @@ def gpu_arm(args, world, rank, local):
         if graph is not None:
             line["config"]["graph"] = True
             del line["op_ms"]
+        if args.gather_rows:
+            line["config"]["a_rows"] = "gathered from x by the gate_up GEMM (no x_perm copy)"
+            line["gpu_launches"] -= args.steps          # no row-gather launch in the permute
         if args.prenorm:
             # the block: post_attention_layernorm, then the layer
             el_x = 2 if w.dtype == "bf16" else 4
@@ -633,6 +638,8 @@ def main():
                     help="time the feed-forward block: the RMSNorm prologue, then the MoE layer")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step's op chain as one captured CUDA graph")
+    ap.add_argument("--gather-rows", action="store_true",
+                    help="no permuted copy of x: the gate_up GEMM gathers the routed rows")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least three untimed warm-up steps
     dense = args.workload in mw.DENSE_WORKLOADS

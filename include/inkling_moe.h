@@ -119,11 +119,12 @@ moe_status_t moe_route(const moe_layer_desc_t* desc, const void* x, const float*
  * pair becomes one row; rows are ordered by (expert, token) ascending.
  *   topk_idx       [T, k] int32 in, values in [0, E)
  *   padding_mask   [T] uint8 (nonzero = padded) or NULL
- *   x              [T, H] dtype in
+ *   x              [T, H] dtype in (not read, and may be NULL, when x_perm is NULL)
  *   expert_offsets [E+1] int32 out: rows of expert e are [off[e], off[e+1])
  *   perm_slot      [T*k] int32 out: for row r < off[E], the slot t*k+j it holds
  *   inv_perm       [T*k] int32 out: for slot t*k+j, its row, or -1 if padded
- *   x_perm         [T*k, H] dtype out: row r = x[perm_slot[r] / k]
+ *   x_perm         [T*k, H] dtype out: row r = x[perm_slot[r] / k]; or NULL:
+ *                  no row copy (moe_expert_ffn can gather the rows itself)
  * The order is deterministic (no atomics decide it).
  */
 moe_status_t moe_permute(const moe_layer_desc_t* desc, const int32_t* topk_idx,
@@ -165,7 +166,12 @@ moe_status_t moe_permute_noalloc(const moe_layer_desc_t* desc, const int32_t* to
  * and for shared expert s and token t (weight shared_gamma[t*S+s]) the same
  * with x[t] and ws_*[s] into y_shared[s*T + t].  The activated rows are
  * rounded to dtype before the down projection; y rows are written in fp32.
- *   x [T,H], x_perm [T*k,H], expert_offsets, perm_slot, topk_w [T*k],
+ * x_perm may be NULL: the gate_up GEMM then reads row r straight from
+ * x[perm_slot[r] / k] (bf16: TMA gathers of 4 rows into the tile), with the
+ * same results bit for bit and without the [T*k, H] copy (memory saved:
+ * T*k*H elements).  With full tiles this mode is slower than the copy (one
+ * TMA instruction per 4 rows and 64 columns instead of one per tile).
+ *   x [T,H], x_perm [T*k,H] or NULL, expert_offsets, perm_slot, topk_w [T*k],
  *   shared_gamma [T*S] (NULL iff S == 0), weights as above,
  *   y_routed [T*k, H] fp32 out (rows < off[E] written), y_shared [S*T, H] fp32 out.
  */
@@ -188,7 +194,8 @@ moe_status_t moe_combine(const moe_layer_desc_t* desc, const void* y_routed, con
 
 /*
  * moe_forward — InklingMoE.forward in one call: moe_route, moe_permute,
- * moe_expert_ffn, moe_combine with every intermediate in `workspace`.
+ * moe_expert_ffn, moe_combine with every intermediate in `workspace`
+ * (including the permuted copy x_perm [T*k, H]).
  *   out [T, H] dtype.  topk_w, topk_idx, shared_gamma are optional outputs
  *   (NULL: kept in the workspace).  padding_mask may be NULL.
  */

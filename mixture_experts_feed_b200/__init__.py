@@ -211,11 +211,11 @@ def moe_permute(layer: Layer, topk_idx, padding_mask, x, expert_offsets, perm_sl
     L = layer
     _expect(topk_idx, "topk_idx", (L.T, L.k), torch.int32)
     _expect(padding_mask, "padding_mask", (L.T,), torch.uint8, allow_none=True)
-    _expect(x, "x", (L.T, L.H), L.dtype)
+    _expect(x, "x", (L.T, L.H), L.dtype, allow_none=x_perm is None)
     _expect(expert_offsets, "expert_offsets", (L.E + 1,), torch.int32)
     _expect(perm_slot, "perm_slot", (L.T * L.k,), torch.int32)
     _expect(inv_perm, "inv_perm", (L.T * L.k,), torch.int32)
-    _expect(x_perm, "x_perm", (L.T * L.k, L.H), L.dtype)
+    _expect(x_perm, "x_perm", (L.T * L.k, L.H), L.dtype, allow_none=True)   # None: no row copy
     _check(LIB.moe_permute(ctypes.byref(L.desc()), _ptr(topk_idx), _ptr(padding_mask), _ptr(x),
                            _ptr(expert_offsets), _ptr(perm_slot), _ptr(inv_perm), _ptr(x_perm),
                            ws.data_ptr(), ws.numel(), _stream(stream)), "moe_permute")
@@ -229,11 +229,11 @@ def moe_permute_noalloc(layer: Layer, topk_idx, padding_mask, x, expert_offsets,
     L = layer
     _expect(topk_idx, "topk_idx", (L.T, L.k), torch.int32)
     _expect(padding_mask, "padding_mask", (L.T,), torch.uint8, allow_none=True)
-    _expect(x, "x", (L.T, L.H), L.dtype)
+    _expect(x, "x", (L.T, L.H), L.dtype, allow_none=x_perm is None)
     _expect(expert_offsets, "expert_offsets", (L.E + 1,), torch.int32)
     _expect(perm_slot, "perm_slot", (L.T * L.k,), torch.int32)
     _expect(inv_perm, "inv_perm", (L.T * L.k,), torch.int32)
-    _expect(x_perm, "x_perm", (L.T * L.k, L.H), L.dtype)
+    _expect(x_perm, "x_perm", (L.T * L.k, L.H), L.dtype, allow_none=True)   # None: no row copy
     _check(LIB.moe_permute_noalloc(ctypes.byref(L.desc()), _ptr(topk_idx), _ptr(padding_mask),
                                    _ptr(x), _ptr(expert_offsets), _ptr(perm_slot), _ptr(inv_perm),
                                    _ptr(x_perm), _stream(stream)), "moe_permute_noalloc")
@@ -243,7 +243,8 @@ def moe_expert_ffn(layer: Layer, x, x_perm, expert_offsets, perm_slot, topk_w, s
                    w_gate_up, w_down, ws_gate_up, ws_down, y_routed, y_shared, ws, stream=None):
     L = layer
     _expect(x, "x", (L.T, L.H), L.dtype)
-    _expect(x_perm, "x_perm", (L.T * L.k, L.H), L.dtype)
+    # None: the gate_up GEMM gathers the routed rows of x through perm_slot
+    _expect(x_perm, "x_perm", (L.T * L.k, L.H), L.dtype, allow_none=True)
     _expect(expert_offsets, "expert_offsets", (L.E + 1,), torch.int32)
     _expect(perm_slot, "perm_slot", (L.T * L.k,), torch.int32)
     if topk_w.numel() != L.T * L.k or topk_w.dtype != torch.float32 or not topk_w.is_contiguous():

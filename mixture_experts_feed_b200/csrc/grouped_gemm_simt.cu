@@ -27,6 +27,7 @@ struct SimtParams {
   int32_t* status;
   int64_t T, a1_base, a1_stride;
   int E, S, K, N, ld_out, rows_cap;
+  int gather_k;   // gate_up: > 0 = routed row r reads x[perm_slot[r] / gather_k] (A[0] = x)
 };
 
 template <bool GATE_UP>
@@ -57,7 +58,18 @@ __global__ void __launch_bounds__(SB_THREADS) grouped_gemm_simt_kernel(const Sim
     const float* B = p.B[gi.src] + static_cast<int64_t>(gi.b_idx) * p.N * p.K;
     const bool a_ok = m * SB_M + lr < gi.rows;
     const bool b_ok = n * SB_N + lr < p.N;
-    const float* ap = A + (gi.a_row0 + m * SB_M + (a_ok ? lr : 0)) * p.K + lk;
+    int64_t a_src = gi.a_row0 + m * SB_M + (a_ok ? lr : 0);
+    if (GATE_UP && p.gather_k > 0 && gi.src == 0) {
+      // gathered routed rows: the row's token; rows past the group read token 0
+      int tok = 0;
+      if (a_ok) {
+        const int slot = p.perm_slot[a_src];
+        if (slot >= 0 && slot < p.rows_cap) tok = slot / p.gather_k;
+        else record_status(p.status, DEV_BAD_ROW);
+      }
+      a_src = tok;
+    }
+    const float* ap = A + a_src * p.K + lk;
     const float* bp = B + static_cast<int64_t>(n * SB_N + (b_ok ? lr : 0)) * p.K + lk;
     float acc[4][4];
 #pragma unroll
@@ -131,7 +143,9 @@ cudaError_t launch_expert_ffn_f32(const Layer& L, const void* x, const void* x_p
   const unsigned grid = static_cast<unsigned>(num_sms * 4);
 
   SimtParams g{};
-  g.A[0] = static_cast<const float*>(x_perm);
+  // with x_perm null the routed rows are read from x through perm_slot
+  g.A[0] = static_cast<const float*>(x_perm != nullptr ? x_perm : x);
+  g.gather_k = x_perm != nullptr ? 0 : L.k;
   g.A[1] = static_cast<const float*>(x);
   g.B[0] = static_cast<const float*>(w_gate_up);
   g.B[1] = L.S > 0 ? static_cast<const float*>(ws_gate_up) : g.B[0];

@@ -35,7 +35,10 @@
 // Roles (192 threads per CTA, one CTA per SM):
 //   warp 0      TMA producer: per stage, this CTA's A tile [128 rows x 64 K]
 //               and its B rows [BN/2 (pairs) or BN rows x 64 K], 128-byte
-//               swizzle; pair loads signal the rank-0 CTA's barrier.
+//               swizzle; pair loads signal the rank-0 CTA's barrier.  Lane 0
+//               waits on the stages and issues the loads; when the routed A
+//               rows are gathered straight from x (kGateUp without x_perm),
+//               each lane issues one tile::gather4 of 4 of the 128 rows.
 //   warp 1      TMEM allocator and (rank-0 CTA only) MMA issuer, one thread:
 //               4 x tcgen05.mma K16 per stage into one of two accumulators
 //               (2 x BN TMEM columns in each CTA).
@@ -100,6 +103,8 @@ struct alignas(64) GemmParams {
   int rows_cap;               // rows of the routed A operand (bound of offsets)
   int ksplit;                 // kRouter, kDown: K-range splits (each writes its own partial)
   int bn;                     // single-CTA expert launches: n-tile width (32..256, multiple of 32)
+  int gather_k;               // kGateUp: > 0 = routed A rows are gathered from x (tmA[0] over
+                              // [T, H], box one row high): row r reads x[perm_slot[r] / gather_k]
   int64_t split_stride;       // kRouter: elements between partial outputs
 };
 
@@ -233,7 +238,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int total_tiles = s_tile[G];
   if (threadIdx.x == 0 && *s_bad) record_status(p.status, DEV_BAD_ROW);
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     int stage = 0;
     uint32_t phase = 0;
@@ -254,24 +259,65 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int b_row = n * bn + (PAIR ? static_cast<int>(rank) * (n_pad >> 1) : 0);
       // single-CTA expert tiles load only the 128-row boxes the tile covers
       const int b_loads = (PAIR || MODE == kRouter) ? TL::B_LOADS : (n_pad + TL::B_BOX - 1) / TL::B_BOX;
+      // gathered A rows: lane l loads rows 4l..4l+3 of this CTA's 128, from
+      // token perm_slot[row] / gather_k.  Lanes whose 4 rows all lie past
+      // the group load nothing (those rows of the tile keep stale data: their
+      // results are never stored); a lane's rows past the group read token 0.
+      const bool gather = MODE == kGateUp && p.gather_k > 0 && gi.src == 0;
+      const int tile_row0 = tile_first_row(m, gi.rows, SET, BM);   // tile's first row in the group
+      auto gathered_bytes = [&](int r) {      // A bytes the gathers of CTA r bring per stage
+        const int rows_r = min(BM, max(0, gi.rows - tile_row0 - r * BM));
+        return ((rows_r + 3) / 4) * 4 * BK * 2;
+      };
+      int tok[4] = {0, 0, 0, 0};
+      const int first = tile_row0 + static_cast<int>(rank) * BM + 4 * lane;   // row inside the group
+      const bool lane_gathers = gather && first < gi.rows;
+      const int a_bytes = gather ? (PAIR ? gathered_bytes(0) + gathered_bytes(1) : gathered_bytes(0))
+                                 : (PAIR ? 2 : 1) * A_BYTES;
+      if (gather) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (first + q < gi.rows) {
+            const int slot = p.perm_slot[gi.a_row0 + first + q];
+            if (slot >= 0 && slot < p.rows_cap) {
+              tok[q] = slot / p.gather_k;
+            } else {
+              record_status(p.status, DEV_BAD_ROW);
+            }
+          }
+        }
+      }
       bool ok = true;
       for (int kt = kt_begin(ks); kt < kt_begin(ks + 1); ++kt) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, s_abort, p.status)) { ok = false; break; }
+        int got = 1;
+        if (lane == 0) got = mbar_wait(&empty[stage], phase ^ 1u, s_abort, p.status) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
         // router: part 2 (smallest) first, then 1, then 0
         const int kb = MODE == kRouter ? kt % k_blocks : kt;
         const int slice = MODE == kRouter ? 2 - kt / k_blocks : gi.b_idx;
+        uint8_t* a_dst = sA + stage * A_BYTES;
         if (PAIR) {
           // both CTAs' bytes complete on the rank-0 CTA's barrier
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (A_BYTES + TL::B_BYTES));
           const uint32_t bar0 = mapa_shared(&full[stage], 0);
-          tma_load_2d_pair(sA + stage * A_BYTES, tmA, bar0, kb * BK, a_row);
-          tma_load_3d_pair(sB + stage * TL::B_BYTES, tmB, bar0, kb * BK, b_row, slice);
+          if (lane == 0) {
+            if (leader) mbar_arrive_expect_tx(&full[stage], a_bytes + 2 * TL::B_BYTES);
+            if (!gather) tma_load_2d_pair(a_dst, tmA, bar0, kb * BK, a_row);
+            tma_load_3d_pair(sB + stage * TL::B_BYTES, tmB, bar0, kb * BK, b_row, slice);
+          }
+          if (lane_gathers)
+            tma_gather4_pair(a_dst + lane * 4 * BK * 2, tmA, bar0, kb * BK, tok[0], tok[1], tok[2],
+                             tok[3]);
         } else {
-          mbar_arrive_expect_tx(&full[stage], A_BYTES + b_loads * (TL::B_BOX * BK * 2));
-          tma_load_2d(sA + stage * A_BYTES, tmA, &full[stage], kb * BK, a_row);
-          for (int i = 0; i < b_loads; ++i)
-            tma_load_3d(sB + stage * TL::B_BYTES + i * (TL::B_BOX * BK * 2), tmB, &full[stage],
-                        kb * BK, b_row + i * TL::B_BOX, slice);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[stage], a_bytes + b_loads * (TL::B_BOX * BK * 2));
+            if (!gather) tma_load_2d(a_dst, tmA, &full[stage], kb * BK, a_row);
+            for (int i = 0; i < b_loads; ++i)
+              tma_load_3d(sB + stage * TL::B_BYTES + i * (TL::B_BOX * BK * 2), tmB, &full[stage],
+                          kb * BK, b_row + i * TL::B_BOX, slice);
+          }
+          if (lane_gathers)
+            tma_gather4(a_dst + lane * 4 * BK * 2, tmA, &full[stage], kb * BK, tok[0], tok[1],
+                        tok[2], tok[3]);
         }
         last_parity[stage] = static_cast<int>(phase);
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -283,12 +329,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // pair's loads all complete on the rank-0 CTA's barriers; the other CTA
     // is covered by the cluster barrier at the end.
     const uint64_t t0 = globaltimer_ns();
-    for (int i = 0; i < STAGES && leader; ++i) {
+    for (int i = 0; i < STAGES && leader && lane == 0; ++i) {
       if (last_parity[i] < 0) continue;
       while (!mbar_try_wait(&full[i], static_cast<uint32_t>(last_parity[i]))) {
         if (globaltimer_ns() - t0 > kWaitLimitNs) { record_status(p.status, DEV_WAIT_TIMEOUT); break; }
       }
     }
+    __syncwarp();
   } else if (warp == 1 && lane == 0 && leader) {
     // ------------------------------------------------------- MMA issuer
     int stage = 0;
@@ -533,13 +580,14 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 2-D bf16 map over [rows, K] (K contiguous), box [BM rows, BK], 128B swizzle.
-static bool encode_a(CUtensorMap* m, const void* base, int64_t rows, int K) {
+// 2-D bf16 map over [rows, K] (K contiguous), box [box_rows, BK], 128B
+// swizzle: BM rows for tile loads, one row for tile::gather4.
+static bool encode_a(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows = BM) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-  cuuint32_t box[2] = {BK, BM};
+  cuuint32_t box[2] = {BK, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -608,7 +656,8 @@ static cudaError_t launch_mode(const GemmParams& p, int sms, cudaStream_t stream
 
 }  // namespace sm100
 
-// gate_up: A0 = x_perm [T*k, H], A1 = x [T, H]; out0 = h rows [0, T*k),
+// gate_up: A0 = x_perm [T*k, H], or, with x_perm null, x [T, H] gathered
+// row by row through perm_slot; A1 = x [T, H]; out0 = h rows [0, T*k),
 // out1 = h rows T*k + s*T + t.  down: A0 = A1 = h [T*k + S*T, I];
 // out0 = y_routed, out1 = y_shared.
 cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_perm,
@@ -631,8 +680,10 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   // With no routed rows (E == 0: the dense layer) the routed maps are never
   // read; they are encoded over the shared operands so that every map is valid.
   const bool routed = L.E > 0 && Rk > 0;
+  const bool gather = routed && x_perm == nullptr;
   GemmParams g{};
-  bool ok = encode_a(&g.tmA[0], routed ? x_perm : x, routed ? Rk : L.T, L.H) &&
+  bool ok = (gather ? encode_a(&g.tmA[0], x, L.T, L.H, 1)
+                    : encode_a(&g.tmA[0], routed ? x_perm : x, routed ? Rk : L.T, L.H)) &&
             encode_a(&g.tmA[1], x, L.T, L.H);
   if (ok && L.E > 0) ok = encode_b(&g.tmB[0], w_gate_up, L.E, 2 * L.I, L.H, BROWS);
   if (ok && L.S > 0) ok = encode_b(&g.tmB[1], ws_gate_up, L.S, 2 * L.I, L.H, BROWS);
@@ -649,6 +700,7 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   g.rows_cap = static_cast<int>(Rk);
   g.ksplit = 1;
   g.bn = tiling.gate_up_bn;
+  g.gather_k = gather ? L.k : 0;
   // paired groups on CTA pairs, the rest on single CTAs (grouping.cuh); with
   // T <= 128 every group has one m-tile and the pair launch is skipped
   // (E == 0, the dense layer: the host knows the one group's m-tiles and

@@ -20,8 +20,8 @@ constexpr size_t kRegionAlign = 1024;
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct WsLayout {
-  size_t status, logits, wparts, counts, chunk, topk_w, topk_idx, gamma, offsets, perm_slot, inv_perm, x_perm,
-      h, y_routed, y_shared, x_norm, total;
+  size_t status, logits, wparts, counts, chunk, topk_w, topk_idx, gamma, offsets, perm_slot, inv_perm,
+      x_perm, h, y_routed, y_shared, x_norm, total;
 };
 
 // Row stride of the router logits: E+S rounded up to 32 (whole 32-column
@@ -226,6 +226,9 @@ moe_status_t forward_checked(const moe_layer_desc_t* desc, const void* x, const 
   void* y_routed = region<void>(workspace, w.y_routed);
   void* y_shared = region<void>(workspace, w.y_shared);
   MOE_TRY(route_impl(L, x, w_router, corr_bias, tw, ti, sg, workspace, s));
+  // the permuted copy of x: the GEMM's A tiles are then whole TMA boxes (the
+  // row-gathering mode, x_perm = null, issues one TMA per 4 rows and runs
+  // slower once tiles are full)
   MOE_TRY(permute_impl(L, ti, padding_mask, x, offsets, perm_slot, inv_perm, x_perm, workspace, s));
   MOE_TRY(ffn_impl(L, x, x_perm, offsets, perm_slot, tw, sg, w_gate_up, w_down, ws_gate_up,
                    ws_down, y_routed, y_shared, workspace, s));
@@ -402,8 +405,9 @@ moe_status_t moe_permute(const moe_layer_desc_t* desc, const int32_t* topk_idx,
                          size_t workspace_bytes, void* stream) {
   Layer L;
   MOE_TRY(check_desc(desc, &L));
-  if (topk_idx == nullptr || !aligned16(x) || expert_offsets == nullptr || perm_slot == nullptr ||
-      inv_perm == nullptr || !aligned16(x_perm))
+  // x_perm null: no row gather (x is then not read and may be null)
+  if (topk_idx == nullptr || expert_offsets == nullptr || perm_slot == nullptr ||
+      inv_perm == nullptr || (x_perm != nullptr && (!aligned16(x) || !aligned16(x_perm))))
     return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_ws(L, workspace, workspace_bytes));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -422,8 +426,8 @@ moe_status_t moe_expert_ffn(const moe_layer_desc_t* desc, const void* x, const v
                             void* workspace, size_t workspace_bytes, void* stream) {
   Layer L;
   MOE_TRY(check_desc(desc, &L));
-  if (!aligned16(x) || !aligned16(x_perm) || expert_offsets == nullptr || perm_slot == nullptr ||
-      topk_w == nullptr || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(y_routed))
+  if (!aligned16(x) || (x_perm != nullptr && !aligned16(x_perm)) || expert_offsets == nullptr ||
+      perm_slot == nullptr || topk_w == nullptr || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(y_routed))
     return MOE_ERR_INVALID_ARG;
   if (L.S > 0 && (shared_gamma == nullptr || !aligned16(ws_gate_up) || !aligned16(ws_down) ||
                   !aligned16(y_shared)))
@@ -490,9 +494,9 @@ int32_t moe_forward_kernel_count(const moe_layer_desc_t* desc) {
   Layer L;
   if (check_desc(desc, &L) != MOE_OK || L.T == 0) return 0;
   // router: (bf16: split + tensor-core logits | fp32: logits) + top-k (plus
-  // a partial-logit sum when K is split 4 or more ways); permute: count,
-  // scan, compact, gather; experts: gate_up + down (bf16 with T > 128:
-  // CTA-pair launch + single-CTA launch each); combine.
+  // a partial-logit sum when K is split 4 or more ways); permute: chunk
+  // counts, chunk scan, scatter, row gather; experts: gate_up + down (bf16
+  // with T > 128: CTA-pair launch + single-CTA launch each); combine.
   const int experts = L.dtype == MOE_BF16 ? (L.T > 128 ? 4 : 2) : 2;
   return (L.dtype == MOE_BF16 ? 2 : 1) + router_topk_launches(router_ksplit(L)) + 4 + experts + 1;
 }

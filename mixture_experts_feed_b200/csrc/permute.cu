@@ -18,7 +18,8 @@
 // Without one (moe_permute_noalloc): perm_count (totals only), perm_scan,
 // and perm_compact: one block per expert walks the tokens in order.
 //   gather_rows   x_perm[r] = x[perm_slot[r] / k], one warp per row,
-//                 16-byte coalesced copies
+//                 16-byte coalesced copies; skipped when x_perm is null (the
+//                 gate_up GEMM then gathers the rows of x itself)
 #include <algorithm>
 
 #include <cuda_bf16.h>
@@ -306,7 +307,18 @@ __global__ void gather_rows_kernel(const TX* __restrict__ x, const int32_t* __re
     }
     const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(slot / k) * H);
     uint4* dst = reinterpret_cast<uint4*>(x_perm + r * H);
-    for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+    // eight 16-byte loads in flight per lane before their stores; the copy
+    // is written evict-first so that x keeps its place in L2
+    constexpr int U = 8;
+    int v = lane;
+    for (; v + 32 * (U - 1) < nvec; v += 32 * U) {
+      uint4 t[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) t[u] = __ldg(src + v + 32 * u);
+#pragma unroll
+      for (int u = 0; u < U; ++u) __stcs(dst + v + 32 * u, t[u]);
+    }
+    for (; v < nvec; v += 32) __stcs(dst + v, __ldg(src + v));
   }
 }
 
@@ -348,6 +360,7 @@ cudaError_t launch_permute(const Layer& L, const int32_t* topk_idx, const uint8_
     perm_compact_kernel<<<L.E, COMPACT_THREADS, 0, stream>>>(topk_idx, padding_mask, L.T, L.k,
                                                              offsets, perm_slot, inv_perm);
   }
+  if (x_perm == nullptr) return cudaGetLastError();   // rows are gathered by the consumer
   const unsigned ggrid = static_cast<unsigned>(
       std::min<int64_t>(ceil_div(slots, 8), static_cast<int64_t>(num_sms) * 8));
   if (L.dtype == MOE_BF16)

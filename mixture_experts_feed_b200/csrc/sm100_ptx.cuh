@@ -205,6 +205,34 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
 
 // TMA tile loads into this CTA's shared memory whose completion is counted
 // on an mbarrier of either CTA of the pair (`bar` is a cluster address).
+// Four rows r0..r3 of a 2-D map whose box is one row high (box width BK),
+// column c0, written to dst as four consecutive box rows (4 x 128 bytes with
+// a 64 x bf16 box); the swizzle follows the destination address, so a
+// gather into offset 512*i of a 1024-byte-aligned tile fills rows 4i..4i+3
+// exactly as one tile load of 128 rows would.
+__device__ __forceinline__ void tma_gather4(void* dst, const void* tmap, uint64_t* bar, int32_t c0,
+                                            int32_t r0, int32_t r1, int32_t r2, int32_t r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1),
+      "r"(r2), "r"(r3)
+      : "memory");
+}
+
+// tma_gather4 for a CTA pair: the bytes complete on `bar`, a barrier of the
+// pair's rank-0 CTA (as tma_load_2d_pair).
+__device__ __forceinline__ void tma_gather4_pair(void* dst, const void* tmap, uint32_t bar,
+                                                 int32_t c0, int32_t r0, int32_t r1, int32_t r2,
+                                                 int32_t r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
+      "r"(r3)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const void* tmap, uint32_t bar,
                                                  int32_t c0, int32_t c1) {
   asm volatile(

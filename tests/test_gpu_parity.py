@@ -185,6 +185,67 @@ def test_expert_ffn_from_oracle_routing():
                      strict=False)
 
 
+@pytest.mark.parametrize("shape,heavy", [
+    ((600, 256, 6, 2, 1, 192, "bf16"), False),    # about 200 rows an expert: CTA pairs, ragged tails
+    ((1100, 256, 16, 2, 1, 128, "bf16"), False),  # 1 to 4 m-tiles an expert: pairs and single CTAs
+    ((1100, 256, 16, 2, 1, 128, "bf16"), True),   # expert 0 takes every token: 9 m-tiles, the
+                                                  # last pair's second CTA has no rows
+    ((40, 256, 64, 4, 1, 128, "bf16"), False),    # decode-like: a few rows in each 128-row tile
+    ((300, 128, 12, 3, 2, 64, "f32"), False),     # the fp32 CUDA-core path
+], ids=["bf16-pairs", "bf16-mixed", "bf16-one-heavy-expert", "bf16-sparse-tiles", "f32"])
+@pytest.mark.parametrize("padded", [False, True])
+def test_gathered_rows_equal_the_permuted_copy(shape, heavy, padded):
+    """moe_expert_ffn with x_perm = None reads each routed row straight from
+    x through perm_slot; the results equal, bit for bit, those computed from
+    the permuted copy of x.  moe_permute with x_perm = None gives the same
+    offsets and permutation as with the copy."""
+    w, inputs = small_case(*shape)
+    if heavy:
+        inputs["corr_bias"] = torch.zeros(w.E)
+        inputs["corr_bias"][0] = 5.0           # every token ranks expert 0 first
+    L = moe.Layer.from_workload(w)
+    d = to_device(inputs)
+    ws = moe.new_workspace(L)
+    T, k, S, H = w.T, w.k, w.S, w.H
+    pm = None
+    if padded:
+        pm = (torch.arange(T) % 7 == 3).to(torch.uint8).cuda()
+    tw = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    ti = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    sg = torch.empty(T, S, dtype=torch.float32, device="cuda") if S else None
+    moe.moe_route(L, d["x"], d["w_router"], d["corr_bias"], tw, ti, sg, ws)
+
+    def permute(with_copy):
+        off = torch.empty(w.E + 1, dtype=torch.int32, device="cuda")
+        ps = torch.full((T * k,), -7, dtype=torch.int32, device="cuda")
+        ip = torch.full((T * k,), -7, dtype=torch.int32, device="cuda")
+        xp = torch.empty(T * k, H, dtype=L.dtype, device="cuda") if with_copy else None
+        moe.moe_permute(L, ti, pm, d["x"] if with_copy else None, off, ps, ip, xp, ws)
+        return off, ps, ip, xp
+
+    def ffn(xp, off, ps):
+        yr = torch.zeros(T * k, H, dtype=torch.float32, device="cuda")
+        ys = torch.zeros(S * T, H, dtype=torch.float32, device="cuda") if S else None
+        moe.moe_expert_ffn(L, d["x"], xp, off, ps, tw, sg, d["w_gate_up"], d["w_down"],
+                           d.get("ws_gate_up") if S else None, d.get("ws_down") if S else None,
+                           yr, ys, ws)
+        return yr, ys
+
+    off, ps, ip, xp = permute(True)
+    off2, ps2, ip2, _ = permute(False)
+    y_copy, ys_copy = ffn(xp, off, ps)
+    y_gath, ys_gath = ffn(None, off, ps)
+    torch.cuda.synchronize()
+    assert moe.read_device_status(ws) == 0
+    assert torch.equal(off, off2) and torch.equal(ip, ip2)
+    R = int(off[-1])
+    assert torch.equal(ps[:R], ps2[:R])
+    assert R < T * k if padded else R == T * k
+    assert torch.equal(y_copy[:R], y_gath[:R])
+    if S:
+        assert torch.equal(ys_copy, ys_gath)
+
+
 def test_out_of_range_expert_id_is_reported_not_faulted():
     w, inputs = small_case(64, 128, 8, 2, 1, 64)
     L = moe.Layer.from_workload(w)
