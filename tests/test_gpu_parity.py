@@ -246,6 +246,38 @@ def test_gathered_rows_equal_the_permuted_copy(shape, heavy, padded):
         assert torch.equal(ys_copy, ys_gath)
 
 
+@pytest.mark.parametrize("T,E,k", [(70000, 256, 8), (300000, 7, 2), (5, 1024, 16)],
+                         ids=["T70000-E256-k8", "T300000-E7-k2", "T5-E1024-k16"])
+def test_permutation_many_chunks(T, E, k):
+    """The stable (expert, token) order at sizes whose T*k slots split into
+    up to 2048 chunks of more than 256 slots each (560000 and 600000 slots:
+    chunks of 512), with skewed ids, repeated ids inside a token and padded
+    tokens: bit-exact against the oracle."""
+    H = 64
+    g = torch.Generator().manual_seed(T + E)
+    # skewed: about a third of the choices go to the first few experts
+    u = torch.rand(T, k, generator=g)
+    idx = torch.where(u < 0.35, torch.randint(0, min(E, 4), (T, k), generator=g),
+                      torch.randint(0, E, (T, k), generator=g)).to(torch.int32)
+    pm = (torch.rand(T, generator=g) < 0.1).to(torch.uint8)
+    L = moe.Layer(T, H, E, k, 0, 64)
+    ws = moe.new_workspace(L)
+    x = torch.randn(T, H, generator=g).to(torch.bfloat16).cuda()
+    out = {n: torch.full((T * k,), -7, dtype=torch.int32, device="cuda") for n in ("ps", "ip")}
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    xp = torch.empty(T * k, H, dtype=torch.bfloat16, device="cuda")
+    moe.moe_permute(L, idx.cuda(), pm.cuda(), x, off, out["ps"], out["ip"], xp, ws)
+    torch.cuda.synchronize()
+    assert moe.read_device_status(ws) == 0
+    ref = oracle.permute(idx.to(torch.int64), E, pm)
+    R = int(ref["offsets"][-1])
+    assert torch.equal(off.cpu().to(torch.int64), ref["offsets"])
+    assert torch.equal(out["ps"][:R].cpu().to(torch.int64), ref["perm_slot"])
+    assert torch.equal(out["ip"].cpu().to(torch.int64), ref["inv_perm"])
+    tok = ref["perm_slot"] // k
+    assert torch.equal(xp[:R].cpu(), x.cpu()[tok])
+
+
 def test_out_of_range_expert_id_is_reported_not_faulted():
     w, inputs = small_case(64, 128, 8, 2, 1, 64)
     L = moe.Layer.from_workload(w)

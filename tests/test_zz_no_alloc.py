@@ -37,7 +37,8 @@ def _noalloc_call(lib, L, idx, pm, x, bufs, stream):
         ctypes.c_void_p(xp.data_ptr()), ctypes.c_void_p(stream))
 
 
-@pytest.mark.parametrize("T,H,E,k,pad", [(300, 256, 12, 3, False), (1000, 128, 64, 6, True)])
+@pytest.mark.parametrize("T,H,E,k,pad", [(300, 256, 12, 3, False), (1000, 128, 64, 6, True),
+                                         (70000, 64, 256, 8, True)])   # 1094 chunks of 512 slots
 def test_noalloc_permute_matches_workspace_permute_twice(T, H, E, k, pad):
     import mixture_experts_feed_b200 as moe
     w = mw.tiny(T=T, H=H, E=E, k=k, S=1, I=64, dtype="bf16", seed=31)
