@@ -8,9 +8,9 @@
 //   perm_chunk_count  per chunk of slots, per-expert counts (block
 //                     histogram), added into the totals; -1 in inv_perm for
 //                     padded slots and slots with an out-of-range expert id
-//   perm_scan         exclusive scan of the totals -> expert_offsets[E+1],
-//                     then each expert's running sum over the chunks: the
-//                     first row of (chunk, expert)
+//   perm_chunk_scan   one block per expert: expert_offsets[e] (the totals
+//                     of the experts before e), then the expert's running
+//                     sum over the chunks: the first row of (expert, chunk)
 //   perm_scatter      per chunk, 32 consecutive slots a warp: a slot's rank
 //                     among earlier slots of its expert is its rank in its
 //                     warp's match group plus the earlier warps' and
