@@ -183,7 +183,7 @@ def cpu_baseline(w, inputs, budget_s: float = 15.0):
     """The oracle as it stands on the host cores, on a bounded token sample."""
     threads = len(os.sched_getaffinity(0))
     per_token_guess = max(1e-3, mw.flops(w, 1)["total"] / 60e9)   # rough fp64 rate
-    n = int(max(4, min(w.T, 256, budget_s / per_token_guess / 2)))
+    n = int(max(4, min(w.T, budget_s / per_token_guess)))          # about 10-20 s of CPU work
     tps, done, secs = oracle_run(w, inputs, n, 1, 0, threads)
     return {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"{done} seeded tokens of {w.name} (oracle fp64, {secs:.1f} s)"}
