@@ -407,7 +407,9 @@ def gpu_arm(args, world, rank, local):
             roof = {"bound": "hbm", "achieved": ffn_bytes / ffn_s / 1e9, "peak": hbm_peak,
                     "unit": "GB/s", "peak_source": f"{peak_src} hbm_gbs"}
         roof["frac"] = roof["achieved"] / roof["peak"]
-        roof["traffic"] = NCU_TRAFFIC_BYTES.get(w.name)
+        # the captured bytes are those of the launches reading x_perm; the
+        # row-gathering mode reads x instead and has no capture
+        roof["traffic"] = None if args.gather_rows else NCU_TRAFFIC_BYTES.get(w.name)
         roof["algorithmic_bytes"] = ffn_bytes
         roof["algorithmic_flops"] = ffn_flops
         roof["touched_groups"] = touched
