@@ -48,6 +48,8 @@
 // chain) overlap the MMAs of the next.  All waits are bounded
 // (sm100_ptx.cuh); on a timeout every role stops, the status word records it
 // and TMEM is released.  No TMA load uses cluster multicast.
+#include <atomic>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -626,14 +628,21 @@ static bool encode_b(CUtensorMap* m, const void* base, int G, int N, int K, int 
 template <int MODE, bool PAIR>
 static cudaError_t launch_mode(const GemmParams& p, int sms, cudaStream_t stream) {
   const int smem = smem_bytes<MODE, PAIR>(p.E, p.S);
-  static int configured_smem[64] = {0};
+  // the attribute is per device; calls from several host threads may set it
+  // concurrently (same value), devices past 64 set it on every launch
+  static std::atomic<int> configured_smem[64];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && configured_smem[dev] < smem) {
+  const bool cached = dev >= 0 && dev < 64;
+  if (!cached || configured_smem[dev].load(std::memory_order_relaxed) < smem) {
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, PAIR>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    configured_smem[dev] = smem;
+    if (cached) {
+      int seen = configured_smem[dev].load(std::memory_order_relaxed);
+      while (seen < smem && !configured_smem[dev].compare_exchange_weak(seen, smem)) {
+      }
+    }
   }
   if (!PAIR) {
     grouped_gemm_kernel<MODE, PAIR><<<sms, NUM_THREADS, smem, stream>>>(p);

@@ -1,6 +1,7 @@
 // The C ABI of libinklingmoe.so (declared in include/inkling_moe.h): argument
 // checks, workspace layout and the order of launches.  Every step of the
 // layer runs in this library's kernels; there is no host compute path.
+#include <atomic>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -110,17 +111,17 @@ moe_status_t check_ws(const Layer& L, const void* ws, size_t bytes) {
 moe_status_t validate_desc(const moe_layer_desc_t* d, Layer* L) { return check_desc(d, L); }
 
 int device_sm_count() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64];   // 0 = not queried yet; same value from any thread
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (dev < 0 || dev >= 64) return 148;
-  if (cached[dev] == 0) {
-    int n = 0;
+  const bool cacheable = dev >= 0 && dev < 64;
+  int n = cacheable ? cached[dev].load(std::memory_order_relaxed) : 0;
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
       n = 148;
-    cached[dev] = n;
+    if (cacheable) cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
 }
 
 namespace {
