@@ -80,7 +80,16 @@ template <int MODE, bool PAIR_> struct Tile {
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int B_BOX = MODE == kRouter ? BN : 128;  // rows per B tensor-map box
   static constexpr int B_LOADS = B_ROWS / B_BOX;            // boxes per stage
-  static constexpr int STAGES = PAIR ? 6 : 4;
+  // Pipeline stages: one stage = this CTA's A tile followed by its B rows,
+  // stages back to back in one ring of RING_BYTES.  Single-CTA expert
+  // launches with n-tiles of at most 128 columns (half the B bytes a stage)
+  // run NARROW_STAGES stages in the same ring, so that as many weight bytes
+  // stay in flight when the launch only streams weights.
+  static constexpr int STAGES = PAIR ? 6 : 4;               // stages of full-width tiles
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
+  static constexpr int NARROW_STAGES = (!PAIR && MODE != kRouter) ? RING_BYTES / (A_BYTES + B_BYTES / 2) : STAGES;
+  static constexpr int MAX_STAGES = NARROW_STAGES > STAGES ? NARROW_STAGES : STAGES;
   static constexpr int TILE_M = PAIR ? 2 * BM : BM;         // rows per tile
   // two accumulators, allocation rounded up to a power of two
   static constexpr uint32_t TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
@@ -118,13 +127,12 @@ constexpr int STAGE_LD = 36;
 constexpr int STAGE_WARP_BYTES = 5120;
 
 template <int MODE, bool PAIR> struct SmemLayout {
-  static constexpr int STAGES = Tile<MODE, PAIR>::STAGES;
-  static constexpr int kA = 0;
-  static constexpr int kB = STAGES * A_BYTES;
-  static constexpr int kStage = kB + STAGES * Tile<MODE, PAIR>::B_BYTES;   // 4 x STAGE_WARP_BYTES
+  static constexpr int MAX_STAGES = Tile<MODE, PAIR>::MAX_STAGES;
+  static constexpr int kRing = 0;                                   // the stage ring
+  static constexpr int kStage = Tile<MODE, PAIR>::RING_BYTES;       // 4 x STAGE_WARP_BYTES
   static constexpr int kBars = kStage + 4 * STAGE_WARP_BYTES;
-  // full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
-  static constexpr int kNumBars = 2 * STAGES + 5;
+  // full[MAX_STAGES], empty[MAX_STAGES], tfull[2], tempty[2], drain
+  static constexpr int kNumBars = 2 * MAX_STAGES + 5;
   static constexpr int kMisc = kBars + kNumBars * 8;   // tmem base, abort, bad
   static constexpr int kTables = kMisc + 16;
 };
@@ -162,13 +170,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   using TL = Tile<MODE, PAIR>;
   using SL = SmemLayout<MODE, PAIR>;
   constexpr int BN = TL::BN;
-  constexpr int STAGES = TL::STAGES;
+  constexpr int STAGES = TL::MAX_STAGES;   // barrier arrays; the ring runs `stages` of them
   constexpr int SET = TL::SET;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* sA = smem + SL::kA;
-  uint8_t* sB = smem + SL::kB;
+  uint8_t* ring = smem + SL::kRing;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SL::kBars);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
@@ -193,6 +200,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // n-tile width: the MMA's full N, except single-CTA expert launches, which
   // may use narrower tiles (more tiles for layers with few rows)
   const int bn = (PAIR || MODE == kRouter) ? BN : p.bn;
+  // the stage ring: narrow single-CTA tiles (bn <= 128) take half the B bytes
+  // a stage and run NARROW_STAGES stages
+  const bool narrow = TL::NARROW_STAGES != TL::STAGES && bn <= 128;
+  const int stages = narrow ? TL::NARROW_STAGES : TL::STAGES;
+  const int stage_bytes = narrow ? A_BYTES + TL::B_BYTES / 2 : TL::STAGE_BYTES;
+  auto stage_a = [&](int st) { return ring + st * stage_bytes; };            // A tile of a stage
+  auto stage_b = [&](int st) { return ring + st * stage_bytes + A_BYTES; };  // its B rows
   const int n_tiles = (p.N + bn - 1) / bn * ksplit;
   const int k_blocks = p.K / BK;                               // per weight part
   const int k_total = MODE == kRouter ? 3 * k_blocks : k_blocks;
@@ -297,14 +311,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // router: part 2 (smallest) first, then 1, then 0
         const int kb = MODE == kRouter ? kt % k_blocks : kt;
         const int slice = MODE == kRouter ? 2 - kt / k_blocks : gi.b_idx;
-        uint8_t* a_dst = sA + stage * A_BYTES;
+        uint8_t* a_dst = stage_a(stage);
         if (PAIR) {
           // both CTAs' bytes complete on the rank-0 CTA's barrier
           const uint32_t bar0 = mapa_shared(&full[stage], 0);
           if (lane == 0) {
             if (leader) mbar_arrive_expect_tx(&full[stage], a_bytes + 2 * TL::B_BYTES);
             if (!gather) tma_load_2d_pair(a_dst, tmA, bar0, kb * BK, a_row);
-            tma_load_3d_pair(sB + stage * TL::B_BYTES, tmB, bar0, kb * BK, b_row, slice);
+            tma_load_3d_pair(stage_b(stage), tmB, bar0, kb * BK, b_row, slice);
           }
           if (lane_gathers)
             tma_gather4_pair(a_dst + lane * 4 * BK * 2, tmA, bar0, kb * BK, tok[0], tok[1], tok[2],
@@ -314,7 +328,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_arrive_expect_tx(&full[stage], a_bytes + b_loads * (TL::B_BOX * BK * 2));
             if (!gather) tma_load_2d(a_dst, tmA, &full[stage], kb * BK, a_row);
             for (int i = 0; i < b_loads; ++i)
-              tma_load_3d(sB + stage * TL::B_BYTES + i * (TL::B_BOX * BK * 2), tmB, &full[stage],
+              tma_load_3d(stage_b(stage) + i * (TL::B_BOX * BK * 2), tmB, &full[stage],
                           kb * BK, b_row + i * TL::B_BOX, slice);
           }
           if (lane_gathers)
@@ -322,7 +336,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         tok[2], tok[3]);
         }
         last_parity[stage] = static_cast<int>(phase);
-        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        if (++stage == stages) { stage = 0; phase ^= 1u; }
       }
       if (!ok) break;
     }
@@ -369,8 +383,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&full[stage], phase, s_abort, p.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        const uint64_t adesc = smem_desc_kmajor_sw128(smem_u32(sA + stage * A_BYTES));
-        const uint64_t bdesc = smem_desc_kmajor_sw128(smem_u32(sB + stage * TL::B_BYTES));
+        const uint64_t adesc = smem_desc_kmajor_sw128(smem_u32(stage_a(stage)));
+        const uint64_t bdesc = smem_desc_kmajor_sw128(smem_u32(stage_b(stage)));
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           // +32 bytes per K=16 step inside the 128-byte swizzle atom
@@ -385,7 +399,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         if (PAIR) mma_commit_pair(&empty[stage], 0x3);   // frees the stage in both CTAs
         else mma_commit(&empty[stage]);
-        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        if (++stage == stages) { stage = 0; phase ^= 1u; }
         if (chain_end) {
           mma_commit(&tfull[acc]);
           ++it;
