@@ -45,10 +45,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # this workload, measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum,
 # one pass, first warm-up step); absent until captured for the current build.
 NCU_TRAFFIC_BYTES = {
-    "bf16-T8192-H6144-E128k8S1-I2048": 14786637568,
-    "zipf-bf16-T16384-H6144-E256k8S1-I1024": 8327614720,
-    "dense-bf16-T8192-H6144-I24576": 7101638656,
-    "model-bf16-T4096-H6144-E256k6S2-I3072": 22768929536,
+    "bf16-T8192-H6144-E128k8S1-I2048": 18305172224,
+    "zipf-bf16-T16384-H6144-E256k8S1-I1024": 11860349952,
+    "dense-bf16-T8192-H6144-I24576": 14797404672,
+    "model-bf16-T4096-H6144-E256k6S2-I3072": 23088262144,
 }
 
 
