@@ -92,10 +92,22 @@ WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
 
 ORDERED = list(WORKLOADS.values())
 
+# Layers sized for small ncu captures of the tcgen05 kernels (one kernel, a
+# few launches, a few GB on the device): not parity workloads.  The same
+# ad-hoc layer as tiny(T=2048, H=6144, E=24, k=3, S=1, I=2048, "bf16",
+# route_scale=2.5, seed=3): the bench workload's H and I, 25 expert groups,
+# about 1.9 GB of expert weights (more than L2).
+PROFILE_WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
+    Workload("adhoc-T2048-H6144-E24k3S1-I2048-bf16", 2048, 6144, 24, 3, 1, 2048,
+             "bf16", 2.5, 1.0, seed=3),
+]}
+
 
 def by_name(name: str) -> Workload:
     if name in WORKLOADS:
         return WORKLOADS[name]
+    if name in PROFILE_WORKLOADS:
+        return PROFILE_WORKLOADS[name]
     # allow 1-based position as a short name ("1".."6")
     if name.isdigit() and 1 <= int(name) <= len(ORDERED):
         return ORDERED[int(name) - 1]
