@@ -38,8 +38,7 @@
 //               swizzle; pair loads signal the rank-0 CTA's barrier.  Lane 0
 //               waits on the stages and issues the loads; when the routed A
 //               rows are gathered straight from x (kGateUp without x_perm),
-//               the whole warp runs the loop and each lane issues one
-//               tile::gather4 of 4 of the 128 rows.
+//               each lane issues one tile::gather4 of 4 of the 128 rows.
 //   warp 1      TMEM allocator and (rank-0 CTA only) MMA issuer, one thread:
 //               4 x tcgen05.mma K16 per stage into one of two accumulators
 //               (2 x BN TMEM columns in each CTA).
@@ -255,12 +254,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int total_tiles = s_tile[G];
   if (threadIdx.x == 0 && *s_bad) record_status(p.status, DEV_BAD_ROW);
 
-  // the whole warp 0 runs the producer loop only when its lanes gather A
-  // rows; otherwise lane 0 alone issues every load
-  const bool warp_producer = MODE == kGateUp && p.gather_k > 0;
-  if (warp == 0 && (lane == 0 || warp_producer)) {
+  if (warp == 0) {
     // ------------------------------------------------------ TMA producer
-    const uint32_t pmask = warp_producer ? 0xffffffffu : 1u;   // the producing lanes
     int stage = 0;
     uint32_t phase = 0;
     int last_parity[STAGES];
@@ -312,7 +307,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int kt = kt_begin(ks); kt < kt_begin(ks + 1); ++kt) {
         int got = 1;
         if (lane == 0) got = mbar_wait(&empty[stage], phase ^ 1u, s_abort, p.status) ? 1 : 0;
-        if (!__shfl_sync(pmask, got, 0)) { ok = false; break; }
+        if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
         // router: part 2 (smallest) first, then 1, then 0
         const int kb = MODE == kRouter ? kt % k_blocks : kt;
         const int slice = MODE == kRouter ? 2 - kt / k_blocks : gi.b_idx;
@@ -356,7 +351,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (globaltimer_ns() - t0 > kWaitLimitNs) { record_status(p.status, DEV_WAIT_TIMEOUT); break; }
       }
     }
-    __syncwarp(pmask);
+    __syncwarp();
   } else if (warp == 1 && lane == 0 && leader) {
     // ------------------------------------------------------- MMA issuer
     int stage = 0;
