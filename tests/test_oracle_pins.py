@@ -228,9 +228,12 @@ def test_full_layer_against_textbook_pieces():
         np.testing.assert_allclose(r["out"][t].numpy(), want, rtol=1e-11, atol=1e-12)
 
 
-def check_permutation(seed=1, T=37, E=7, k=3, pad=False):
+def check_permutation(seed=1, T=37, E=7, k=3, pad=False, repeats=False):
     rng = np.random.default_rng(seed)
-    idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)])
+    if repeats:   # an expert id may repeat inside a token (caller-given selections)
+        idx = rng.integers(0, E, size=(T, k))
+    else:
+        idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)])
     pm = torch.from_numpy(rng.random(T) < 0.3) if pad else None
     p = oracle.permute(torch.from_numpy(idx), E, pm)
     live = [t for t in range(T) if not (pad and bool(pm[t]))]
@@ -254,6 +257,13 @@ def test_permutation_against_python_sort():
 def test_permutation_with_padding():
     for seed in range(3):
         check_permutation(seed, pad=True)
+
+
+def test_permutation_with_repeated_ids_keeps_choice_order():
+    # rows of one (expert, token) keep the order of their choices j
+    for seed in range(3):
+        check_permutation(seed, T=40, E=3, k=5, repeats=True)
+        check_permutation(seed + 10, T=40, E=3, k=5, pad=True, repeats=True)
 
 
 def test_padding_drops_routed_keeps_shared():
