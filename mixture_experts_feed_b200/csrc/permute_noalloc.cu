@@ -65,9 +65,11 @@ extern "C" moe_status_t moe_permute_noalloc(const moe_layer_desc_t* desc, const 
   const moe_status_t st = validate_desc(desc, &L);
   if (st != MOE_OK) return st;
   if (L.E > kNoAllocMaxExperts) return MOE_ERR_UNSUPPORTED;
-  if (topk_idx == nullptr || x == nullptr || expert_offsets == nullptr || perm_slot == nullptr ||
-      inv_perm == nullptr || x_perm == nullptr ||
-      (reinterpret_cast<uintptr_t>(x) & 15) != 0 || (reinterpret_cast<uintptr_t>(x_perm) & 15) != 0)
+  // as moe_permute: x_perm null means no row copy (x is then not read)
+  if (topk_idx == nullptr || expert_offsets == nullptr || perm_slot == nullptr ||
+      inv_perm == nullptr ||
+      (x_perm != nullptr && (x == nullptr || (reinterpret_cast<uintptr_t>(x) & 15) != 0 ||
+                             (reinterpret_cast<uintptr_t>(x_perm) & 15) != 0)))
     return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (L.T == 0)

@@ -121,6 +121,18 @@ def test_null_and_misaligned_pointers_are_rejected_before_launch():
     assert _status("moe_read_device_status", None, None, None) == 1
 
 
+def test_noalloc_permute_host_checks():
+    L = moe.Layer(16, 128, 8, 2, 1, 64)
+    d = ctypes.byref(L.desc())
+    fake = 1 << 20          # aligned, never dereferenced: the checks fail first
+    f = moe.LIB.moe_permute_noalloc
+    assert f(d, None, None, fake, fake, fake, fake, fake, None) == 1          # no topk_idx
+    assert f(d, fake, None, None, fake, fake, fake, fake, None) == 1          # a copy needs x
+    assert f(d, fake, None, fake + 8, fake, fake, fake, fake, None) == 1      # misaligned x
+    assert f(d, fake, None, fake, fake, fake, fake, fake + 4, None) == 1      # misaligned x_perm
+    assert f(d, fake, None, fake, fake, None, fake, fake, None) == 1          # no perm_slot
+
+
 def test_binding_checks_shapes_on_host():
     L = moe.Layer(4, 128, 8, 2, 1, 64, torch.float32)
     x = torch.zeros(4, 64)   # wrong H, on CPU: rejected before the C call
