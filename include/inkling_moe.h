@@ -39,7 +39,8 @@
  *     fp32 and rounded once, in moe_combine).
  *   - Sizes: T = num_tokens, H = hidden, E = n_routed, k = top_k,
  *     S = n_shared, I = intermediate.  Limits: 1 <= k <= min(E, 16),
- *     E <= 1024, S <= 8, H % 64 == 0, I % 64 == 0, T*(k+S) < 2^31.
+ *     E <= 1024, S <= 8, H % 64 == 0, I % 64 == 0, T <= 2^26,
+ *     T*(k+S) < 2^31 (else MOE_ERR_UNSUPPORTED).
  *     T = 0 is accepted and launches nothing.
  *   - `workspace` is a device buffer of at least moe_workspace_size() bytes.
  *     Its first 256 bytes hold a sticky device status word; zero them once
