@@ -87,6 +87,7 @@ def test_invalid_descriptors_are_rejected():
         moe.Layer(4, 128, 2048, 2, 1, 64),     # E > 1024
         moe.Layer(4, 128, 64, 17, 1, 64),      # k > 16
         moe.Layer(4, 128, 8, 2, 9, 64),        # S > 8
+        moe.Layer(2**26 + 1, 128, 8, 2, 1, 64),  # T > 2^26 (with k + S <= 24, T * (k + S) < 2^31)
     ]
     for L in unsupported:
         assert _status("moe_workspace_size", ctypes.byref(L.desc()), ctypes.byref(n)) == 2
