@@ -8,10 +8,16 @@ shared expert GEMMs, recombination) over one batch of T tokens, through the
 library's C ABI, inputs resident in HBM.  The default workload is the layer
 at the pages' hidden size: T=8192, H=6144, E=128, k=8, S=1, I=2048, bf16.
 
-N > 1 (launched by torch.distributed.run): every rank runs an independent
+N > 1 (launched by torch.distributed.run, or with ``--gpus N`` alone, which
+starts the N ranks itself the same way): every rank runs an independent
 replica on its own GPU with its own token batch; the layer has no exchange
 step, so there is no collective on the data path (weak scaling).  Timing is
 taken on the device with CUDA events and reduced as the max over ranks.
+
+On one GPU the line also carries ``per_config``: the task's other
+workloads (the H=2048 layer, one decode step, the Zipf-skewed layer) timed in
+the same run, each with its expert-GEMM roofline and its whole-step HBM
+fraction.
 
 ``--impl reference`` times the CPU fp64 oracle instead, on a bounded token
 sample per step, on rank 0 only.
@@ -42,14 +48,34 @@ METRIC = "Inkling MoE-layer tokens/s and TFLOP/s (% of B200 bf16 peak / % HBM BW
 DEFAULT_WORKLOAD = "bf16-T8192-H6144-E128k8S1-I2048"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes of one moe_expert_ffn call (its four grouped-GEMM launches) on
-# this workload, measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum,
-# one pass, first warm-up step); absent until captured for the current build.
+# these workloads: ncu dram__bytes_read.sum + dram__bytes_write.sum, one pass,
+# summed over the four launches of one call.  A capture constant, not a
+# measurement of this run: each entry names its capture.  An entry is removed
+# when the kernels change, until it is captured again.
 NCU_TRAFFIC_BYTES = {
-    "bf16-T8192-H6144-E128k8S1-I2048": 18305172224,
-    "zipf-bf16-T16384-H6144-E256k8S1-I1024": 11860349952,
-    "dense-bf16-T8192-H6144-I24576": 14797404672,
-    "model-bf16-T4096-H6144-E256k6S2-I3072": 23088262144,
+    "bf16-T8192-H6144-E128k8S1-I2048": (18305172224, "ncu capture of 2026-12-02, "
+                                        "profiles/counters_bf16-T8192-H6144-E128k8S1-I2048.md"),
+    "zipf-bf16-T16384-H6144-E256k8S1-I1024": (11860349952, "ncu capture of 2026-12-02, "
+                                              "profiles/counters_zipf-bf16-T16384-H6144-E256k8S1-I1024.md"),
+    "dense-bf16-T8192-H6144-I24576": (14797404672, "ncu capture of 2026-12-02, "
+                                      "profiles/counters_dense-bf16-T8192-H6144-I24576.md"),
+    "model-bf16-T4096-H6144-E256k6S2-I3072": (23088262144, "ncu capture of 2026-12-02, "
+                                              "profiles/counters_model-bf16-T4096-H6144-E256k6S2-I3072.md"),
 }
+# The other workloads the benchmark spec states, timed in the same run as the default
+# one (the "per_config" block of the JSON line).
+PER_CONFIG = ["bf16-T4096-H2048-E64k6S2-I1024", "decode-bf16-T32-H6144-E128k8S1-I2048",
+              "zipf-bf16-T16384-H6144-E256k8S1-I1024"]
+# Tokens of the oracle's sample per step (reference arm and cpu_baseline
+# alike, so that the two report the same rate): the oracle converts every
+# touched expert's weights to float64 on each call, so a step of a few tokens
+# would time that set-up alone.
+ORACLE_TOKENS_PER_STEP = 2048
+
+
+def traffic_of(name):
+    t = NCU_TRAFFIC_BYTES.get(name)
+    return (None, None) if t is None else t
 
 
 def load_peaks():
@@ -163,13 +189,14 @@ def finish(world: int):
 
 
 # --------------------------------------------------------- CPU (oracle) arm
-def oracle_run(w, inputs, tokens_per_step: int, steps: int, warmup: int, threads: int):
+def oracle_run(w, inputs, tokens_per_step: int, steps: int, warmup: int, threads: int,
+               seed_offset: int = 0):
     import oracle
     torch.set_num_threads(threads)
     n_done = 0
     t_total = 0.0
     for i in range(warmup + steps):
-        tok = mw.token_sample(w, tokens_per_step, seed_offset=1000 + i)
+        tok = mw.token_sample(w, tokens_per_step, seed_offset=1000 + seed_offset + i)
         t0 = time.perf_counter()
         oracle.moe_forward_workload(inputs, w, tokens=tok, threads=threads)
         dt = time.perf_counter() - t0
@@ -180,19 +207,19 @@ def oracle_run(w, inputs, tokens_per_step: int, steps: int, warmup: int, threads
 
 
 def cpu_baseline(w, inputs, min_s: float = 10.0):
-    """The oracle as it stands on the host cores, on a bounded token sample:
-    samples of 512, 1024, ... tokens until one takes at least ``min_s``
-    seconds or covers the whole batch; that last sample is reported (the
-    oracle's per-expert set-up makes small samples slow per token)."""
+    """The oracle as it stands on the host cores, on bounded token samples of
+    ORACLE_TOKENS_PER_STEP tokens (the reference arm's step): seeded samples
+    until the oracle has run for at least ``min_s`` seconds."""
     threads = len(os.sched_getaffinity(0))
-    n = min(w.T, 512)
-    while True:
-        tps, done, secs = oracle_run(w, inputs, n, 1, 0, threads)
-        if secs >= min_s or n >= w.T:
-            break
-        n = min(w.T, 2 * n)
-    return {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{done} seeded tokens of {w.name} (oracle fp64, {secs:.1f} s)"}
+    n = min(w.T, ORACLE_TOKENS_PER_STEP)
+    done, secs, steps = 0, 0.0, 0
+    while secs < min_s:
+        _, d1, s1 = oracle_run(w, inputs, n, 1, 0, threads, seed_offset=steps)
+        done, secs, steps = done + d1, secs + s1, steps + 1
+        if n >= w.T and steps >= 1 and secs >= min_s / 4:
+            break   # the whole batch once is enough of a sample
+    return {"value": done / secs, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{steps} seeded samples of {n} tokens of {w.name} (oracle fp64, {secs:.1f} s)"}
 
 
 def reference_arm(args, world, rank):
@@ -202,8 +229,8 @@ def reference_arm(args, world, rank):
         return
     inputs = mw.generate(w)
     threads = len(os.sched_getaffinity(0))
-    # bounded sample per step so that warmup + steps stay within a few minutes
-    tokens_per_step = int(max(1, min(64, 240 // max(1, args.steps + args.warmup))))
+    # the same bounded sample per step as cpu_baseline: a few seconds per step
+    tokens_per_step = min(w.T, ORACLE_TOKENS_PER_STEP)
     tps, done, secs = oracle_run(w, inputs, tokens_per_step, args.steps, args.warmup, threads)
     fl = mw.flops(w, 1)["total"]
     line = {
@@ -223,6 +250,126 @@ def reference_arm(args, world, rank):
 
 
 # ----------------------------------------------------------------- GPU arm
+def expert_ffn_bytes(w, touched: int) -> int:
+    """Algorithmic bytes of moe_expert_ffn: the weights of every group with
+    rows (routed experts with a nonzero count, every shared expert) once, the
+    routed A rows (x_perm) and shared A rows (x) read once, h written and read
+    once in the dtype, the fp32 down rows written once."""
+    el = 2 if w.dtype == "bf16" else 4
+    rows = w.T * (w.k + w.S)
+    return touched * 3 * w.H * w.I * el + rows * (w.H * el + 2 * w.I * el + 4 * w.H)
+
+
+def step_bytes(w, touched: int) -> int:
+    """Algorithmic bytes of one layer step: the expert call's bytes, plus the
+    fp32 router bank and bias, x read by the router and the shared experts'
+    row gather, x_perm written, the fp32 rows read back by the combine and
+    the output written."""
+    el = 2 if w.dtype == "bf16" else 4
+    router = 4 * (w.E + w.S) * w.H + 4 * w.E + w.T * w.H * el
+    permute = w.T * w.k * w.H * el
+    combine = 4 * w.T * (w.k + w.S) * w.H + w.T * w.H * el
+    return expert_ffn_bytes(w, touched) + router + permute + combine
+
+
+def gemm_roofline(w, ffn_ms: float, touched: int, peaks, peak_src: str):
+    """Roofline of the expert GEMMs (the four launches of moe_expert_ffn):
+    tensor-bound against the measured burst bf16 peak (the calls are timed in
+    a region of well under a second), or HBM-bound against the measured copy
+    bandwidth when their flops per algorithmic byte fall below the ridge."""
+    fl = mw.flops(w)
+    ffn_flops = fl["routed"] + fl["shared"]
+    ffn_bytes = expert_ffn_bytes(w, touched)
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    s = ffn_ms / 1e3
+    if ffn_flops / ffn_bytes >= peak * 1e12 / (hbm_peak * 1e9):
+        roof = {"bound": "tensor", "achieved": ffn_flops / s / 1e12, "peak": peak,
+                "unit": "TFLOP/s", "peak_source": f"{peak_src} bf16_tflops (burst)"}
+        roof["frac"] = roof["achieved"] / peak
+        roof["frac_of_sustained"] = roof["achieved"] / peak_sus
+    else:
+        roof = {"bound": "hbm", "achieved": ffn_bytes / s / 1e9, "peak": hbm_peak,
+                "unit": "GB/s", "peak_source": f"{peak_src} hbm_gbs"}
+        roof["frac"] = roof["achieved"] / hbm_peak
+    roof["algorithmic_bytes"] = ffn_bytes
+    roof["algorithmic_flops"] = ffn_flops
+    roof["touched_groups"] = touched
+    return roof
+
+
+def time_workload(moe, name: str, steps: int, warmup: int, dev, stream, peaks, peak_src):
+    """One of the task's other workloads, timed in this run: its op chain
+    (route, permute, expert GEMMs, combine) for ``warmup`` + ``steps`` steps
+    on device-resident seeded inputs, CUDA events around every op."""
+    w = mw.by_name(name)
+    inputs = mw.generate(w)
+    L = moe.Layer.from_workload(w)
+    d = {k: v.to(dev).contiguous() for k, v in inputs.items()}
+    del inputs
+    ws = moe.new_workspace(L, device=dev)
+    T, k, S, H, E = L.T, L.k, L.S, L.H, L.E
+    tw = torch.empty(T, k, dtype=torch.float32, device=dev)
+    ti = torch.empty(T, k, dtype=torch.int32, device=dev)
+    sg = torch.empty(T, S, dtype=torch.float32, device=dev) if S else None
+    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    ps = torch.empty(T * k, dtype=torch.int32, device=dev)
+    ip = torch.empty(T * k, dtype=torch.int32, device=dev)
+    xp = torch.empty(T * k, H, dtype=L.dtype, device=dev)
+    yr = torch.empty(T * k, H, dtype=torch.float32, device=dev)
+    ys = torch.empty(S * T, H, dtype=torch.float32, device=dev) if S else None
+    out = torch.empty(T, H, dtype=L.dtype, device=dev)
+    wsgu, wsd = (d["ws_gate_up"], d["ws_down"]) if S else (None, None)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        moe.moe_route(L, d["x"], d["w_router"], d["corr_bias"], tw, ti, sg, ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        moe.moe_permute(L, ti, None, d["x"], off, ps, ip, xp, ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        moe.moe_expert_ffn(L, d["x"], xp, off, ps, tw, sg, d["w_gate_up"], d["w_down"], wsgu,
+                           wsd, yr, ys, ws, stream)
+        if ev is not None:
+            ev[3].record(stream)
+        moe.moe_combine(L, yr, ys, ip, out, ws, stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    moe.read_device_status(ws, stream)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    with ClockSampler(dev.index or 0) as clk:
+        torch.cuda.synchronize(dev)
+        for i in range(steps):
+            step(evs[i])
+        torch.cuda.synchronize(dev)
+    moe.read_device_status(ws, stream)
+    ms = evs[0][0].elapsed_time(evs[-1][4]) / steps
+    op_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i in range(4)]
+    counts = (off[1:] - off[:-1]).cpu()
+    touched = int((counts > 0).sum()) + S
+    roof = gemm_roofline(w, op_ms[2], touched, peaks, peak_src)
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    sb = step_bytes(w, touched)
+    res = {"ms_per_step": ms, "tokens_per_s": T / (ms / 1e3),
+           "tflops": mw.flops(w)["total"] / (ms / 1e3) / 1e12,
+           "op_ms": {"route": op_ms[0], "permute": op_ms[1], "expert_ffn": op_ms[2],
+                     "combine": op_ms[3]},
+           "expert_gemms": roof,
+           "step_hbm": {"algorithmic_bytes": sb, "achieved_gbs": sb / (ms / 1e3) / 1e9,
+                        "frac": sb / (ms / 1e3) / 1e9 / hbm_peak},
+           "clocks": clk.summary()}
+    del d, ws, xp, yr, ys
+    torch.cuda.empty_cache()
+    return res
+
+
 def gpu_arm(args, world, rank, local):
     import mixture_experts_feed_b200 as moe
 
@@ -390,35 +537,19 @@ def gpu_arm(args, world, rank, local):
     if rank == 0:
         peaks, peak_src = load_peaks()
         fl = mw.flops(w)
-        ffn_flops = fl["routed"] + fl["shared"]
         # per-op times need the events between ops; a graph replay has only the
         # step's: the roofline then charges the expert flops with the whole step
-        ffn_s = (op_ms[2] if graph is None else ms_step) / 1e3
-        # algorithmic bytes of moe_expert_ffn: the weights of every group with
-        # rows (routed experts with a nonzero count, every shared expert) once,
-        # x_perm / x rows read once, h written and read once in the dtype, the
-        # fp32 down rows written once
-        el = 2 if w.dtype == "bf16" else 4
+        ffn_ms = op_ms[2] if graph is None else ms_step
         counts = (off[1:] - off[:-1]).cpu()
         touched = int((counts > 0).sum()) + S
-        rows = T * (k + S)
-        ffn_bytes = touched * 3 * H * w.I * el + rows * (H * el + 2 * w.I * el + 4 * H)
-        peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-        hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-        ridge = peak * 1e12 / (hbm_peak * 1e9)
-        if ffn_flops / ffn_bytes >= ridge:
-            roof = {"bound": "tensor", "achieved": ffn_flops / ffn_s / 1e12, "peak": peak,
-                    "unit": "TFLOP/s", "peak_source": f"{peak_src} bf16_tflops_sustained"}
-        else:
-            roof = {"bound": "hbm", "achieved": ffn_bytes / ffn_s / 1e9, "peak": hbm_peak,
-                    "unit": "GB/s", "peak_source": f"{peak_src} hbm_gbs"}
-        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof = gemm_roofline(w, ffn_ms, touched, peaks, peak_src)
         # the captured bytes are those of the launches reading x_perm; the
         # row-gathering mode reads x instead and has no capture
-        roof["traffic"] = None if args.gather_rows else NCU_TRAFFIC_BYTES.get(w.name)
-        roof["algorithmic_bytes"] = ffn_bytes
-        roof["algorithmic_flops"] = ffn_flops
-        roof["touched_groups"] = touched
+        traffic, traffic_src = traffic_of(w.name)
+        roof["traffic"] = None if args.gather_rows else traffic
+        roof["traffic_source"] = None if args.gather_rows or traffic is None else traffic_src
+        hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        sb = step_bytes(w, touched)
         tokens_s = world * T / (ms_step / 1e3)
         line = {
             "metric": METRIC, "value": tokens_s, "unit": "tokens/s", "n_gpus": world,
@@ -436,6 +567,8 @@ def gpu_arm(args, world, rank, local):
             "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
                     "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
+            "step_hbm": {"algorithmic_bytes": sb, "achieved_gbs": sb / (ms_step / 1e3) / 1e9,
+                         "frac": sb / (ms_step / 1e3) / 1e9 / hbm_peak},
             "gpu_launches": (moe.forward_prenorm_kernel_count(L) if args.prenorm
                              else moe.forward_kernel_count(L)) * args.steps,
             "clocks": clocks,
@@ -457,6 +590,13 @@ def gpu_arm(args, world, rank, local):
                                             "peak": hbm_peak, "unit": "GB/s",
                                             "frac": nb / (norm_ms / 1e3) / 1e9 / hbm_peak,
                                             "algorithmic_bytes": nb}
+        if world == 1 and not args.no_per_config and w.name == DEFAULT_WORKLOAD and graph is None:
+            # the task's other workloads, timed in this run with the same
+            # step counts (one GPU only: the replicas time the default one)
+            del d, xp, yr, ys, ws
+            torch.cuda.empty_cache()
+            line["per_config"] = {n: time_workload(moe, n, args.steps, args.warmup, dev, stream,
+                                                   peaks, peak_src) for n in PER_CONFIG}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, inputs)
         print(json.dumps(line), flush=True)
@@ -634,6 +774,19 @@ def dense_gpu_arm(args, world, rank, local):
     finish(world)
 
 
+def relaunch_ranks(n: int) -> int:
+    """Run this script again under torch.distributed.run with n ranks on this
+    node (rendezvous on 127.0.0.1, a free port); returns its exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}",
+           os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -642,6 +795,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time the default workload only (no per_config block)")
     ap.add_argument("--prenorm", action="store_true",
                     help="time the feed-forward block: the RMSNorm prologue, then the MoE layer")
     ap.add_argument("--graph", action="store_true",
@@ -649,6 +804,10 @@ def main():
     ap.add_argument("--gather-rows", action="store_true",
                     help="no permuted copy of x: the gate_up GEMM gathers the routed rows")
     args = ap.parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # N ranks requested without an outer launcher: start them here, one
+        # process per GPU under torch.distributed.run, and exit with its status
+        sys.exit(relaunch_ranks(args.gpus))
     args.warmup = max(3, args.warmup)   # at least three untimed warm-up steps
     dense = args.workload in mw.DENSE_WORKLOADS
     if args.impl == "reference":

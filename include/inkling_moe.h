@@ -144,8 +144,10 @@ moe_status_t moe_permute(const moe_layer_desc_t* desc, const int32_t* topk_idx,
  *     (4 KiB) that every GPU loading the library keeps until exit, so
  *     E must be <= 1024 (else MOE_ERR_UNSUPPORTED).
  *   - The first call on a device looks up that array's device address (a
- *     one-time set-up per device); make that first call before any stream
- *     capture.
+ *     one-time set-up per device) and keeps it for the life of the process;
+ *     make that first call before any stream capture, and do not call
+ *     cudaDeviceReset on that device between calls (a reset would leave the
+ *     kept address pointing at memory the library no longer owns).
  *   - All calls share the array and it keeps the last call's contents; each
  *     call clears it on `stream` first.  Calls that overlap on the GPU
  *     (other streams or threads) race on it: order them.

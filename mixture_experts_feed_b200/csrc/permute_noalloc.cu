@@ -32,8 +32,9 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) int32_t g_permute_scratch[kNoAllocMaxExperts];
 
-// Device address of g_permute_scratch, looked up once per device.  In host
-// code the name g_permute_scratch is a host-side stand-in, not a device
+// Device address of g_permute_scratch, looked up once per device and kept
+// for the life of the process (so no cudaDeviceReset between calls).  In
+// host code the name g_permute_scratch is a host-side stand-in, not a device
 // address, so it must never be passed to a kernel.
 int32_t* g_scratch_ptr[kMaxDevices] = {nullptr};
 std::mutex g_scratch_mutex;

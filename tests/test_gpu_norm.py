@@ -108,9 +108,9 @@ def test_forward_prenorm_full_size():
     nw = mw.norm_weight(w.H, seed=w.seed)
     r, _, _ = run_prenorm(w, inputs, nw)
     xn = oracle.rmsnorm(inputs["x"], nw, EPS, out_dtype=w.torch_dtype)
-    tokens = torch.cat([torch.tensor([0, w.T - 1]), mw.token_sample(w, 30)]).unique()
-    stats, _ = check_all(w, {**inputs, "x": xn}, r, tokens=tokens, strict=True)
-    print(f"prenorm {w.name}: {stats}")
+    stats, _ = check_all(w, {**inputs, "x": xn}, r, strict=True)   # every token
+    print(f"prenorm {w.name}: all {w.T} tokens, max|out - oracle| / RMS = {stats['rel_err']:.4f}; "
+          f"{stats}")
 
 
 def test_dense_prenorm():

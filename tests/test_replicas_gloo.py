@@ -2,7 +2,9 @@
 
 The layer has no exchange step, so N GPUs run N independent replicas; the
 only cross-rank work is the timing reduction (max over ranks) and the
-barriers around the timed region.  These run here as two CPU processes.
+barriers around the timed region.  These run here as two CPU processes, and
+``bench.py --gpus 2`` is run end to end (it starts its own two ranks under
+torch.distributed.run) with the CPU reference arm.
 """
 from __future__ import annotations
 
@@ -59,3 +61,23 @@ def test_reference_arm_nonzero_rank_exits_without_work():
                        timeout=120)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+def test_bench_gpus2_starts_two_ranks_and_prints_one_line():
+    """``bench.py --gpus 2`` with no outer launcher starts two ranks itself
+    (the driver's plain call); rank 0 prints the one JSON line, n_gpus = 2,
+    rank 1 prints nothing.  The CPU reference arm runs on the small fp32
+    workload, so no GPU is needed."""
+    import json
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                        "--impl", "reference", "--workload", "tiny-f32-T64-H128-E8k2S1-I64",
+                        "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["impl"] == "reference"
+    assert line["value"] > 0
