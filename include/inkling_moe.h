@@ -174,6 +174,9 @@ moe_status_t moe_permute_noalloc(const moe_layer_desc_t* desc, const int32_t* to
  * same results bit for bit and without the [T*k, H] copy (memory saved:
  * T*k*H elements).  With full tiles this mode is slower than the copy (one
  * TMA instruction per 4 rows and 64 columns instead of one per tile).
+ *   perm_slot may be NULL when x_perm is given: the rows are then already in
+ *   slot order (row r holds slot r, weight topk_w[r]), as the rows an
+ *   expert-parallel rank receives are (moe_ep_dispatch_prep).
  *   x [T,H], x_perm [T*k,H] or NULL, expert_offsets, perm_slot, topk_w [T*k],
  *   shared_gamma [T*S] (NULL iff S == 0), weights as above,
  *   y_routed [T*k, H] fp32 out (rows < off[E] written), y_shared [S*T, H] fp32 out.
@@ -184,6 +187,46 @@ moe_status_t moe_expert_ffn(const moe_layer_desc_t* desc, const void* x, const v
                             const void* w_gate_up, const void* w_down, const void* ws_gate_up,
                             const void* ws_down, void* y_routed, void* y_shared,
                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * moe_shared_ffn — the shared experts alone (layers page,
+ * InklingSharedExperts.forward(hidden_states, gammas)): for shared expert s
+ * and token t,
+ *   y_shared[s*T + t] = ( gamma[t,s] * silu(G[0::2]) * G[1::2] ) @ ws_down[s]^T,
+ *   G = x[t] @ ws_gate_up[s]^T,
+ * with the arithmetic of moe_expert_ffn (bf16: tensor cores, fp32
+ * accumulation, activated rows rounded to dtype, y rows fp32).  It serves a
+ * rank whose routed experts run elsewhere (expert parallelism).  S >= 1.
+ *   x [T,H] dtype, shared_gamma [T,S] fp32, ws_gate_up [S,2I,H],
+ *   ws_down [S,H,I], y_shared [S*T,H] fp32 out; workspace as moe_workspace_size.
+ */
+moe_status_t moe_shared_ffn(const moe_layer_desc_t* desc, const void* x, const float* shared_gamma,
+                            const void* ws_gate_up, const void* ws_down, void* y_shared,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Number of kernels moe_shared_ffn launches for this layer. */
+int32_t moe_shared_ffn_kernel_count(const moe_layer_desc_t* desc);
+
+/*
+ * moe_ep_dispatch_prep — the sending side of expert parallelism (layers page:
+ * GroupedExperts' expert-parallel sharding; the parallelizer shards
+ * InklingMoE.experts over the expert-parallel mesh).  After moe_permute the
+ * permuted rows are ordered by global expert, so the rows bound for the rank
+ * that owns experts [d*El, (d+1)*El) form one run.  For the R = offsets[E]
+ * permuted rows:
+ *   row_w[r]         = topk_w[perm_slot[r]]   (the routing weight travels
+ *                                              with its row)
+ *   expert_counts[e] = offsets[e+1] - offsets[e]
+ *   expert_offsets [E+1], perm_slot [T*k] (from moe_permute), topk_w [T*k]
+ *   in; row_w [T*k] fp32 out (rows >= R untouched), expert_counts [E] int32
+ *   out.  workspace: any buffer of at least 256 bytes whose head is an
+ *   initialised status word (a moe_workspace_size() workspace will do); a
+ *   slot out of range is recorded there and its row weight is 0.
+ */
+moe_status_t moe_ep_dispatch_prep(const moe_layer_desc_t* desc, const int32_t* expert_offsets,
+                                  const int32_t* perm_slot, const float* topk_w, float* row_w,
+                                  int32_t* expert_counts, void* workspace, size_t workspace_bytes,
+                                  void* stream);
 
 /*
  * moe_combine — InklingMoE.forward recombination:

@@ -71,6 +71,10 @@ LIB.moe_permute.argtypes = [_DESC, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size
 LIB.moe_permute_noalloc.argtypes = [_DESC, _P, _P, _P, _P, _P, _P, _P, _P]
 LIB.moe_expert_ffn.argtypes = [_DESC] + [_P] * 13 + [ctypes.c_size_t, _P]
 LIB.moe_combine.argtypes = [_DESC, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+LIB.moe_shared_ffn.argtypes = [_DESC, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+LIB.moe_shared_ffn_kernel_count.restype = ctypes.c_int32
+LIB.moe_shared_ffn_kernel_count.argtypes = [_DESC]
+LIB.moe_ep_dispatch_prep.argtypes = [_DESC, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 LIB.moe_forward.argtypes = [_DESC] + [_P] * 13 + [ctypes.c_size_t, _P]
 LIB.moe_selftest_wait_timeout.argtypes = [_P, ctypes.c_size_t, ctypes.c_uint32, _P]
 _DDESC = ctypes.POINTER(DenseDesc)
@@ -90,7 +94,8 @@ LIB.moe_dense_prenorm_kernel_count.argtypes = [_DDESC]
 for _f in ("moe_workspace_size", "moe_workspace_init", "moe_read_device_status", "moe_route",
            "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_selftest_wait_timeout", "moe_dense_workspace_size", "moe_dense_mlp",
-           "moe_rmsnorm", "moe_forward_prenorm", "moe_dense_mlp_prenorm"):
+           "moe_rmsnorm", "moe_forward_prenorm", "moe_dense_mlp_prenorm", "moe_shared_ffn",
+           "moe_ep_dispatch_prep"):
     getattr(LIB, _f).restype = ctypes.c_int
 
 
@@ -246,7 +251,8 @@ def moe_expert_ffn(layer: Layer, x, x_perm, expert_offsets, perm_slot, topk_w, s
     # None: the gate_up GEMM gathers the routed rows of x through perm_slot
     _expect(x_perm, "x_perm", (L.T * L.k, L.H), L.dtype, allow_none=True)
     _expect(expert_offsets, "expert_offsets", (L.E + 1,), torch.int32)
-    _expect(perm_slot, "perm_slot", (L.T * L.k,), torch.int32)
+    # perm_slot None (with x_perm given): the rows are already in slot order
+    _expect(perm_slot, "perm_slot", (L.T * L.k,), torch.int32, allow_none=x_perm is not None)
     if topk_w.numel() != L.T * L.k or topk_w.dtype != torch.float32 or not topk_w.is_contiguous():
         raise ValueError("topk_w must be a contiguous fp32 tensor of T*k entries")
     if L.S > 0 and (shared_gamma is None or shared_gamma.numel() != L.T * L.S):
@@ -262,6 +268,40 @@ def moe_expert_ffn(layer: Layer, x, x_perm, expert_offsets, perm_slot, topk_w, s
                               _ptr(w_down), _ptr(ws_gate_up), _ptr(ws_down), _ptr(y_routed),
                               _ptr(y_shared), ws.data_ptr(), ws.numel(), _stream(stream)),
            "moe_expert_ffn")
+
+
+def moe_shared_ffn(layer: Layer, x, shared_gamma, ws_gate_up, ws_down, y_shared, ws, stream=None):
+    """The shared experts alone (``InklingSharedExperts.forward``): y_shared
+    rows s*T + t in fp32."""
+    L = layer
+    _expect(x, "x", (L.T, L.H), L.dtype)
+    _expect(shared_gamma, "shared_gamma", (L.T, L.S), torch.float32)
+    _expect(ws_gate_up, "ws_gate_up", (L.S, 2 * L.I, L.H), L.dtype)
+    _expect(ws_down, "ws_down", (L.S, L.H, L.I), L.dtype)
+    _expect(y_shared, "y_shared", (L.S * L.T, L.H), torch.float32)
+    _check(LIB.moe_shared_ffn(ctypes.byref(L.desc()), _ptr(x), _ptr(shared_gamma),
+                              _ptr(ws_gate_up), _ptr(ws_down), _ptr(y_shared), ws.data_ptr(),
+                              ws.numel(), _stream(stream)), "moe_shared_ffn")
+
+
+def shared_ffn_kernel_count(layer: Layer) -> int:
+    return int(LIB.moe_shared_ffn_kernel_count(ctypes.byref(layer.desc())))
+
+
+def moe_ep_dispatch_prep(layer: Layer, expert_offsets, perm_slot, topk_w, row_w, expert_counts,
+                         ws, stream=None):
+    """Routing weight of every permuted row and the per-expert row counts
+    (the sending side of expert parallelism)."""
+    L = layer
+    _expect(expert_offsets, "expert_offsets", (L.E + 1,), torch.int32)
+    _expect(perm_slot, "perm_slot", (L.T * L.k,), torch.int32)
+    if topk_w.numel() != L.T * L.k or topk_w.dtype != torch.float32 or not topk_w.is_contiguous():
+        raise ValueError("topk_w must be a contiguous fp32 tensor of T*k entries")
+    _expect(row_w, "row_w", (L.T * L.k,), torch.float32)
+    _expect(expert_counts, "expert_counts", (L.E,), torch.int32)
+    _check(LIB.moe_ep_dispatch_prep(ctypes.byref(L.desc()), _ptr(expert_offsets), _ptr(perm_slot),
+                                    _ptr(topk_w), _ptr(row_w), _ptr(expert_counts), ws.data_ptr(),
+                                    ws.numel(), _stream(stream)), "moe_ep_dispatch_prep")
 
 
 def moe_combine(layer: Layer, y_routed, y_shared, inv_perm, out, ws, stream=None):

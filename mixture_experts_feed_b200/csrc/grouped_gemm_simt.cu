@@ -106,7 +106,9 @@ __global__ void __launch_bounds__(SB_THREADS) grouped_gemm_simt_kernel(const Sim
         if (GATE_UP) {
           float w;
           if (gi.src == 0) {
-            const int slot = p.perm_slot[gi.a_row0 + r];
+            // no perm_slot: the rows are already in slot order (row r is slot r)
+            const int slot = p.perm_slot != nullptr ? p.perm_slot[gi.a_row0 + r]
+                                                    : static_cast<int>(gi.a_row0 + r);
             if (slot >= 0 && slot < p.rows_cap) {
               w = p.topk_w[slot];
             } else {

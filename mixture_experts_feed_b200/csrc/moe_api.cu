@@ -427,8 +427,10 @@ moe_status_t moe_expert_ffn(const moe_layer_desc_t* desc, const void* x, const v
                             void* workspace, size_t workspace_bytes, void* stream) {
   Layer L;
   MOE_TRY(check_desc(desc, &L));
+  // perm_slot may be NULL only with x_perm given: rows already in slot order
   if (!aligned16(x) || (x_perm != nullptr && !aligned16(x_perm)) || expert_offsets == nullptr ||
-      perm_slot == nullptr || topk_w == nullptr || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(y_routed))
+      (perm_slot == nullptr && x_perm == nullptr) || topk_w == nullptr || !aligned16(w_gate_up) ||
+      !aligned16(w_down) || !aligned16(y_routed))
     return MOE_ERR_INVALID_ARG;
   if (L.S > 0 && (shared_gamma == nullptr || !aligned16(ws_gate_up) || !aligned16(ws_down) ||
                   !aligned16(y_shared)))
@@ -438,6 +440,44 @@ moe_status_t moe_expert_ffn(const moe_layer_desc_t* desc, const void* x, const v
   return ffn_impl(L, x, x_perm, expert_offsets, perm_slot, topk_w, shared_gamma, w_gate_up, w_down,
                   ws_gate_up, ws_down, y_routed, y_shared, workspace,
                   static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_shared_ffn(const moe_layer_desc_t* desc, const void* x, const float* shared_gamma,
+                            const void* ws_gate_up, const void* ws_down, void* y_shared,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  Layer L;
+  MOE_TRY(check_desc(desc, &L));
+  if (L.S == 0) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || shared_gamma == nullptr || !aligned16(ws_gate_up) || !aligned16(ws_down) ||
+      !aligned16(y_shared))
+    return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(L, workspace, workspace_bytes));
+  if (L.T == 0) return MOE_OK;
+  // the S shared groups alone: no routed group (E = 0, k = 0)
+  const WsLayout w = ws_layout(L);
+  Layer Ls = L;
+  Ls.E = 0;
+  Ls.k = 0;
+  void* h = region<void>(workspace, w.h);
+  int32_t* status = region<int32_t>(workspace, w.status);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (L.dtype == MOE_BF16) {
+    bool map_error = false;
+    const cudaError_t e = launch_expert_ffn_bf16(Ls, x, x, nullptr, nullptr, nullptr, shared_gamma,
+                                                 nullptr, nullptr, ws_gate_up, ws_down, h, y_shared,
+                                                 y_shared, status, num_sms(), s, &map_error);
+    if (map_error) return MOE_ERR_INVALID_ARG;
+    return cuda_status(e);
+  }
+  return cuda_status(launch_expert_ffn_f32(Ls, x, x, nullptr, nullptr, nullptr, shared_gamma,
+                                           nullptr, nullptr, ws_gate_up, ws_down, h, y_shared,
+                                           y_shared, status, num_sms(), s));
+}
+
+int32_t moe_shared_ffn_kernel_count(const moe_layer_desc_t* desc) {
+  Layer L;
+  if (check_desc(desc, &L) != MOE_OK || L.T == 0 || L.S == 0) return 0;
+  return 2;   // gate_up + down, each one launch (all S groups have T rows)
 }
 
 moe_status_t moe_combine(const moe_layer_desc_t* desc, const void* y_routed, const void* y_shared,

@@ -11,7 +11,18 @@
 // bf16 is done here on the fp64 bit pattern, round to nearest with ties to
 // even, in one step.
 //
-// One warp per token row, 16-byte vectors along the row, streamed twice:
+// Rows of up to 1024 vectors (bf16: H <= 8192; fp32: H <= 4096) run in
+// rmsnorm_rows_kernel: a team of TPR threads (32..256, one to eight warps)
+// per row, each thread holding up to four 16-byte vectors of its row in
+// registers.  Every vector of the row is loaded at once (one HBM read per
+// element, all of a row's loads in flight together), each thread adds its
+// squares into fp64 partials per element position, the warps reduce by a
+// butterfly and the row's warps' sums are added in warp order through shared
+// memory (a fixed order: the same sum on every run), and the thread scales
+// and stores the vectors it holds.  Longer rows take the streamed kernel
+// below.
+//
+// Streamed kernel: one warp per token row, 16-byte vectors along the row, streamed twice:
 // pass 1 sums the squares, pass 2 re-reads the row (from L1: a few blocks
 // per SM keep their rows there) and writes the result.  Both passes load
 // their vectors in explicit batches (RMS_BATCH vectors a lane in registers
@@ -171,12 +182,101 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// Row-resident variant: TPR = 1 << tpr_log2 threads per row (32..256), each
+// holding VPT vectors; 256 / TPR rows per block.  The loop over row groups
+// is uniform across the block (every thread reaches every barrier).
+template <typename R, int VPT>
+__global__ void __launch_bounds__(kThreads)
+    rmsnorm_rows_kernel(const void* x_, const void* __restrict__ w_, void* out_, int64_t T, int H,
+                        double eps, int tpr_log2) {
+  using Vec = typename R::Vec;
+  __shared__ double s_part[kThreads / 32];
+  const Vec* x = static_cast<const Vec*>(x_);
+  const Vec* w = static_cast<const Vec*>(w_);
+  Vec* out = static_cast<Vec*>(out_);
+  const int nv = H / R::V;
+  const int tpr = 1 << tpr_log2;
+  const int rpb = kThreads >> tpr_log2;                  // rows per block
+  const int r_in_b = threadIdx.x >> tpr_log2;
+  const int t_in_r = threadIdx.x & (tpr - 1);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int wpr = tpr >> 5;                              // warps per row
+  const int first_warp = r_in_b * wpr;
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * rpb; base < T;
+       base += static_cast<int64_t>(gridDim.x) * rpb) {
+    const int64_t t = base + r_in_b;
+    const bool live = t < T;
+    const Vec* row = x + (live ? t : 0) * nv;
+    Vec buf[VPT];
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = t_in_r + j * tpr;
+      if (live && v < nv) buf[j] = row[v];
+    }
+    double part[R::V];
+#pragma unroll
+    for (int i = 0; i < R::V; ++i) part[i] = 0.0;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = t_in_r + j * tpr;
+      if (live && v < nv) R::sumsq(buf[j], part);
+    }
+    double acc = 0.0;
+#pragma unroll
+    for (int i = 0; i < R::V; ++i) acc += part[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) s_part[warp] = acc;
+    __syncthreads();
+    double total = 0.0;
+    for (int i = 0; i < wpr; ++i) total += s_part[first_warp + i];   // warp order
+    __syncthreads();                                     // s_part free for the next rows
+    if (live) {
+      const double inv = 1.0 / sqrt(total / H + eps);
+      const float inv32 = __double2float_rn(inv);
+      Vec* orow = out + t * nv;
+#pragma unroll
+      for (int j = 0; j < VPT; ++j) {
+        const int v = t_in_r + j * tpr;
+        if (v < nv) orow[v] = R::scale(buf[j], w[v], inv32, inv);
+      }
+    }
+  }
+}
+
+template <typename R>
+cudaError_t launch_rows(int64_t T, int H, double eps, const void* x, const void* weight,
+                        void* out, int num_sms, cudaStream_t stream) {
+  const int nv = H / R::V;
+  // the fewest threads per row (32..256) that hold the row in at most 4
+  // vectors a thread; fewer vectors a thread when the row allows it
+  int tpr_log2 = 5;
+  while ((1 << tpr_log2) * 4 < nv && tpr_log2 < 8) ++tpr_log2;
+  const int tpr = 1 << tpr_log2;
+  const int vpt = (nv + tpr - 1) / tpr;
+  const int rpb = kThreads / tpr;
+  const int64_t blocks = (T + rpb - 1) / rpb;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(blocks, static_cast<int64_t>(num_sms) * 8));
+  switch (vpt) {
+    case 1: rmsnorm_rows_kernel<R, 1><<<grid, kThreads, 0, stream>>>(x, weight, out, T, H, eps, tpr_log2); break;
+    case 2: rmsnorm_rows_kernel<R, 2><<<grid, kThreads, 0, stream>>>(x, weight, out, T, H, eps, tpr_log2); break;
+    case 3: rmsnorm_rows_kernel<R, 3><<<grid, kThreads, 0, stream>>>(x, weight, out, T, H, eps, tpr_log2); break;
+    default: rmsnorm_rows_kernel<R, 4><<<grid, kThreads, 0, stream>>>(x, weight, out, T, H, eps, tpr_log2); break;
+  }
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_rmsnorm(int64_t T, int H, int dtype, float eps, const void* x,
                            const void* weight, void* out, int num_sms, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  // one warp per row, 8 rows per block, a few blocks per SM (rows re-read from L1)
+  // rows of at most 1024 vectors: held in registers by a team of threads
+  if (H / (dtype == MOE_BF16 ? Bf16Row::V : F32Row::V) <= 1024)
+    return dtype == MOE_BF16 ? launch_rows<Bf16Row>(T, H, eps, x, weight, out, num_sms, stream)
+                             : launch_rows<F32Row>(T, H, eps, x, weight, out, num_sms, stream);
+  // longer rows: one warp per row, 8 rows per block, a few blocks per SM
+  // (rows re-read from L1)
   const int64_t blocks = (T + kThreads / 32 - 1) / (kThreads / 32);
   const unsigned grid = static_cast<unsigned>(
       std::min<int64_t>(blocks, static_cast<int64_t>(num_sms) * RMS_BLOCKS_PER_SM));

@@ -37,7 +37,11 @@ def gpu_rmsnorm(x, w, eps=EPS, inplace=False):
 
 @pytest.mark.parametrize("T,H,dtype", [(300, 512, torch.bfloat16), (1, 64, torch.bfloat16),
                                        (8192, 6144, torch.bfloat16), (77, 192, torch.float32),
-                                       (1000, 2048, torch.float32)])
+                                       (1000, 2048, torch.float32),
+                                       (1001, 8192, torch.bfloat16),    # 1024 vectors: 4 a thread
+                                       (33, 8256, torch.bfloat16),      # longer rows: streamed kernel
+                                       (20, 4160, torch.float32),       # streamed, fp32
+                                       (5, 2112, torch.bfloat16)])      # 264 vectors, ragged team
 def test_rmsnorm_bitexact(T, H, dtype):
     g = torch.Generator().manual_seed(T + H)
     x = torch.randn(T, H, generator=g).to(dtype)

@@ -399,3 +399,76 @@ def test_maximum_limits():
     r = run_chain(L, to_device(inputs))
     stats, _ = check_all(w, inputs, r)
     print(f"max limits: {stats}")
+
+
+@pytest.mark.parametrize("shape", [(300, 256, 12, 3, 2, 320, "bf16"), (1100, 256, 16, 2, 1, 128, "bf16"),
+                                   (77, 192, 10, 2, 3, 192, "f32")],
+                         ids=["bf16-T300-S2", "bf16-T1100-S1", "f32-T77-S3"])
+def test_shared_ffn_alone(shape):
+    """moe_shared_ffn: every token through every shared expert, weighted by
+    its gamma (InklingSharedExperts.forward), against the oracle's shared
+    experts; and bitwise equal to the shared rows moe_expert_ffn writes."""
+    w, inputs = small_case(*shape)
+    L = moe.Layer.from_workload(w)
+    d = to_device(inputs)
+    ws = moe.new_workspace(L)
+    g = oracle.gate(inputs["x"], inputs["w_router"], inputs["corr_bias"], w.E, w.k, w.S,
+                    w.route_scale, w.global_scale)
+    gamma = g["shared_gamma"].float().contiguous()
+    ys = torch.full((w.S * w.T, w.H), float("nan"), dtype=torch.float32, device="cuda")
+    moe.moe_shared_ffn(L, d["x"], gamma.cuda(), d["ws_gate_up"], d["ws_down"], ys, ws)
+    torch.cuda.synchronize()
+    assert moe.read_device_status(ws) == 0
+    x64 = inputs["x"].double()
+    for s in range(w.S):
+        ref = oracle.expert_mlp(x64, inputs["ws_gate_up"][s].double(), inputs["ws_down"][s].double(),
+                                g["shared_gamma"][:, s])
+        check_output(ys[s * w.T:(s + 1) * w.T].cpu(), ref, L.dtype, f"y_shared[{s}]", strict=False)
+    # the same shared rows as the full expert call, fed the same gammas
+    r = run_chain(L, d)
+    tw = r["topk_w"].cuda()
+    yr = torch.empty(w.T * w.k, w.H, dtype=torch.float32, device="cuda")
+    ys2 = torch.empty_like(ys)
+    moe.moe_expert_ffn(L, d["x"], r["x_perm"].cuda(), r["offsets"].cuda(), r["perm_slot"].cuda(), tw,
+                       gamma.cuda(), d["w_gate_up"], d["w_down"], d["ws_gate_up"], d["ws_down"],
+                       yr, ys2, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(ys, ys2)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_expert_ffn_rows_in_slot_order(dtype):
+    """moe_expert_ffn with perm_slot = None: row r of x_perm is slot r and
+    its weight is topk_w[r] (the rows an expert-parallel rank receives).
+    Against the oracle per expert group, and bitwise equal to passing the
+    identity map explicitly."""
+    R, H, E, I = 700, 256, 9, 192
+    L = moe.Layer(R, H, E, 1, 0, I, torch.bfloat16 if dtype == "bf16" else torch.float32, 1.0, 1.0)
+    w = mw.tiny(T=R, H=H, E=E, k=1, S=1, I=I, dtype=dtype, seed=44)
+    inputs = mw.generate(w, threads=4)
+    gen = torch.Generator().manual_seed(5)
+    counts = torch.bincount(torch.randint(0, E, (R,), generator=gen), minlength=E)
+    counts[3] = 0                                          # an empty group
+    counts[0] += R - int(counts.sum())
+    off = torch.cat([torch.zeros(1, dtype=torch.int64), counts.cumsum(0)]).to(torch.int32)
+    rw = (torch.rand(R, generator=gen) * 2.0).float()
+    x = inputs["x"]
+    d = {k: v.cuda() for k, v in inputs.items()}
+    ws = moe.new_workspace(L)
+    outs = []
+    for ps in (None, torch.arange(R, dtype=torch.int32).cuda()):
+        y = torch.full((R, H), float("nan"), dtype=torch.float32, device="cuda")
+        moe.moe_expert_ffn(L, d["x"], d["x"], off.cuda(), ps, rw.cuda(), None, d["w_gate_up"],
+                           d["w_down"], None, None, y, None, ws)
+        outs.append(y)
+    torch.cuda.synchronize()
+    assert moe.read_device_status(ws) == 0
+    assert torch.equal(outs[0], outs[1])
+    x64 = x.double()
+    ref = torch.empty(R, H, dtype=torch.float64)
+    for e in range(E):
+        a, b = int(off[e]), int(off[e + 1])
+        if b > a:
+            ref[a:b] = oracle.expert_mlp(x64[a:b], inputs["w_gate_up"][e].double(),
+                                         inputs["w_down"][e].double(), rw[a:b].double())
+    check_output(outs[0].cpu(), ref, L.dtype, "rows in slot order", strict=False)
