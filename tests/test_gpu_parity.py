@@ -472,3 +472,40 @@ def test_expert_ffn_rows_in_slot_order(dtype):
             ref[a:b] = oracle.expert_mlp(x64[a:b], inputs["w_gate_up"][e].double(),
                                          inputs["w_down"][e].double(), rw[a:b].double())
     check_output(outs[0].cpu(), ref, L.dtype, "rows in slot order", strict=False)
+
+
+@pytest.mark.parametrize("shape,heavy", [
+    ((1100, 4096, 6, 2, 1, 448, "bf16"), True),    # gate_up N = 896: a 512-wide tile, then 384
+                                                   # (second MMA 128 wide); expert 0 takes every token
+    ((1000, 4096, 3, 3, 1, 320, "bf16"), False),   # k = E: 1000 rows a group (8 m-tiles: pairs);
+                                                   # N = 640: the last tile has no second MMA
+], ids=["H4096-N896-heavy", "H4096-N640-keqE"])
+def test_wide_gate_up_tiles(shape, heavy):
+    """At H >= 4096 the gate_up CTA pairs run 256 x 512 tiles (two N=256 MMAs
+    a K step, one 512-column accumulator released half by half).  Ragged
+    last tiles, the oracle's bar on every row, and the row-gathering mode
+    bit for bit against the copied rows."""
+    w, inputs = small_case(*shape)
+    if heavy:
+        inputs["corr_bias"] = torch.zeros(w.E)
+        inputs["corr_bias"][0] = 5.0
+    L = moe.Layer.from_workload(w)
+    d = to_device(inputs)
+    r = run_chain(L, d)
+    stats, ref = check_all(w, inputs, r)
+    R = int(r["offsets"][-1])
+    slots = r["perm_slot"][:R].to(torch.int64)
+    check_output(r["y_routed"][:R], ref["routed"].reshape(w.T * w.k, w.H)[slots], w.torch_dtype,
+                 "y_routed", strict=False)
+    # the row-gathering mode (x_perm = None) on the same tiles: the same bits
+    ws = moe.new_workspace(L)
+    yr = torch.zeros(w.T * w.k, w.H, dtype=torch.float32, device="cuda")
+    ys = torch.zeros(w.S * w.T, w.H, dtype=torch.float32, device="cuda")
+    moe.moe_expert_ffn(L, d["x"], None, r["offsets"].cuda(), r["perm_slot"].cuda(),
+                       r["topk_w"].cuda(), r["shared_gamma"].cuda(), d["w_gate_up"], d["w_down"],
+                       d["ws_gate_up"], d["ws_down"], yr, ys, ws)
+    torch.cuda.synchronize()
+    assert moe.read_device_status(ws) == 0
+    assert torch.equal(yr[:R].cpu(), r["y_routed"][:R])
+    assert torch.equal(ys.cpu(), r["y_shared"])
+    print(f"wide tiles {w.name}: {stats}")
