@@ -307,7 +307,10 @@ __global__ void gather_rows_kernel(const TX* __restrict__ x, const int32_t* __re
     }
     const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(slot / k) * H);
     uint4* dst = reinterpret_cast<uint4*>(x_perm + r * H);
-    // eight 16-byte loads in flight per lane before their stores
+    // eight 16-byte loads in flight per lane before their stores; the
+    // stores are marked evict-first (streaming), so that the copy, k times
+    // the size of x, does not push the rows of x out of L2 before their
+    // other k - 1 reads
     constexpr int U = 8;
     int v = lane;
     for (; v + 32 * (U - 1) < nvec; v += 32 * U) {
@@ -315,9 +318,9 @@ __global__ void gather_rows_kernel(const TX* __restrict__ x, const int32_t* __re
 #pragma unroll
       for (int u = 0; u < U; ++u) t[u] = __ldg(src + v + 32 * u);
 #pragma unroll
-      for (int u = 0; u < U; ++u) dst[v + 32 * u] = t[u];
+      for (int u = 0; u < U; ++u) __stcs(dst + v + 32 * u, t[u]);
     }
-    for (; v < nvec; v += 32) dst[v] = __ldg(src + v);
+    for (; v < nvec; v += 32) __stcs(dst + v, __ldg(src + v));
   }
 }
 

@@ -100,6 +100,15 @@ ORDERED = list(WORKLOADS.values())
 PROFILE_WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
     Workload("adhoc-T2048-H6144-E24k3S1-I2048-bf16", 2048, 6144, 24, 3, 1, 2048,
              "bf16", 2.5, 1.0, seed=3),
+    # many tokens, small experts: x (201 MB) and the fp32 rows (805 MB) larger
+    # than L2 for the HBM-bound kernels (norm, router, permutation, row
+    # gather, combine), about 2 GB on the device in all
+    Workload("adhoc-T16384-H6144-E16k2S1-I256-bf16", 16384, 6144, 16, 2, 1, 256,
+             "bf16", 2.5, 1.0, seed=3),
+    # one decode step over 17 expert groups (1.3 GB of weights, more than L2):
+    # the weight-streaming expert GEMMs
+    Workload("adhoc-decode-T32-H6144-E16k8S1-I2048-bf16", 32, 6144, 16, 8, 1, 2048,
+             "bf16", 2.5, 1.0, seed=3),
 ]}
 
 

@@ -207,3 +207,45 @@ def test_binding_argtypes_match_the_header():
             assert n == 0, f"{name}: no ctypes prototype for {n} parameters"
         else:
             assert len(fn.argtypes) == n, f"{name}: {len(fn.argtypes)} argtypes, header has {n}"
+
+
+def test_new_entry_points_host_checks():
+    """moe_shared_ffn and moe_ep_dispatch_prep reject bad arguments on the
+    host, before any CUDA call (fake aligned pointers are never touched)."""
+    fake, big = 1 << 20, 1 << 40
+    L = moe.Layer(64, 128, 8, 2, 0, 64)                      # no shared expert
+    d = ctypes.byref(L.desc())
+    assert moe.LIB.moe_shared_ffn(d, fake, fake, fake, fake, fake, fake, big, None) == 1
+    L1 = moe.Layer(64, 128, 8, 2, 1, 64)
+    d1 = ctypes.byref(L1.desc())
+    assert moe.LIB.moe_shared_ffn(d1, fake + 8, fake, fake, fake, fake, fake, big, None) == 1   # misaligned x
+    assert moe.LIB.moe_shared_ffn(d1, fake, None, fake, fake, fake, fake, big, None) == 1       # no gammas
+    assert moe.LIB.moe_shared_ffn(d1, fake, fake, fake, fake, fake, fake, 100, None) == 3       # workspace
+    assert moe.LIB.moe_shared_ffn_kernel_count(d1) == 2
+    assert moe.LIB.moe_shared_ffn_kernel_count(d) == 0
+    L0 = moe.Layer(0, 128, 8, 2, 1, 64)
+    assert moe.LIB.moe_shared_ffn(ctypes.byref(L0.desc()), fake, fake, fake, fake, fake, fake, big,
+                                  None) == 0                 # T = 0: nothing launched
+    for i in range(5):                                        # each required pointer null in turn
+        args = [fake] * 5
+        args[i] = None
+        assert moe.LIB.moe_ep_dispatch_prep(d1, *args, fake, 4096, None) == 1
+    assert moe.LIB.moe_ep_dispatch_prep(d1, fake, fake, fake, fake, fake, fake + 16, 4096, None) == 1
+    assert moe.LIB.moe_ep_dispatch_prep(d1, fake, fake, fake, fake, fake, fake, 100, None) == 1
+
+
+def test_expert_ffn_needs_a_row_map_or_a_copy():
+    """moe_expert_ffn takes perm_slot = NULL only when x_perm is given (rows
+    already in slot order); with neither the rows cannot be found."""
+    fake, big = 1 << 20, 1 << 40
+    L = moe.Layer(64, 128, 8, 2, 0, 64)
+    d = ctypes.byref(L.desc())
+    args = [fake, None, fake, None, fake, None, fake, fake, None, None, fake, None]
+    assert moe.LIB.moe_expert_ffn(d, *args, fake, big, None) == 1
+
+
+def test_ep_partition():
+    from mixture_experts_feed_b200.ep import partition
+    assert partition(128, 8, 3) == (48, 16)
+    with pytest.raises(ValueError):
+        partition(10, 4, 0)
