@@ -41,7 +41,7 @@
 //               each lane issues one tile::gather4 of 4 of the 128 rows.
 //   warp 1      TMEM allocator and (rank-0 CTA only) MMA issuer, one thread:
 //               4 x tcgen05.mma K16 per stage into one of two accumulators
-//               (2 x BN TMEM columns in each CTA).
+//               (2 x BN TMEM columns in each CTA; the router keeps three).
 //   warps 2..5  epilogue: tcgen05.ld this CTA's accumulator rows (warp w
 //               reads TMEM lanes 32*(w%4) .. +31), fused math, global stores.
 // The two accumulators let the epilogue of one tile (or, for kRouter, one K
@@ -62,13 +62,6 @@
 namespace moe {
 namespace sm100 {
 
-#ifndef MOE_WIDE_EARLY_START
-#define MOE_WIDE_EARLY_START 1
-#endif
-#ifndef MOE_WIDE_GATE_UP_MIN_K
-#define MOE_WIDE_GATE_UP_MIN_K 4096   // hidden size from which gate_up pairs take 256 x 512 tiles
-#endif
-
 constexpr int BM = 128;          // A rows per CTA
 constexpr int BK = 64;
 constexpr int A_BYTES = BM * BK * 2;
@@ -78,38 +71,33 @@ constexpr int ROUTER_CHAIN = 2;
 
 enum Mode { kGateUp = 0, kDown = 1, kRouter = 2 };
 
-template <int MODE, bool PAIR_, int NSUB_ = 1> struct Tile {
+template <int MODE, bool PAIR_> struct Tile {
   static constexpr bool PAIR = PAIR_;                       // CTA-pair (M=256) MMAs
-  // MMAs of MMA_N columns a tile spans side by side, sharing each A tile:
-  // 1, or 2 for the wide gate_up tiles of CTA pairs (256 x 512)
-  static constexpr int NSUB = NSUB_;
   // which m-tiles of each group the launch covers (grouping.cuh)
   static constexpr int SET = PAIR ? kPairs : (MODE == kRouter ? kAllTiles : kSingles);
-  static constexpr int MMA_N = MODE == kRouter ? 160 : 256; // N of one MMA
-  static constexpr int BN = MMA_N * NSUB;                   // tile width = accumulator columns
+  static constexpr int BN = MODE == kRouter ? 160 : 256;    // MMA N = accumulator columns
   static constexpr int B_ROWS = PAIR ? BN / 2 : BN;         // B rows one CTA loads
   static constexpr int B_BYTES = B_ROWS * BK * 2;
-  static constexpr int B_BOX = MODE == kRouter ? MMA_N : 128;   // rows per B tensor-map box
+  static constexpr int B_BOX = MODE == kRouter ? BN : 128;  // rows per B tensor-map box
   static constexpr int B_LOADS = B_ROWS / B_BOX;            // boxes per stage
   // Pipeline stages: one stage = this CTA's A tile followed by its B rows,
   // stages back to back in one ring of RING_BYTES.  Single-CTA expert
   // launches with n-tiles of at most 128 columns (half the B bytes a stage)
   // run NARROW_STAGES stages in the same ring, so that as many weight bytes
   // stay in flight when the launch only streams weights.
-  static constexpr int STAGES = PAIR ? (NSUB == 2 ? 4 : 6) : 4;   // stages of full-width tiles
+  static constexpr int STAGES = PAIR ? 6 : 4;               // stages of full-width tiles
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
   static constexpr int NARROW_STAGES = (!PAIR && MODE != kRouter) ? RING_BYTES / (A_BYTES + B_BYTES / 2) : STAGES;
   static constexpr int MAX_STAGES = NARROW_STAGES > STAGES ? NARROW_STAGES : STAGES;
   static constexpr int TILE_M = PAIR ? 2 * BM : BM;         // rows per tile
-  // accumulators: two of BN columns (the epilogue of one tile overlaps the
-  // next tile's MMAs), or one when two would not fit the 512 TMEM columns;
-  // the allocation is rounded up to a power of two
-  // (the router's 160-column accumulation chains: three, so that the MMAs
-  // run a chain further ahead of the epilogue that sums them)
-  static constexpr int NACC = MODE == kRouter ? 3 : (2 * BN <= 512 ? 2 : 1);
+  // accumulators: two (the epilogue of one tile overlaps the next tile's
+  // MMAs); the router's 160-column accumulation chains keep three, so that
+  // the MMAs run a chain further ahead of the epilogue that sums them.  The
+  // allocation is rounded up to a power of two.
+  static constexpr int NACC = MODE == kRouter ? 3 : 2;
   static constexpr uint32_t TMEM_COLS = NACC * BN <= 256 ? 256 : 512;
-  static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, MMA_N);
+  static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, BN);
 };
 
 struct alignas(64) GemmParams {
@@ -142,10 +130,10 @@ constexpr int STAGE_LD = 36;
 // on a 1024-byte boundary, as a 128-byte-swizzled TMA box requires
 constexpr int STAGE_WARP_BYTES = 5120;
 
-template <int MODE, bool PAIR, int NSUB = 1> struct SmemLayout {
-  static constexpr int MAX_STAGES = Tile<MODE, PAIR, NSUB>::MAX_STAGES;
+template <int MODE, bool PAIR> struct SmemLayout {
+  static constexpr int MAX_STAGES = Tile<MODE, PAIR>::MAX_STAGES;
   static constexpr int kRing = 0;                                   // the stage ring
-  static constexpr int kStage = Tile<MODE, PAIR, NSUB>::RING_BYTES; // 4 x STAGE_WARP_BYTES
+  static constexpr int kStage = Tile<MODE, PAIR>::RING_BYTES;       // 4 x STAGE_WARP_BYTES
   static constexpr int kBars = kStage + 4 * STAGE_WARP_BYTES;
   // full[MAX_STAGES], empty[MAX_STAGES], tfull[3], tempty[3], drain
   static constexpr int kNumBars = 2 * MAX_STAGES + 7;
@@ -153,9 +141,9 @@ template <int MODE, bool PAIR, int NSUB = 1> struct SmemLayout {
   static constexpr int kTables = kMisc + 16;
 };
 
-template <int MODE, bool PAIR, int NSUB = 1>
+template <int MODE, bool PAIR>
 __host__ __device__ inline int smem_bytes(int E, int S) {
-  return 1024 /* alignment slack */ + SmemLayout<MODE, PAIR, NSUB>::kTables + 4 * ((E + 1) + (E + S + 1));
+  return 1024 /* alignment slack */ + SmemLayout<MODE, PAIR>::kTables + 4 * ((E + 1) + (E + S + 1));
 }
 
 // Write one warp's 32 rows x 32 fp32 columns through the staging tile so that
@@ -180,22 +168,13 @@ __device__ __forceinline__ void store_rows_f32(float* st, const uint32_t (&v)[32
   __syncwarp();
 }
 
-template <int MODE, bool PAIR, int NSUB = 1>
+template <int MODE, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
-  using TL = Tile<MODE, PAIR, NSUB>;
-  using SL = SmemLayout<MODE, PAIR, NSUB>;
+  using TL = Tile<MODE, PAIR>;
+  using SL = SmemLayout<MODE, PAIR>;
   constexpr int BN = TL::BN;
-  constexpr int MMA_N = TL::MMA_N;
   constexpr int NACC = TL::NACC;
-  // TMEM columns between the two accumulators (0: one accumulator)
-  constexpr int ACC_STRIDE = NACC == 2 ? BN : 0;
-  // Wide tiles (one accumulator of two MMA_N-column halves): the epilogue
-  // releases each half as soon as it has read it (tempty[0], tempty[1]); the
-  // next tile starts on the first half and defers each stage's second-half
-  // MMAs until the second half is free, holding at most all the stages.
-  constexpr bool SPLIT = NSUB == 2 && MOE_WIDE_EARLY_START;
-  static_assert(NSUB == 1 || (NSUB == 2 && PAIR && MODE == kGateUp), "wide tiles: gate_up CTA pairs");
   constexpr int STAGES = TL::MAX_STAGES;   // barrier arrays; the ring runs `stages` of them
   constexpr int SET = TL::SET;
   extern __shared__ uint8_t smem_raw[];
@@ -296,13 +275,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const void* tmB = &p.tmB[gi.src];
       const int a_row = static_cast<int>(gi.a_row0) + tile_first_row(m, gi.rows, SET, BM) +
                         static_cast<int>(rank) * BM;
-      // pairs: this CTA's half of each MMA's (possibly narrowed) N range;
-      // wide tiles (NSUB = 2) load one 128-row box for each of their MMAs
-      const int n_tile = min(bn, p.N - n * bn);
-      const int n_pad = (min(MMA_N, n_tile) + 31) & ~31;
+      // pairs: this CTA's half of the tile's (possibly narrowed) N range
+      const int n_pad = (min(bn, p.N - n * bn) + 31) & ~31;
       const int b_row = n * bn + (PAIR ? static_cast<int>(rank) * (n_pad >> 1) : 0);
-      const int n_pad1 = NSUB == 2 ? (max(0, n_tile - MMA_N) + 31) & ~31 : 0;   // second MMA
-      const int b_row1 = n * bn + MMA_N + (PAIR ? static_cast<int>(rank) * (n_pad1 >> 1) : 0);
       // single-CTA expert tiles load only the 128-row boxes the tile covers
       const int b_loads = (PAIR || MODE == kRouter) ? TL::B_LOADS : (n_pad + TL::B_BOX - 1) / TL::B_BOX;
       // gathered A rows: lane l loads rows 4l..4l+3 of this CTA's 128, from
@@ -346,13 +321,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // both CTAs' bytes complete on the rank-0 CTA's barrier
           const uint32_t bar0 = mapa_shared(&full[stage], 0);
           if (lane == 0) {
-            // each CTA loads one 128-row B box per MMA of the tile
-            const int boxes = NSUB == 2 && n_pad1 > 0 ? 2 : 1;
-            if (leader) mbar_arrive_expect_tx(&full[stage], a_bytes + 2 * boxes * (TL::B_BOX * BK * 2));
+            if (leader) mbar_arrive_expect_tx(&full[stage], a_bytes + 2 * TL::B_BYTES);
             if (!gather) tma_load_2d_pair(a_dst, tmA, bar0, kb * BK, a_row);
             tma_load_3d_pair(stage_b(stage), tmB, bar0, kb * BK, b_row, slice);
-            if (boxes == 2)
-              tma_load_3d_pair(stage_b(stage) + TL::B_BOX * BK * 2, tmB, bar0, kb * BK, b_row1, slice);
           }
           if (lane_gathers)
             tma_gather4_pair(a_dst + lane * 4 * BK * 2, tmA, bar0, kb * BK, tok[0], tok[1], tok[2],
@@ -396,34 +367,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int g, m, nv;
       decode_tile(tile, s_tile, G, s_off, p.E, p.T, SET, BM, g, m, nv);
       const int n = nv / ksplit, ks = nv - n * ksplit;
-      // a narrow or ragged last n-tile runs a narrower MMA (N multiple of 32);
-      // a wide tile's second MMA covers the columns past MMA_N, if any
+      // a narrow or ragged last n-tile runs a narrower MMA (N multiple of 32)
       const int n_here = min(bn, p.N - n * bn);
-      const int n0 = min(MMA_N, n_here), n1 = NSUB == 2 ? max(0, n_here - MMA_N) : 0;
-      const uint32_t idesc = n0 >= MMA_N ? TL::IDESC : idesc_bf16_f32(TL::TILE_M, (n0 + 31) & ~31);
-      const uint32_t idesc1 = n1 >= MMA_N ? TL::IDESC : idesc_bf16_f32(TL::TILE_M, (n1 + 31) & ~31);
+      const uint32_t idesc = n_here >= BN ? TL::IDESC : idesc_bf16_f32(TL::TILE_M, (n_here + 31) & ~31);
       if (MODE != kRouter) {
-        const int acc = it % NACC;   // SPLIT: tempty[0] is the first half
+        const int acc = it % NACC;
         if (!mbar_wait(&tempty[acc], ((it / NACC) & 1) ^ 1u, s_abort, p.status)) { ok = false; break; }
         tc_fence_after();
       }
-      // SPLIT: stages whose second-half MMAs wait for the second half
-      bool hi_free = !SPLIT || it == 0;   // the first tile finds TMEM free
-      int n_def = 0;
-      int def_stage[SPLIT ? TL::MAX_STAGES : 1];
-      bool def_first[SPLIT ? TL::MAX_STAGES : 1];
-      const uint32_t hi_parity = (static_cast<uint32_t>(it) & 1u) ^ 1u;
-      const uint32_t d_hi = tmem_base + MMA_N;
-      // second-half MMAs of a stage, then the stage's release
-      auto issue_hi = [&](int st, bool first) {
-        const uint64_t ad = smem_desc_kmajor_sw128(smem_u32(stage_a(st)));
-        const uint64_t bd = smem_desc_kmajor_sw128(smem_u32(stage_b(st) + TL::B_BOX * BK * 2));
-#pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk)
-          mma_bf16_ss_pair(d_hi, ad + static_cast<uint64_t>(2 * kk), bd + static_cast<uint64_t>(2 * kk),
-                           idesc1, (first && kk == 0) ? 0u : 1u);
-        mma_commit_pair(&empty[st], 0x3);
-      };
       const int kb0 = kt_begin(ks), kb1 = kt_begin(ks + 1);
       for (int kb = kb0; kb < kb1; ++kb) {
         const int acc = it % NACC;
@@ -436,63 +387,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         if (!mbar_wait(&full[stage], phase, s_abort, p.status)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(MODE == kRouter ? acc * BN : (it % NACC) * ACC_STRIDE);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         const uint64_t adesc = smem_desc_kmajor_sw128(smem_u32(stage_a(stage)));
         const uint64_t bdesc = smem_desc_kmajor_sw128(smem_u32(stage_b(stage)));
-        const uint64_t bdesc1 = smem_desc_kmajor_sw128(smem_u32(stage_b(stage) + TL::B_BOX * BK * 2));
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           // +32 bytes per K=16 step inside the 128-byte swizzle atom
           // router: a fresh sum per chain; experts: accumulate over the tile
           const bool accumulate = MODE == kRouter ? (!chain_start || kk != 0) : (((kb - kb0) | kk) != 0);
-          if (PAIR) {
+          if (PAIR)
             mma_bf16_ss_pair(d_tmem, adesc + static_cast<uint64_t>(2 * kk),
                              bdesc + static_cast<uint64_t>(2 * kk), idesc, accumulate ? 1u : 0u);
-            if (NSUB == 2 && !SPLIT && n1 > 0)   // the same A tile against the next MMA_N columns
-              mma_bf16_ss_pair(d_tmem + MMA_N, adesc + static_cast<uint64_t>(2 * kk),
-                               bdesc1 + static_cast<uint64_t>(2 * kk), idesc1, accumulate ? 1u : 0u);
-          } else {
+          else
             mma_bf16_ss(d_tmem, adesc + static_cast<uint64_t>(2 * kk),
                         bdesc + static_cast<uint64_t>(2 * kk), idesc, accumulate ? 1u : 0u);
-          }
         }
-        if (SPLIT && n1 > 0) {
-          // the second half: now if it is free, else deferred (the stage stays held)
-          if (hi_free) {
-            issue_hi(stage, kb == kb0);
-          } else {
-            def_stage[n_def] = stage;
-            def_first[n_def] = kb == kb0;
-            ++n_def;
-            hi_free = mbar_try_wait(&tempty[1], hi_parity);
-            if (!hi_free && n_def == stages) {   // every stage held: wait for the half
-              if (!mbar_wait(&tempty[1], hi_parity, s_abort, p.status)) { ok = false; break; }
-              hi_free = true;
-            }
-            if (hi_free) {
-              tc_fence_after();
-              for (int d = 0; d < n_def; ++d) issue_hi(def_stage[d], def_first[d]);
-              n_def = 0;
-            }
-          }
-        } else if (PAIR) {
-          mma_commit_pair(&empty[stage], 0x3);   // frees the stage in both CTAs
-        } else {
-          mma_commit(&empty[stage]);
-        }
+        if (PAIR) mma_commit_pair(&empty[stage], 0x3);   // frees the stage in both CTAs
+        else mma_commit(&empty[stage]);
         if (++stage == stages) { stage = 0; phase ^= 1u; }
         if (chain_end) {
           mma_commit(&tfull[acc]);
           ++it;
-        }
-      }
-      if (SPLIT && ok && n_def > 0) {   // a short tile still holding stages
-        if (!mbar_wait(&tempty[1], hi_parity, s_abort, p.status)) {
-          ok = false;
-        } else {
-          tc_fence_after();
-          for (int d = 0; d < n_def; ++d) issue_hi(def_stage[d], def_first[d]);
-          n_def = 0;
         }
       }
       if (!ok) break;
@@ -595,9 +510,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           w = p.gamma != nullptr ? p.gamma[static_cast<int64_t>(r) * p.S + gi.s] : p.uniform_w;
         }
       }
-      const uint32_t t_row = t_lane + static_cast<uint32_t>(acc * ACC_STRIDE);
+      const uint32_t t_row = t_lane + static_cast<uint32_t>(acc * BN);
       const int n_here = min(bn, p.N - n * bn);
-      bool lo_released = false;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         const int col0 = n * bn + c * 32;
@@ -605,13 +519,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t v[32];
         tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * 32), v);
         tmem_ld_wait();
-        if (SPLIT && c == MMA_N / 32 - 1) {
-          // the first half is read: the next tile's MMAs may start on it
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(mapa_shared(&tempty[0], 0));
-          lo_released = true;
-        }
         if (MODE == kGateUp) {
           if (!valid) continue;
           uint32_t packed[8];
@@ -663,14 +570,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        if (SPLIT) {   // both halves: the first unless a chunk loop already released it
-          if (!lo_released) mbar_arrive_cluster(mapa_shared(&tempty[0], 0));
-          mbar_arrive_cluster(mapa_shared(&tempty[1], 0));
-        } else if (PAIR) {
-          mbar_arrive_cluster(mapa_shared(&tempty[acc], 0));   // the issuer's barrier
-        } else {
-          mbar_arrive(&tempty[acc]);
-        }
+        if (PAIR) mbar_arrive_cluster(mapa_shared(&tempty[acc], 0));   // the issuer's barrier
+        else mbar_arrive(&tempty[acc]);
       }
       ++it;
     }
@@ -745,9 +646,9 @@ static bool encode_b(CUtensorMap* m, const void* base, int G, int N, int K, int 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE, bool PAIR, int NSUB = 1>
+template <int MODE, bool PAIR>
 static cudaError_t launch_mode(const GemmParams& p, int sms, cudaStream_t stream) {
-  const int smem = smem_bytes<MODE, PAIR, NSUB>(p.E, p.S);
+  const int smem = smem_bytes<MODE, PAIR>(p.E, p.S);
   // the attribute is per device; calls from several host threads may set it
   // concurrently (same value), devices past 64 set it on every launch
   static std::atomic<int> configured_smem[64];
@@ -755,7 +656,7 @@ static cudaError_t launch_mode(const GemmParams& p, int sms, cudaStream_t stream
   cudaGetDevice(&dev);
   const bool cached = dev >= 0 && dev < 64;
   if (!cached || configured_smem[dev].load(std::memory_order_relaxed) < smem) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, PAIR, NSUB>,
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, PAIR>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     if (cached) {
@@ -765,7 +666,7 @@ static cudaError_t launch_mode(const GemmParams& p, int sms, cudaStream_t stream
     }
   }
   if (!PAIR) {
-    grouped_gemm_kernel<MODE, PAIR, NSUB><<<sms, NUM_THREADS, smem, stream>>>(p);
+    grouped_gemm_kernel<MODE, PAIR><<<sms, NUM_THREADS, smem, stream>>>(p);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
@@ -780,7 +681,7 @@ static cudaError_t launch_mode(const GemmParams& p, int sms, cudaStream_t stream
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, PAIR, NSUB>, p);
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, PAIR>, p);
 }
 
 }  // namespace sm100
@@ -836,15 +737,7 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   // launches only the kind of CTA that has tiles)
   const bool pairs = L.T > BM && (L.E > 0 || group_paired(static_cast<int>((L.T + BM - 1) / BM)));
   const bool singles = L.E > 0 || !pairs;
-  // CTA pairs run 256 x 512 tiles when K is long: two N=256 MMAs share each A
-  // tile, so an SM moves 48 KB per K block for twice the MMA work of a
-  // 256 x 256 tile (32 KB).  The 512-column accumulator fills TMEM, so a
-  // tile's epilogue no longer overlaps the next tile's MMAs; with K >= 4096
-  // that wait is a small share of a tile.
-  const bool wide = L.H >= MOE_WIDE_GATE_UP_MIN_K;
-  cudaError_t e = !pairs ? cudaSuccess
-                         : wide ? launch_mode<kGateUp, true, 2>(g, num_sms, stream)
-                                : launch_mode<kGateUp, true>(g, num_sms, stream);
+  cudaError_t e = pairs ? launch_mode<kGateUp, true>(g, num_sms, stream) : cudaSuccess;
   if (e == cudaSuccess && singles) e = launch_mode<kGateUp, false>(g, num_sms, stream);
   if (e != cudaSuccess) return e;
 

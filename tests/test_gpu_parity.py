@@ -475,16 +475,15 @@ def test_expert_ffn_rows_in_slot_order(dtype):
 
 
 @pytest.mark.parametrize("shape,heavy", [
-    ((1100, 4096, 6, 2, 1, 448, "bf16"), True),    # gate_up N = 896: a 512-wide tile, then 384
-                                                   # (second MMA 128 wide); expert 0 takes every token
+    ((1100, 4096, 6, 2, 1, 448, "bf16"), True),    # gate_up N = 896; expert 0 takes every token
     ((1000, 4096, 3, 3, 1, 320, "bf16"), False),   # k = E: 1000 rows a group (8 m-tiles: pairs);
-                                                   # N = 640: the last tile has no second MMA
+                                                   # N = 640
 ], ids=["H4096-N896-heavy", "H4096-N640-keqE"])
-def test_wide_gate_up_tiles(shape, heavy):
-    """At H >= 4096 the gate_up CTA pairs run 256 x 512 tiles (two N=256 MMAs
-    a K step, one 512-column accumulator released half by half).  Ragged
-    last tiles, the oracle's bar on every row, and the row-gathering mode
-    bit for bit against the copied rows."""
+def test_long_k_ragged_gate_up_tiles(shape, heavy):
+    """A long K (H = 4096) on CTA pairs with ragged last n-tiles (N = 896:
+    a 128-column last tile; N = 640) and a group of 9 m-tiles: the oracle's
+    bar on every row, and the row-gathering mode bit for bit against the
+    copied rows."""
     w, inputs = small_case(*shape)
     if heavy:
         inputs["corr_bias"] = torch.zeros(w.E)
@@ -508,4 +507,4 @@ def test_wide_gate_up_tiles(shape, heavy):
     assert moe.read_device_status(ws) == 0
     assert torch.equal(yr[:R].cpu(), r["y_routed"][:R])
     assert torch.equal(ys.cpu(), r["y_shared"])
-    print(f"wide tiles {w.name}: {stats}")
+    print(f"long K {w.name}: {stats}")
