@@ -299,14 +299,26 @@ def gemm_roofline(w, ffn_ms: float, touched: int, peaks, peak_src: str):
     return roof
 
 
-def time_workload(moe, name: str, steps: int, warmup: int, dev, stream, peaks, peak_src):
+def device_inputs(moe, inputs, dev, down_f16: bool):
+    """Inputs on the device; with ``down_f16`` the down projections' weights
+    are replaced by their exact fp16 copies (made once, as at model load)."""
+    d = {k: v.to(dev).contiguous() for k, v in inputs.items()}
+    if down_f16:
+        for n in ("w_down", "ws_down"):
+            if n in d and d[n].numel():
+                d[n] = moe.prepare_down_weights(d[n])
+    return d
+
+
+def time_workload(moe, name: str, steps: int, warmup: int, dev, stream, peaks, peak_src,
+                  down_bf16: bool = False):
     """One of the task's other workloads, timed in this run: its op chain
     (route, permute, expert GEMMs, combine) for ``warmup`` + ``steps`` steps
     on device-resident seeded inputs, CUDA events around every op."""
     w = mw.by_name(name)
     inputs = mw.generate(w)
-    L = moe.Layer.from_workload(w)
-    d = {k: v.to(dev).contiguous() for k, v in inputs.items()}
+    L = moe.Layer.from_workload(w, down_f16=w.dtype == "bf16" and not down_bf16)
+    d = device_inputs(moe, inputs, dev, L.down_f16)
     del inputs
     ws = moe.new_workspace(L, device=dev)
     T, k, S, H, E = L.T, L.k, L.S, L.H, L.E
@@ -380,9 +392,11 @@ def gpu_arm(args, world, rank, local):
     if rank > 0:
         g = torch.Generator().manual_seed(10_000 + rank)
         inputs["x"] = torch.randn(w.T, w.H, generator=g).to(w.torch_dtype)
-    L = moe.Layer.from_workload(w)
+    # bf16 layers run their down projections in fp16 (the weights copied once
+    # to fp16 here, as at model load; outside every timed region)
+    L = moe.Layer.from_workload(w, down_f16=w.dtype == "bf16" and not args.down_bf16)
     dev = torch.device("cuda", local)
-    d = {k: v.to(dev).contiguous() for k, v in inputs.items()}
+    d = device_inputs(moe, inputs, dev, L.down_f16)
     x_host = inputs["x"].pin_memory()
     stream = torch.cuda.current_stream(dev)
     ws = moe.new_workspace(L, device=dev)
@@ -558,6 +572,8 @@ def gpu_arm(args, world, rank, local):
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02^2) weights, random init)",
             "config": {"workload": w.name, "T": T, "H": H, "E": E, "k": k, "S": S, "I": w.I,
                        "route_scale": w.route_scale, "parallelism": f"replicas x{world}",
+                       "down_projection": ("fp16: weights copied once from bf16 (exact), activated "
+                                           "rows rounded to fp16" if L.down_f16 else w.dtype),
                        "l2": "inputs larger than L2 (expert weights %.1f GB)" % (mw.weight_bytes(w) / 1e9)},
             "tflops": world * fl["total"] / (ms_step / 1e3) / 1e12,
             "op_ms": {"route": op_ms[0], "permute": op_ms[1], "expert_ffn": op_ms[2], "combine": op_ms[3]},
@@ -596,7 +612,8 @@ def gpu_arm(args, world, rank, local):
             del d, xp, yr, ys, ws
             torch.cuda.empty_cache()
             line["per_config"] = {n: time_workload(moe, n, args.steps, args.warmup, dev, stream,
-                                                   peaks, peak_src) for n in PER_CONFIG}
+                                                   peaks, peak_src, args.down_bf16)
+                                  for n in PER_CONFIG}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, inputs)
         print(json.dumps(line), flush=True)
@@ -655,9 +672,9 @@ def dense_gpu_arm(args, world, rank, local):
     if rank > 0:
         g = torch.Generator().manual_seed(10_000 + rank)
         inputs["x"] = torch.randn(w.T, w.H, generator=g).to(w.torch_dtype)
-    L = moe.DenseLayer.from_workload(w)
+    L = moe.DenseLayer.from_workload(w, down_f16=w.dtype == "bf16" and not args.down_bf16)
     dev = torch.device("cuda", local)
-    d = {k: v.to(dev).contiguous() for k, v in inputs.items()}
+    d = device_inputs(moe, inputs, dev, L.down_f16)
     stream = torch.cuda.current_stream(dev)
     ws = moe.new_dense_workspace(L, device=dev)
     out = torch.empty(w.T, w.H, dtype=w.torch_dtype, device=dev)
@@ -753,6 +770,7 @@ def dense_gpu_arm(args, world, rank, local):
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02^2) weights, random init)",
             "config": {"workload": w.name, "T": w.T, "H": w.H, "I": w.I,
                        "global_scale": w.global_scale, "parallelism": f"replicas x{world}",
+                       "down_projection": "fp16 (weights copied once from bf16)" if L.down_f16 else w.dtype,
                        "l2": "inputs larger than L2 (weights %.2f GB)" % (3 * w.H * w.I * el / 1e9)},
             "tflops": world * flops / s_step / 1e12,
             "roofline": {"kernel": "dense gate_up + down GEMM launches of moe_dense_mlp (whole call timed)",
@@ -803,6 +821,8 @@ def main():
                     help="replay each step's op chain as one captured CUDA graph")
     ap.add_argument("--gather-rows", action="store_true",
                     help="no permuted copy of x: the gate_up GEMM gathers the routed rows")
+    ap.add_argument("--down-bf16", action="store_true",
+                    help="bf16 down projections (bf16 activated rows) instead of fp16")
     args = ap.parse_args()
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         # N ranks requested without an outer launcher: start them here, one

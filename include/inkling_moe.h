@@ -34,9 +34,10 @@
  *       w_gate_up  [E, 2I, H]       row 2j = gate_j, row 2j+1 = up_j
  *       w_down     [E, H, I]
  *       ws_gate_up [S, 2I, H], ws_down [S, H, I]   (shared experts)
- *     x, the expert weights, x_perm and out share `dtype`; the expert output
- *     rows y_routed / y_shared are fp32 in every dtype (they are summed in
- *     fp32 and rounded once, in moe_combine).
+ *     x, the expert weights, x_perm and out share `dtype` (MOE_BF16_F16DOWN:
+ *     bf16, with w_down and ws_down fp16); the expert output rows
+ *     y_routed / y_shared are fp32 in every dtype (they are summed in fp32
+ *     and rounded once, in moe_combine).
  *   - Sizes: T = num_tokens, H = hidden, E = n_routed, k = top_k,
  *     S = n_shared, I = intermediate.  Limits: 1 <= k <= min(E, 16),
  *     E <= 1024, S <= 8, H % 64 == 0, I % 64 == 0, T <= 2^26,
@@ -69,7 +70,26 @@ typedef enum {
   MOE_ERR_TIMEOUT = 6        /* a kernel's bounded pipeline wait expired */
 } moe_status_t;
 
-typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+/*
+ * Layer dtypes.
+ *   MOE_F32           everything fp32; the expert GEMMs run in fp32 on the
+ *                     CUDA cores.
+ *   MOE_BF16          x, out and every expert weight bf16; the activated
+ *                     rows h are rounded to bf16 before the down projection.
+ *   MOE_BF16_F16DOWN  x, out, the router input and the gate_up weights bf16,
+ *                     as MOE_BF16; the down projections' weights (w_down,
+ *                     ws_down) fp16, and the activated rows h rounded to
+ *                     fp16, 8 times finer than bf16.  The fp16 weights are
+ *                     the checkpoint's bf16 values copied once with
+ *                     moe_convert_bf16_to_f16 (exact for |w| in [2^-14, 65504]
+ *                     and zero).  With bf16 h the rounding of h adds up to
+ *                     about 1% of the output's RMS to the error of the final
+ *                     bf16 rounding (1.7% of RMS when outputs reach 6 x RMS);
+ *                     with fp16 h it adds about 0.1%.  An h value at or beyond
+ *                     65520 in magnitude (an fp16 infinity) is recorded in the
+ *                     workspace status word (MOE_ERR_DEVICE_CHECK).
+ */
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_BF16_F16DOWN = 2 } moe_dtype_t;
 
 /* Layer description (the MoE fields of InklingTextConfig, with T added). */
 typedef struct {
@@ -168,7 +188,8 @@ moe_status_t moe_permute_noalloc(const moe_layer_desc_t* desc, const int32_t* to
  *   G = x_perm[r] @ w_gate_up[e]^T                       (fp32 accumulation)
  * and for shared expert s and token t (weight shared_gamma[t*S+s]) the same
  * with x[t] and ws_*[s] into y_shared[s*T + t].  The activated rows are
- * rounded to dtype before the down projection; y rows are written in fp32.
+ * rounded to dtype (MOE_BF16_F16DOWN: fp16) before the down projection; y
+ * rows are written in fp32.
  * x_perm may be NULL: the gate_up GEMM then reads row r straight from
  * x[perm_slot[r] / k] (bf16: TMA gathers of 4 rows into the tile), with the
  * same results bit for bit and without the [T*k, H] copy (memory saved:
@@ -317,7 +338,7 @@ typedef struct {
   int64_t num_tokens;    /* T */
   int32_t hidden;        /* H: hidden_size */
   int32_t intermediate;  /* I */
-  moe_dtype_t dtype;     /* x, weights, out */
+  moe_dtype_t dtype;     /* x, weights, out (MOE_BF16_F16DOWN: w_down fp16) */
   float global_scale;    /* finite */
 } moe_dense_desc_t;
 
@@ -349,6 +370,20 @@ moe_status_t moe_dense_mlp_prenorm(const moe_dense_desc_t* desc, const void* x,
 
 /* Number of kernels moe_dense_mlp_prenorm launches (moe_dense_mlp's + 1). */
 int32_t moe_dense_prenorm_kernel_count(const moe_dense_desc_t* desc);
+
+/* ------------------------------------------------------------------------
+ * moe_convert_bf16_to_f16 — the one-time copy of the down projections'
+ * weights for MOE_BF16_F16DOWN layers (no counterpart on the pages: a
+ * load-time preparation of the checkpoint's bf16 w_down / ws_down).
+ *   n      elements, a multiple of 8 (n = 0 does nothing)
+ *   src    bf16 [n], dst fp16 [n] (device, 16-byte aligned, not overlapping)
+ *   inexact  optional device int32 (NULL: none): increased by the number of
+ *          elements whose fp16 value differs from the bf16 one (magnitude
+ *          below 2^-24 granularity, above 65504, or NaN); 0 means an exact copy.
+ * Asynchronous on `stream`.
+ * ---------------------------------------------------------------------- */
+moe_status_t moe_convert_bf16_to_f16(int64_t n, const void* src, void* dst, int32_t* inexact,
+                                     void* stream);
 
 const char* moe_status_string(moe_status_t status);
 int32_t moe_version(void);

@@ -28,7 +28,7 @@ if not os.path.exists(_LIB_PATH):
 LIB = ctypes.CDLL(_LIB_PATH)
 LIB_PATH = _LIB_PATH
 
-MOE_F32, MOE_BF16 = 0, 1
+MOE_F32, MOE_BF16, MOE_BF16_F16DOWN = 0, 1, 2
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_CHECK", 6: "MOE_ERR_TIMEOUT"}
 
@@ -75,6 +75,7 @@ LIB.moe_shared_ffn.argtypes = [_DESC, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _
 LIB.moe_shared_ffn_kernel_count.restype = ctypes.c_int32
 LIB.moe_shared_ffn_kernel_count.argtypes = [_DESC]
 LIB.moe_ep_dispatch_prep.argtypes = [_DESC, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+LIB.moe_convert_bf16_to_f16.argtypes = [ctypes.c_int64, _P, _P, _P, _P]
 LIB.moe_forward.argtypes = [_DESC] + [_P] * 13 + [ctypes.c_size_t, _P]
 LIB.moe_selftest_wait_timeout.argtypes = [_P, ctypes.c_size_t, ctypes.c_uint32, _P]
 _DDESC = ctypes.POINTER(DenseDesc)
@@ -95,7 +96,7 @@ for _f in ("moe_workspace_size", "moe_workspace_init", "moe_read_device_status",
            "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_selftest_wait_timeout", "moe_dense_workspace_size", "moe_dense_mlp",
            "moe_rmsnorm", "moe_forward_prenorm", "moe_dense_mlp_prenorm", "moe_shared_ffn",
-           "moe_ep_dispatch_prep"):
+           "moe_ep_dispatch_prep", "moe_convert_bf16_to_f16"):
     getattr(LIB, _f).restype = ctypes.c_int
 
 
@@ -111,17 +112,23 @@ class Layer:
     dtype: torch.dtype = torch.bfloat16
     route_scale: float = 1.0
     global_scale: float = 1.0
+    # bf16 layers only: the down projections' weights are fp16 copies and the
+    # activated rows are rounded to fp16 (MOE_BF16_F16DOWN)
+    down_f16: bool = False
 
     def desc(self) -> LayerDesc:
-        code = {torch.float32: MOE_F32, torch.bfloat16: MOE_BF16}.get(self.dtype)
-        if code is None:
-            raise ValueError(f"unsupported dtype {self.dtype}")
-        return LayerDesc(self.T, self.H, self.E, self.k, self.S, self.I, code,
-                         self.route_scale, self.global_scale)
+        return LayerDesc(self.T, self.H, self.E, self.k, self.S, self.I,
+                         _layer_code(self.dtype, self.down_f16), self.route_scale, self.global_scale)
+
+    @property
+    def down_dtype(self) -> torch.dtype:
+        """dtype of w_down / ws_down."""
+        return torch.float16 if self.down_f16 else self.dtype
 
     @staticmethod
-    def from_workload(w) -> "Layer":
-        return Layer(w.T, w.H, w.E, w.k, w.S, w.I, w.torch_dtype, w.route_scale, w.global_scale)
+    def from_workload(w, down_f16: bool = False) -> "Layer":
+        return Layer(w.T, w.H, w.E, w.k, w.S, w.I, w.torch_dtype, w.route_scale, w.global_scale,
+                     down_f16)
 
 
 @dataclass(frozen=True)
@@ -132,16 +139,27 @@ class DenseLayer:
     I: int
     dtype: torch.dtype = torch.bfloat16
     global_scale: float = 1.0
+    down_f16: bool = False          # bf16 only: w_down fp16, activated rows fp16
 
     def desc(self) -> DenseDesc:
-        code = {torch.float32: MOE_F32, torch.bfloat16: MOE_BF16}.get(self.dtype)
-        if code is None:
-            raise ValueError(f"unsupported dtype {self.dtype}")
-        return DenseDesc(self.T, self.H, self.I, code, self.global_scale)
+        return DenseDesc(self.T, self.H, self.I, _layer_code(self.dtype, self.down_f16),
+                         self.global_scale)
+
+    @property
+    def down_dtype(self) -> torch.dtype:
+        return torch.float16 if self.down_f16 else self.dtype
 
     @staticmethod
-    def from_workload(w) -> "DenseLayer":
-        return DenseLayer(w.T, w.H, w.I, w.torch_dtype, w.global_scale)
+    def from_workload(w, down_f16: bool = False) -> "DenseLayer":
+        return DenseLayer(w.T, w.H, w.I, w.torch_dtype, w.global_scale, down_f16)
+
+
+def _layer_code(dtype: torch.dtype, down_f16: bool) -> int:
+    if dtype == torch.float32 and not down_f16:
+        return MOE_F32
+    if dtype == torch.bfloat16:
+        return MOE_BF16_F16DOWN if down_f16 else MOE_BF16
+    raise ValueError(f"unsupported layer dtype {dtype} (down_f16={down_f16})")
 
 
 def _check(status: int, where: str) -> None:
@@ -258,9 +276,9 @@ def moe_expert_ffn(layer: Layer, x, x_perm, expert_offsets, perm_slot, topk_w, s
     if L.S > 0 and (shared_gamma is None or shared_gamma.numel() != L.T * L.S):
         raise ValueError("shared_gamma must hold T*S entries")
     _expect(w_gate_up, "w_gate_up", (L.E, 2 * L.I, L.H), L.dtype)
-    _expect(w_down, "w_down", (L.E, L.H, L.I), L.dtype)
+    _expect(w_down, "w_down", (L.E, L.H, L.I), L.down_dtype)
     _expect(ws_gate_up, "ws_gate_up", (L.S, 2 * L.I, L.H), L.dtype, allow_none=L.S == 0)
-    _expect(ws_down, "ws_down", (L.S, L.H, L.I), L.dtype, allow_none=L.S == 0)
+    _expect(ws_down, "ws_down", (L.S, L.H, L.I), L.down_dtype, allow_none=L.S == 0)
     _expect(y_routed, "y_routed", (L.T * L.k, L.H), torch.float32)
     _expect(y_shared, "y_shared", (L.S * L.T, L.H), torch.float32, allow_none=L.S == 0)
     _check(LIB.moe_expert_ffn(ctypes.byref(L.desc()), _ptr(x), _ptr(x_perm), _ptr(expert_offsets),
@@ -277,7 +295,7 @@ def moe_shared_ffn(layer: Layer, x, shared_gamma, ws_gate_up, ws_down, y_shared,
     _expect(x, "x", (L.T, L.H), L.dtype)
     _expect(shared_gamma, "shared_gamma", (L.T, L.S), torch.float32)
     _expect(ws_gate_up, "ws_gate_up", (L.S, 2 * L.I, L.H), L.dtype)
-    _expect(ws_down, "ws_down", (L.S, L.H, L.I), L.dtype)
+    _expect(ws_down, "ws_down", (L.S, L.H, L.I), L.down_dtype)
     _expect(y_shared, "y_shared", (L.S * L.T, L.H), torch.float32)
     _check(LIB.moe_shared_ffn(ctypes.byref(L.desc()), _ptr(x), _ptr(shared_gamma),
                               _ptr(ws_gate_up), _ptr(ws_down), _ptr(y_shared), ws.data_ptr(),
@@ -322,9 +340,9 @@ def moe_forward(layer: Layer, x, w_router, corr_bias, w_gate_up, w_down, ws_gate
     _expect(w_router, "w_router", (L.E + L.S, L.H), torch.float32)
     _expect(corr_bias, "corr_bias", (L.E,), torch.float32)
     _expect(w_gate_up, "w_gate_up", (L.E, 2 * L.I, L.H), L.dtype)
-    _expect(w_down, "w_down", (L.E, L.H, L.I), L.dtype)
+    _expect(w_down, "w_down", (L.E, L.H, L.I), L.down_dtype)
     _expect(ws_gate_up, "ws_gate_up", (L.S, 2 * L.I, L.H), L.dtype, allow_none=L.S == 0)
-    _expect(ws_down, "ws_down", (L.S, L.H, L.I), L.dtype, allow_none=L.S == 0)
+    _expect(ws_down, "ws_down", (L.S, L.H, L.I), L.down_dtype, allow_none=L.S == 0)
     _expect(out, "out", (L.T, L.H), L.dtype)
     _expect(padding_mask, "padding_mask", (L.T,), torch.uint8, allow_none=True)
     _expect(topk_w, "topk_w", (L.T, L.k), torch.float32, allow_none=True)
@@ -365,9 +383,9 @@ def moe_forward_prenorm(layer: Layer, x, norm_weight, norm_eps, w_router, corr_b
     _expect(w_router, "w_router", (L.E + L.S, L.H), torch.float32)
     _expect(corr_bias, "corr_bias", (L.E,), torch.float32)
     _expect(w_gate_up, "w_gate_up", (L.E, 2 * L.I, L.H), L.dtype)
-    _expect(w_down, "w_down", (L.E, L.H, L.I), L.dtype)
+    _expect(w_down, "w_down", (L.E, L.H, L.I), L.down_dtype)
     _expect(ws_gate_up, "ws_gate_up", (L.S, 2 * L.I, L.H), L.dtype, allow_none=L.S == 0)
-    _expect(ws_down, "ws_down", (L.S, L.H, L.I), L.dtype, allow_none=L.S == 0)
+    _expect(ws_down, "ws_down", (L.S, L.H, L.I), L.down_dtype, allow_none=L.S == 0)
     _expect(out, "out", (L.T, L.H), L.dtype)
     _expect(padding_mask, "padding_mask", (L.T,), torch.uint8, allow_none=True)
     _expect(topk_w, "topk_w", (L.T, L.k), torch.float32, allow_none=True)
@@ -386,7 +404,7 @@ def moe_dense_mlp_prenorm(layer: "DenseLayer", x, norm_weight, norm_eps, w_gate_
     _expect(norm_weight, "norm_weight", (L.H,), L.dtype)
     _expect(x, "x", (L.T, L.H), L.dtype)
     _expect(w_gate_up, "w_gate_up", (2 * L.I, L.H), L.dtype)
-    _expect(w_down, "w_down", (L.H, L.I), L.dtype)
+    _expect(w_down, "w_down", (L.H, L.I), L.down_dtype)
     _expect(out, "out", (L.T, L.H), L.dtype)
     _check(LIB.moe_dense_mlp_prenorm(ctypes.byref(L.desc()), _ptr(x), _ptr(norm_weight), norm_eps,
                                      _ptr(w_gate_up), _ptr(w_down), _ptr(out), ws.data_ptr(),
@@ -430,7 +448,7 @@ def moe_dense_mlp(layer: DenseLayer, x, w_gate_up, w_down, out, ws, stream=None)
     L = layer
     _expect(x, "x", (L.T, L.H), L.dtype)
     _expect(w_gate_up, "w_gate_up", (2 * L.I, L.H), L.dtype)
-    _expect(w_down, "w_down", (L.H, L.I), L.dtype)
+    _expect(w_down, "w_down", (L.H, L.I), L.down_dtype)
     _expect(out, "out", (L.T, L.H), L.dtype)
     _check(LIB.moe_dense_mlp(ctypes.byref(L.desc()), _ptr(x), _ptr(w_gate_up), _ptr(w_down),
                              _ptr(out), ws.data_ptr(), ws.numel(), _stream(stream)),
@@ -439,6 +457,33 @@ def moe_dense_mlp(layer: DenseLayer, x, w_gate_up, w_down, out, ws, stream=None)
 
 def dense_kernel_count(layer: DenseLayer) -> int:
     return int(LIB.moe_dense_kernel_count(ctypes.byref(layer.desc())))
+
+
+def convert_bf16_to_f16(src: torch.Tensor, out: Optional[torch.Tensor] = None,
+                        inexact: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """``moe_convert_bf16_to_f16``: the fp16 copy of bf16 down-projection
+    weights (for layers with ``down_f16``), asynchronous; ``inexact`` (an
+    int32 CUDA tensor of one element) counts the elements not copied exactly."""
+    if src.dtype != torch.bfloat16 or not src.is_contiguous() or not src.is_cuda:
+        raise ValueError("src must be a contiguous bf16 CUDA tensor")
+    out = torch.empty(src.shape, dtype=torch.float16, device=src.device) if out is None else out
+    _expect(out, "out", tuple(src.shape), torch.float16)
+    if inexact is not None:
+        _expect(inexact, "inexact", (1,), torch.int32)
+    _check(LIB.moe_convert_bf16_to_f16(src.numel(), _ptr(src), _ptr(out), _ptr(inexact),
+                                       _stream(stream)), "moe_convert_bf16_to_f16")
+    return out
+
+
+def prepare_down_weights(w_down: torch.Tensor, stream=None) -> torch.Tensor:
+    """The fp16 copy of one bf16 down-projection weight tensor, checked to be
+    exact (raises ValueError otherwise; synchronises ``stream``)."""
+    count = torch.zeros(1, dtype=torch.int32, device=w_down.device)
+    out = convert_bf16_to_f16(w_down.contiguous(), inexact=count, stream=stream)
+    n = int(count.item())
+    if n:
+        raise ValueError(f"{n} down-projection weights are not exactly representable in fp16")
+    return out
 
 
 class InklingMoE:
@@ -456,6 +501,8 @@ class InklingMoE:
         self.H = self.w["w_router"].shape[1]
         self.I = self.w["w_down"].shape[2]
         self.dtype = self.w["w_gate_up"].dtype
+        # fp16 down weights (from prepare_down_weights): fp16 down projections
+        self.down_f16 = self.w["w_down"].dtype == torch.float16
         self.route_scale, self.global_scale = route_scale, global_scale
         self.device = device
         self._ws = None
@@ -463,7 +510,7 @@ class InklingMoE:
 
     def layer(self, T: int) -> Layer:
         return Layer(T, self.H, self.E, self.k, self.S, self.I, self.dtype, self.route_scale,
-                     self.global_scale)
+                     self.global_scale, self.down_f16)
 
     def __call__(self, x: torch.Tensor, padding_mask: Optional[torch.Tensor] = None,
                  stream=None) -> torch.Tensor:
@@ -505,13 +552,14 @@ class InklingDenseMLP:
         self.H = self.w_gate_up.shape[1]
         self.I = self.w_down.shape[1]
         self.dtype = self.w_gate_up.dtype
+        self.down_f16 = self.w_down.dtype == torch.float16
         self.global_scale = global_scale
         self.device = device
         self._ws = None
         self._ws_T = -1
 
     def layer(self, T: int) -> DenseLayer:
-        return DenseLayer(T, self.H, self.I, self.dtype, self.global_scale)
+        return DenseLayer(T, self.H, self.I, self.dtype, self.global_scale, self.down_f16)
 
     def __call__(self, x: torch.Tensor, stream=None) -> torch.Tensor:
         lead = x.shape[:-1]

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -16,6 +17,7 @@ enum DeviceCode : int32_t {
   DEV_OK = 0,
   DEV_BAD_EXPERT_ID = 0x101,   // topk_idx outside [0, E)
   DEV_BAD_ROW = 0x102,         // inv_perm / perm_slot outside its range
+  DEV_H_OVERFLOW = 0x103,      // an activated row value beyond the fp16 range (fp16 down projections)
   DEV_WAIT_TIMEOUT = 0x201,    // a pipeline wait ran past its time limit
 };
 
@@ -42,6 +44,14 @@ __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162flo
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Two fp32 values rounded to nearest fp16; `overflow` is set when either
+// rounds to an infinity (|v| at or beyond 65520) or is not finite.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi, bool& overflow) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  if (__hisinf(h.x) || __hisinf(h.y) || __hisnan(h.x) || __hisnan(h.y)) overflow = true;
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 __host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }

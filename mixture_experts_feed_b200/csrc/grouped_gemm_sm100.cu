@@ -120,6 +120,7 @@ struct alignas(64) GemmParams {
   int bn;                     // single-CTA expert launches: n-tile width (32..256, multiple of 32)
   int gather_k;               // kGateUp: > 0 = routed A rows are gathered from x (tmA[0] over
                               // [T, H], box one row high): row r reads x[perm_slot[r] / gather_k]
+  int f16;                    // kGateUp: h written in fp16; kDown: A (h) and B (weights) fp16
   int64_t split_stride;       // kRouter: elements between partial outputs
 };
 
@@ -369,7 +370,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int n = nv / ksplit, ks = nv - n * ksplit;
       // a narrow or ragged last n-tile runs a narrower MMA (N multiple of 32)
       const int n_here = min(bn, p.N - n * bn);
-      const uint32_t idesc = n_here >= BN ? TL::IDESC : idesc_bf16_f32(TL::TILE_M, (n_here + 31) & ~31);
+      uint32_t idesc = n_here >= BN ? TL::IDESC : idesc_bf16_f32(TL::TILE_M, (n_here + 31) & ~31);
+      if (MODE == kDown && p.f16) idesc = idesc_as_f16(idesc);   // fp16 h and fp16 weights
       if (MODE != kRouter) {
         const int acc = it % NACC;
         if (!mbar_wait(&tempty[acc], ((it / NACC) & 1) ^ 1u, s_abort, p.status)) { ok = false; break; }
@@ -432,6 +434,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     int it = 0;
     bool ok = true;
+    bool h_overflow = false;   // an activated value beyond the fp16 range
     for (int tile = unit; tile < total_tiles && ok; tile += units) {
       int g, m, nv;
       decode_tile(tile, s_tile, G, s_off, p.E, p.T, SET, BM, g, m, nv);
@@ -530,9 +533,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const float u1 = __uint_as_float(v[4 * i + 3]);
             const float h0 = w * (g0 / (1.0f + __expf(-g0))) * u0;
             const float h1 = w * (g1 / (1.0f + __expf(-g1))) * u1;
-            packed[i] = pack_bf16x2(h0, h1);
+            // fp16 down projections: h rounded to fp16 (8x finer than bf16)
+            packed[i] = p.f16 ? pack_f16x2(h0, h1, h_overflow) : pack_bf16x2(h0, h1);
           }
-          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out[gi.src]);
+          uint16_t* out = static_cast<uint16_t*>(p.out[gi.src]);   // bf16 or fp16 bits
           uint4* dst = reinterpret_cast<uint4*>(out + out_row * p.ld_out + col0 / 2);
           dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
           dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
@@ -575,6 +579,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       ++it;
     }
+    if (MODE == kGateUp && __any_sync(0xffffffffu, h_overflow) && lane == 0)
+      record_status(p.status, DEV_H_OVERFLOW);
     // the warp's TMA stores complete before the block (and its shared memory) goes
     if (MODE == kDown && lane == 0) bulk_wait_group0();
   }
@@ -605,14 +611,16 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // 2-D bf16 map over [rows, K] (K contiguous), box [box_rows, BK], 128B
 // swizzle: BM rows for tile loads, one row for tile::gather4.
-static bool encode_a(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows = BM) {
+static bool encode_a(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows = BM,
+                     bool f16 = false) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
   cuuint32_t box[2] = {BK, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+  return enc(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+             const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -631,8 +639,9 @@ static bool encode_y(CUtensorMap* m, void* base, int64_t rows, int H) {
              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D bf16 map over [G][N][K] (K contiguous), box [1][bn][BK], 128B swizzle.
-static bool encode_b(CUtensorMap* m, const void* base, int G, int N, int K, int bn) {
+// 3-D bf16 (or fp16) map over [G][N][K] (K contiguous), box [1][bn][BK], 128B swizzle.
+static bool encode_b(CUtensorMap* m, const void* base, int G, int N, int K, int bn,
+                     bool f16 = false) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N),
@@ -641,7 +650,8 @@ static bool encode_b(CUtensorMap* m, const void* base, int G, int N, int K, int 
                            static_cast<cuuint64_t>(K) * 2 * static_cast<cuuint64_t>(N)};
   cuuint32_t box[3] = {BK, static_cast<cuuint32_t>(bn), 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+  return enc(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+             const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -731,6 +741,7 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   g.ksplit = 1;
   g.bn = tiling.gate_up_bn;
   g.gather_k = gather ? L.k : 0;
+  g.f16 = L.down_f16 ? 1 : 0;   // h in fp16 for fp16 down projections
   // paired groups on CTA pairs, the rest on single CTAs (grouping.cuh); with
   // T <= 128 every group has one m-tile and the pair launch is skipped
   // (E == 0, the dense layer: the host knows the one group's m-tiles and
@@ -743,10 +754,11 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
 
   // ---------------- down: h [rows, I] x [H, I]^T -> y [rows, H] (fp32)
   GemmParams d{};
-  ok = encode_a(&d.tmA[0], h, Rh, L.I);
-  if (ok && L.E > 0) ok = encode_b(&d.tmB[0], w_down, L.E, L.H, L.I, BROWS);
+  const bool f16 = L.down_f16;   // h and the down weights in fp16
+  ok = encode_a(&d.tmA[0], h, Rh, L.I, BM, f16);
+  if (ok && L.E > 0) ok = encode_b(&d.tmB[0], w_down, L.E, L.H, L.I, BROWS, f16);
   d.tmA[1] = d.tmA[0];
-  if (ok && L.S > 0) ok = encode_b(&d.tmB[1], ws_down, L.S, L.H, L.I, BROWS);
+  if (ok && L.S > 0) ok = encode_b(&d.tmB[1], ws_down, L.S, L.H, L.I, BROWS, f16);
   if (L.E == 0) d.tmB[0] = d.tmB[1];
   if (L.S == 0) d.tmB[1] = d.tmB[0];
   // output maps: routed rows [T*k, H]; shared rows [S*T, H], or one partial
@@ -768,6 +780,7 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   d.ksplit = tiling.down_ksplit;
   d.split_stride = L.T * static_cast<int64_t>(L.H);   // partial rows of the shared groups
   d.bn = 256;
+  d.f16 = f16 ? 1 : 0;
   e = pairs ? launch_mode<kDown, true>(d, num_sms, stream) : cudaSuccess;
   if (e == cudaSuccess && singles) e = launch_mode<kDown, false>(d, num_sms, stream);
   return e;

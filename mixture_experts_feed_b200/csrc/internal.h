@@ -11,8 +11,11 @@ namespace moe {
 struct Layer {
   int64_t T;
   int H, E, k, S, I;
-  int dtype;   // MOE_F32 / MOE_BF16
+  int dtype;   // activations: MOE_F32 / MOE_BF16
   float route_scale, global_scale;
+  // MOE_BF16_F16DOWN layers: the down projections' weights are fp16 and the
+  // activated rows h are rounded to fp16 (dtype is MOE_BF16)
+  bool down_f16 = false;
 };
 
 // moe_api.cu: SM count of the current device (cached per device), and the

@@ -79,7 +79,8 @@ moe_status_t check_desc(const moe_layer_desc_t* d, Layer* L) {
       d->n_shared < 0 || d->intermediate <= 0)
     return MOE_ERR_INVALID_ARG;
   if (d->top_k > d->n_routed) return MOE_ERR_INVALID_ARG;
-  if (d->dtype != MOE_F32 && d->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (d->dtype != MOE_F32 && d->dtype != MOE_BF16 && d->dtype != MOE_BF16_F16DOWN)
+    return MOE_ERR_INVALID_ARG;
   if (!isfinite(d->route_scale) || !isfinite(d->global_scale)) return MOE_ERR_INVALID_ARG;
   if (d->top_k > 16 || d->n_routed > 1024 || d->n_shared > 8) return MOE_ERR_UNSUPPORTED;
   if (d->hidden % 64 != 0 || d->intermediate % 64 != 0) return MOE_ERR_UNSUPPORTED;
@@ -92,7 +93,8 @@ moe_status_t check_desc(const moe_layer_desc_t* d, Layer* L) {
   L->k = d->top_k;
   L->S = d->n_shared;
   L->I = d->intermediate;
-  L->dtype = d->dtype;
+  L->dtype = d->dtype == MOE_F32 ? MOE_F32 : MOE_BF16;
+  L->down_f16 = d->dtype == MOE_BF16_F16DOWN;
   L->route_scale = d->route_scale;
   L->global_scale = d->global_scale;
   return MOE_OK;
@@ -278,7 +280,8 @@ FfnTiling dense_tiling(const Layer& L) {
 moe_status_t check_dense(const moe_dense_desc_t* d, Layer* L) {
   if (d == nullptr) return MOE_ERR_INVALID_ARG;
   if (d->num_tokens < 0 || d->hidden <= 0 || d->intermediate <= 0) return MOE_ERR_INVALID_ARG;
-  if (d->dtype != MOE_F32 && d->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (d->dtype != MOE_F32 && d->dtype != MOE_BF16 && d->dtype != MOE_BF16_F16DOWN)
+    return MOE_ERR_INVALID_ARG;
   if (!isfinite(d->global_scale)) return MOE_ERR_INVALID_ARG;
   if (d->hidden % 64 != 0 || d->intermediate % 64 != 0) return MOE_ERR_UNSUPPORTED;
   if (d->num_tokens >= (int64_t{1} << 26)) return MOE_ERR_UNSUPPORTED;
@@ -288,7 +291,8 @@ moe_status_t check_dense(const moe_dense_desc_t* d, Layer* L) {
   L->k = 0;
   L->S = 1;
   L->I = d->intermediate;
-  L->dtype = d->dtype;
+  L->dtype = d->dtype == MOE_F32 ? MOE_F32 : MOE_BF16;
+  L->down_f16 = d->dtype == MOE_BF16_F16DOWN;
   L->route_scale = 1.0f;
   L->global_scale = d->global_scale;
   return MOE_OK;

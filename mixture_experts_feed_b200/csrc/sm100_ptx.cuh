@@ -314,5 +314,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// The same descriptor with A and B fp16 (format code 0 in bits 7-9 and
+// 10-12).  A and B always share one type.
+__host__ __device__ constexpr uint32_t idesc_as_f16(uint32_t idesc) {
+  return idesc & ~((7u << 7) | (7u << 10));
+}
+
 }  // namespace sm100
 }  // namespace moe

@@ -128,12 +128,13 @@ class ExpertParallelMoE:
         self.H = self.w["w_router"].shape[1]
         self.I = self.w["w_down"].shape[2]
         self.dtype = self.w["w_gate_up"].dtype
+        self.down_f16 = self.w["w_down"].dtype == torch.float16   # fp16 down projections
         self.route_scale, self.global_scale = route_scale, global_scale
         self.last_counts = None       # (rows sent per destination, rows received per source)
 
     def layer(self, T: int) -> Layer:
         return self.ops.Layer(T, self.H, self.E, self.k, self.S, self.I, self.dtype,
-                              self.route_scale, self.global_scale)
+                              self.route_scale, self.global_scale, self.down_f16)
 
     def __call__(self, x: torch.Tensor, padding_mask: Optional[torch.Tensor] = None) -> torch.Tensor:
         ops, dev, W, El, H = self.ops, self.device, self.W, self.El, self.H
@@ -191,7 +192,7 @@ class ExpertParallelMoE:
         self.comm.exchange(sends, recvs)
         # 5: the local experts over the received rows (already grouped, in slot order)
         Ll = self.ops.Layer(R_in, H, El, 1, 0, self.I, self.dtype, self.route_scale,
-                            self.global_scale)
+                            self.global_scale, self.down_f16)
         y_in = torch.empty(R_in, H, dtype=torch.float32, device=dev)
         if R_in > 0:
             off_loc = torch.tensor(loc_off, dtype=torch.int32).to(dev)

@@ -29,8 +29,22 @@ def out_tolerance(dtype: torch.dtype) -> float:
     return 2e-2 if dtype == torch.bfloat16 else 1e-4
 
 
-def to_device(inputs: Dict[str, torch.Tensor]) -> Dict[str, torch.Tensor]:
-    return {k: v.to("cuda", non_blocking=True).contiguous() for k, v in inputs.items()}
+def to_device(inputs: Dict[str, torch.Tensor], down_f16: bool = False) -> Dict[str, torch.Tensor]:
+    """Inputs on the GPU; ``down_f16``: the down projections' weights as their
+    exact fp16 copies (moe_convert_bf16_to_f16), for MOE_BF16_F16DOWN layers."""
+    d = {k: v.to("cuda", non_blocking=True).contiguous() for k, v in inputs.items()}
+    if down_f16:
+        for n in ("w_down", "ws_down"):
+            if n in d and d[n].numel():
+                d[n] = moe.prepare_down_weights(d[n])
+            elif n in d:
+                d[n] = d[n].to(torch.float16)
+    return d
+
+
+def down_f16_of(w) -> bool:
+    """The bf16 workloads run their down projections in fp16 (MOE_BF16_F16DOWN)."""
+    return w.dtype == "bf16"
 
 
 def run_chain(L: moe.Layer, d: Dict[str, torch.Tensor], padding_mask: Optional[torch.Tensor] = None,

@@ -23,9 +23,9 @@ except ImportError:   # collected on CPU-only machines too; the gpu marker desel
     moe = None
 
 
-def run_dense(w, inputs, d=None):
-    L = moe.DenseLayer.from_workload(w)
-    d = d or to_device(inputs)
+def run_dense(w, inputs, d=None, down_f16=False):
+    L = moe.DenseLayer.from_workload(w, down_f16=down_f16)
+    d = d or to_device(inputs, down_f16=down_f16)
     ws = moe.new_dense_workspace(L)
     out = torch.empty(w.T, w.H, dtype=w.torch_dtype, device="cuda")
     moe.moe_dense_mlp(L, d["x"], d["w_gate_up"], d["w_down"], out, ws)
@@ -57,12 +57,15 @@ def test_dense_small_shapes(shape):
     check_output(out, ref, w.torch_dtype, "dense out", strict=False)
 
 
+@pytest.mark.parametrize("down_f16", [False, True], ids=["down-bf16", "down-f16"])
 @pytest.mark.parametrize("name", list(mw.DENSE_WORKLOADS))
-def test_dense_workloads(name):
+def test_dense_workloads(name, down_f16):
     w = mw.dense_by_name(name)
+    if down_f16 and w.dtype != "bf16":
+        pytest.skip("fp16 down projections are a bf16-layer mode")
     inputs = mw.generate_dense(w)
-    d = to_device(inputs)
-    out = run_dense(w, inputs, d)
+    d = to_device(inputs, down_f16=down_f16)
+    out = run_dense(w, inputs, d, down_f16=down_f16)
     del d
     # every token (7.4 TFLOP in fp64 at the model's sizes: seconds on the host cores)
     ref = oracle.dense_mlp(inputs["x"], inputs["w_gate_up"], inputs["w_down"], w.global_scale)
@@ -70,7 +73,7 @@ def test_dense_workloads(name):
     # a bf16 ulp of the exact value on top (their outputs reach 5 x RMS, where
     # the final rounding alone costs 2^-8 x 5 = 2% of RMS)
     rel = check_output(out, ref, w.torch_dtype, f"{name} out", strict=w.H >= 2048)
-    print(f"{name}: all {w.T} tokens, max|err|/RMS = {rel:.4f}")
+    print(f"{name} ({'fp16' if down_f16 else 'bf16'} down): all {w.T} tokens, max|err|/RMS = {rel:.4f}")
 
 
 def test_dense_module_leading_dims_and_determinism():

@@ -52,28 +52,34 @@ def run_ranks(inputs, world, T_rank, E, k, S, route_scale, pm=None):
 
 
 CASES = [
-    # world, T a rank, H, E, k, S, I, skew
-    (2, 256, 256, 16, 4, 1, 192, False),
-    (4, 128, 256, 16, 2, 2, 128, False),
-    (4, 128, 128, 16, 2, 1, 64, True),    # every row to rank 0's experts: ranks 1-3 receive none
+    # world, T a rank, H, E, k, S, I, skew, fp16 down projections
+    (2, 256, 256, 16, 4, 1, 192, False, True),
+    (2, 256, 256, 16, 4, 1, 192, False, False),
+    (4, 128, 256, 16, 2, 2, 128, False, True),
+    (4, 128, 128, 16, 2, 1, 64, True, True),    # every row to rank 0's experts: ranks 1-3 receive none
 ]
 
 
 @pytest.mark.parametrize("case", CASES, ids=[f"W{c[0]}-T{c[1]}-H{c[2]}-E{c[3]}k{c[4]}S{c[5]}-I{c[6]}"
-                                             + ("-skew" if c[7] else "") for c in CASES])
+                                             + ("-skew" if c[7] else "") + ("-down-f16" if c[8] else "")
+                                             for c in CASES])
 def test_ep_virtual_ranks(case):
-    world, T_rank, H, E, k, S, I, skew = case
+    world, T_rank, H, E, k, S, I, skew, down_f16 = case
     w = mw.tiny(T=T_rank * world, H=H, E=E, k=k, S=S, I=I, dtype="bf16", route_scale=2.5, seed=23)
     inputs = mw.generate(w, threads=4)
     if skew:
         inputs["corr_bias"] = torch.zeros(E)
         inputs["corr_bias"][:E // world] = 3.0
     pm = (torch.arange(w.T) % 7 == 4).to(torch.uint8)
-    out_ep, counts = run_ranks(inputs, world, T_rank, E, k, S, w.route_scale, pm=pm)
+    rank_inputs = dict(inputs)
+    if down_f16:   # the ranks hold the exact fp16 copies of the down weights
+        rank_inputs["w_down"] = inputs["w_down"].to(torch.float16)
+        rank_inputs["ws_down"] = inputs["ws_down"].to(torch.float16)
+    out_ep, counts = run_ranks(rank_inputs, world, T_rank, E, k, S, w.route_scale, pm=pm)
     if skew:
         assert all(sum(counts[r][1]) == 0 for r in range(1, world))
-    L = __import__("mixture_experts_feed_b200").Layer.from_workload(w)
-    one = run_forward(L, to_device(inputs), padding_mask=pm)
+    L = __import__("mixture_experts_feed_b200").Layer.from_workload(w, down_f16=down_f16)
+    one = run_forward(L, to_device(inputs, down_f16=down_f16), padding_mask=pm)
     assert torch.equal(out_ep, one["out"]), "expert-parallel output differs from the one-GPU layer"
     ref = oracle.moe_forward_workload(inputs, w, padding_mask=pm,
                                       given_topk_idx=one["topk_idx"].to(torch.int64))

@@ -63,9 +63,9 @@ def test_rmsnorm_in_place_and_zero_row():
     assert torch.equal(want[5], torch.zeros(256, dtype=torch.bfloat16))
 
 
-def run_prenorm(w, inputs, nw):
-    L = moe.Layer.from_workload(w)
-    d = to_device(inputs)
+def run_prenorm(w, inputs, nw, down_f16=False):
+    L = moe.Layer.from_workload(w, down_f16=down_f16)
+    d = to_device(inputs, down_f16=down_f16)
     ws = moe.new_workspace(L)
     T, k, S, H = w.T, w.k, w.S, w.H
     out = torch.empty(T, H, dtype=w.torch_dtype, device="cuda")
@@ -110,7 +110,7 @@ def test_forward_prenorm_full_size():
     w = mw.by_name("bf16-T8192-H6144-E128k8S1-I2048")
     inputs = mw.generate(w)
     nw = mw.norm_weight(w.H, seed=w.seed)
-    r, _, _ = run_prenorm(w, inputs, nw)
+    r, _, _ = run_prenorm(w, inputs, nw, down_f16=True)
     xn = oracle.rmsnorm(inputs["x"], nw, EPS, out_dtype=w.torch_dtype)
     stats, _ = check_all(w, {**inputs, "x": xn}, r, strict=True)   # every token
     print(f"prenorm {w.name}: all {w.T} tokens, max|out - oracle| / RMS = {stats['rel_err']:.4f}; "

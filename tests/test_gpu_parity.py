@@ -13,7 +13,7 @@ import torch
 import moe_workloads as mw
 import oracle
 from moe_gpu_helpers import (check_output, check_permutation, check_routing, check_x_perm,
-                             out_tolerance, run_chain, run_forward, to_device)
+                             down_f16_of, out_tolerance, run_chain, run_forward, to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -57,11 +57,14 @@ def check_all(w, inputs, r, padding_mask=None, tokens=None, strict=False):
     return stats, ref
 
 
+@pytest.mark.parametrize("down_f16", [False, True], ids=["down-bf16", "down-f16"])
 @pytest.mark.parametrize("shape", SMALL, ids=[f"T{s[0]}-H{s[1]}-E{s[2]}k{s[3]}S{s[4]}-I{s[5]}-{s[6]}" for s in SMALL])
-def test_small_shapes_op_chain(shape):
+def test_small_shapes_op_chain(shape, down_f16):
+    if down_f16 and shape[6] != "bf16":
+        pytest.skip("fp16 down projections are a bf16-layer mode")
     w, inputs = small_case(*shape)
-    L = moe.Layer.from_workload(w)
-    d = to_device(inputs)
+    L = moe.Layer.from_workload(w, down_f16=down_f16)
+    d = to_device(inputs, down_f16=down_f16)
     r = run_chain(L, d)
     stats, ref = check_all(w, inputs, r)
     # y rows of the routed experts, one by one, against the oracle's per-choice outputs
@@ -82,11 +85,14 @@ def test_workload_full_size(w):
     on all T rows under the stated bound as is, and each routed expert output
     row y_routed against the oracle's row for that (token, choice)."""
     inputs = mw.generate(w, pin_memory=False)
-    L = moe.Layer.from_workload(w)
-    d = to_device(inputs)
+    # bf16 layers with fp16 down projections: the output bound holds on every
+    # element (with bf16 activated rows the Zipf layer's worst element over
+    # its 100 M reaches 2.2% of RMS, 1.7% of it the final bf16 rounding)
+    L = moe.Layer.from_workload(w, down_f16=down_f16_of(w))
+    d = to_device(inputs, down_f16=L.down_f16)
     r = run_chain(L, d)
     del d
-    f = run_forward(L, to_device(inputs))
+    f = run_forward(L, to_device(inputs, down_f16=L.down_f16))
     assert torch.equal(f["out"], r["out"])
     del f
     stats, ref = check_all(w, inputs, r, strict=True)   # the stated bound, as is
@@ -508,3 +514,42 @@ def test_long_k_ragged_gate_up_tiles(shape, heavy):
     assert torch.equal(yr[:R].cpu(), r["y_routed"][:R])
     assert torch.equal(ys.cpu(), r["y_shared"])
     print(f"long K {w.name}: {stats}")
+
+
+
+def test_down_weight_conversion_counts_inexact_values():
+    """moe_convert_bf16_to_f16 copies bf16 values exactly where fp16 holds
+    them and counts the rest (too small, too large, NaN), element for element
+    as the library's own float16 conversion decides."""
+    g = torch.Generator().manual_seed(9)
+    t = (torch.randn(4096, generator=g) * 0.02).to(torch.bfloat16)
+    t[:5] = torch.tensor([1e-9, 3e-7, 7e4, -1e6, float("nan")]).to(torch.bfloat16)
+    t[5:9] = torch.tensor([0.0, -0.0, 2.0 ** -14, 65504.0]).to(torch.bfloat16)
+    count = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = moe.convert_bf16_to_f16(t.cuda(), inexact=count)
+    torch.cuda.synchronize()
+    ref = t.to(torch.float16)
+    same = (ref.float() == t.float())
+    assert int(count.item()) == int((~same).sum())
+    assert torch.equal(out.cpu()[same], ref[same])
+    ok = moe.prepare_down_weights((torch.randn(64, 128, generator=g) * 0.02).to(torch.bfloat16).cuda())
+    assert ok.dtype == torch.float16
+    with pytest.raises(ValueError):
+        moe.prepare_down_weights(t.cuda())
+
+
+def test_fp16_activation_overflow_is_reported():
+    """With fp16 down projections an activated value beyond the fp16 range is
+    recorded in the status word (0x103), not passed on silently."""
+    w, inputs = small_case(64, 128, 8, 2, 1, 64)
+    inputs["w_gate_up"] = (inputs["w_gate_up"].float() * 3000.0).to(torch.bfloat16)
+    L = moe.Layer.from_workload(w, down_f16=True)
+    d = to_device(inputs, down_f16=True)
+    ws = moe.new_workspace(L)
+    out = torch.empty(w.T, w.H, dtype=L.dtype, device="cuda")
+    moe.moe_forward(L, d["x"], d["w_router"], d["corr_bias"], d["w_gate_up"], d["w_down"],
+                    d["ws_gate_up"], d["ws_down"], out, ws)
+    torch.cuda.synchronize()
+    with pytest.raises(moe.MoEError) as ei:
+        moe.read_device_status(ws)
+    assert ei.value.device_code == 0x103
