@@ -81,8 +81,9 @@ typedef enum {
  *                     ws_down) fp16, and the activated rows h rounded to
  *                     fp16, 8 times finer than bf16.  The fp16 weights are
  *                     the checkpoint's bf16 values copied once with
- *                     moe_convert_bf16_to_f16 (exact for |w| in [2^-14, 65504]
- *                     and zero).  With bf16 h the rounding of h adds up to
+ *                     moe_convert_bf16_to_f16 (exact for |w| in [2^-17, 65504]
+ *                     and zero; smaller values change by at most 2^-25).
+ *                     With bf16 h the rounding of h adds up to
  *                     about 1% of the output's RMS to the error of the final
  *                     bf16 rounding (1.7% of RMS when outputs reach 6 x RMS);
  *                     with fp16 h it adds about 0.1%.  An h value at or beyond
@@ -376,13 +377,16 @@ int32_t moe_dense_prenorm_kernel_count(const moe_dense_desc_t* desc);
  * weights for MOE_BF16_F16DOWN layers (no counterpart on the pages: a
  * load-time preparation of the checkpoint's bf16 w_down / ws_down).
  *   n      elements, a multiple of 8 (n = 0 does nothing)
- *   src    bf16 [n], dst fp16 [n] (device, 16-byte aligned, not overlapping)
- *   inexact  optional device int32 (NULL: none): increased by the number of
- *          elements whose fp16 value differs from the bf16 one (magnitude
- *          below 2^-24 granularity, above 65504, or NaN); 0 means an exact copy.
+ *   src    bf16 [n], dst fp16 [n] (device, 16-byte aligned, not overlapping):
+ *          each value rounded to nearest fp16, which is exact for magnitudes
+ *          in [2^-17, 65504] and zero; smaller magnitudes (fp16 subnormals)
+ *          change by at most 2^-25
+ *   nonfinite  optional device int32 (NULL: none): increased by the number of
+ *          elements with no finite fp16 value (magnitude beyond 65504, NaN);
+ *          0 means the copy is usable.
  * Asynchronous on `stream`.
  * ---------------------------------------------------------------------- */
-moe_status_t moe_convert_bf16_to_f16(int64_t n, const void* src, void* dst, int32_t* inexact,
+moe_status_t moe_convert_bf16_to_f16(int64_t n, const void* src, void* dst, int32_t* nonfinite,
                                      void* stream);
 
 const char* moe_status_string(moe_status_t status);

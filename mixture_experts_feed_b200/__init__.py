@@ -460,29 +460,32 @@ def dense_kernel_count(layer: DenseLayer) -> int:
 
 
 def convert_bf16_to_f16(src: torch.Tensor, out: Optional[torch.Tensor] = None,
-                        inexact: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                        nonfinite: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """``moe_convert_bf16_to_f16``: the fp16 copy of bf16 down-projection
-    weights (for layers with ``down_f16``), asynchronous; ``inexact`` (an
-    int32 CUDA tensor of one element) counts the elements not copied exactly."""
+    weights (for layers with ``down_f16``), asynchronous; ``nonfinite`` (an
+    int32 CUDA tensor of one element) counts the elements with no finite fp16
+    value."""
     if src.dtype != torch.bfloat16 or not src.is_contiguous() or not src.is_cuda:
         raise ValueError("src must be a contiguous bf16 CUDA tensor")
     out = torch.empty(src.shape, dtype=torch.float16, device=src.device) if out is None else out
     _expect(out, "out", tuple(src.shape), torch.float16)
-    if inexact is not None:
-        _expect(inexact, "inexact", (1,), torch.int32)
-    _check(LIB.moe_convert_bf16_to_f16(src.numel(), _ptr(src), _ptr(out), _ptr(inexact),
+    if nonfinite is not None:
+        _expect(nonfinite, "nonfinite", (1,), torch.int32)
+    _check(LIB.moe_convert_bf16_to_f16(src.numel(), _ptr(src), _ptr(out), _ptr(nonfinite),
                                        _stream(stream)), "moe_convert_bf16_to_f16")
     return out
 
 
 def prepare_down_weights(w_down: torch.Tensor, stream=None) -> torch.Tensor:
-    """The fp16 copy of one bf16 down-projection weight tensor, checked to be
-    exact (raises ValueError otherwise; synchronises ``stream``)."""
+    """The fp16 copy of one bf16 down-projection weight tensor (exact for
+    magnitudes from 2^-17 to 65504; smaller ones change by at most 2^-25);
+    raises ValueError when an element has no finite fp16 value (synchronises
+    ``stream``)."""
     count = torch.zeros(1, dtype=torch.int32, device=w_down.device)
-    out = convert_bf16_to_f16(w_down.contiguous(), inexact=count, stream=stream)
+    out = convert_bf16_to_f16(w_down.contiguous(), nonfinite=count, stream=stream)
     n = int(count.item())
     if n:
-        raise ValueError(f"{n} down-projection weights are not exactly representable in fp16")
+        raise ValueError(f"{n} down-projection weights have no finite fp16 value")
     return out
 
 

@@ -517,23 +517,28 @@ def test_long_k_ragged_gate_up_tiles(shape, heavy):
 
 
 
-def test_down_weight_conversion_counts_inexact_values():
-    """moe_convert_bf16_to_f16 copies bf16 values exactly where fp16 holds
-    them and counts the rest (too small, too large, NaN), element for element
-    as the library's own float16 conversion decides."""
+def test_down_weight_conversion():
+    """moe_convert_bf16_to_f16 rounds each bf16 value to the nearest fp16,
+    element for element as the library's own float16 conversion does (exact
+    from 2^-17 to 65504, within 2^-25 below), and counts the elements with no
+    finite fp16 value (beyond 65504, NaN)."""
     g = torch.Generator().manual_seed(9)
     t = (torch.randn(4096, generator=g) * 0.02).to(torch.bfloat16)
     t[:5] = torch.tensor([1e-9, 3e-7, 7e4, -1e6, float("nan")]).to(torch.bfloat16)
     t[5:9] = torch.tensor([0.0, -0.0, 2.0 ** -14, 65504.0]).to(torch.bfloat16)
     count = torch.zeros(1, dtype=torch.int32, device="cuda")
-    out = moe.convert_bf16_to_f16(t.cuda(), inexact=count)
+    out = moe.convert_bf16_to_f16(t.cuda(), nonfinite=count)
     torch.cuda.synchronize()
     ref = t.to(torch.float16)
-    same = (ref.float() == t.float())
-    assert int(count.item()) == int((~same).sum())
-    assert torch.equal(out.cpu()[same], ref[same])
-    ok = moe.prepare_down_weights((torch.randn(64, 128, generator=g) * 0.02).to(torch.bfloat16).cuda())
-    assert ok.dtype == torch.float16
+    assert int(count.item()) == 3                       # 7e4, -1e6 (beyond 65504) and the NaN
+    fin = torch.isfinite(ref)
+    assert torch.equal(out.cpu()[fin], ref[fin])
+    assert bool(torch.isnan(out.cpu()[4]))
+    big = t.float().abs() >= 2.0 ** -17
+    assert bool((out.cpu().float()[fin & big] == t.float()[fin & big]).all())     # exact there
+    assert float((out.cpu().float()[fin] - t.float()[fin]).abs().max()) <= 2.0 ** -25
+    w = (torch.randn(64, 128, generator=g) * 0.02).to(torch.bfloat16)
+    assert moe.prepare_down_weights(w.cuda()).dtype == torch.float16
     with pytest.raises(ValueError):
         moe.prepare_down_weights(t.cuda())
 
