@@ -5,7 +5,10 @@
 
 A step is one full forward pass of the layer (router, permutation, routed and
 shared expert GEMMs, recombination) over one batch of T tokens, through the
-library's C ABI, inputs resident in HBM.  The default workload is the layer
+library's one-call entry point ``moe_forward``, inputs resident in HBM.  The
+same steps are then run as the op chain (``moe_route``, ``moe_permute``,
+``moe_expert_ffn``, ``moe_combine``) with CUDA events between the ops, for the
+per-op breakdown and the expert GEMMs' roofline.  The default workload is the layer
 at the pages' hidden size: T=8192, H=6144, E=128, k=8, S=1, I=2048, bf16.
 
 N > 1 (launched by torch.distributed.run, or with ``--gpus N`` alone, which
@@ -351,18 +354,33 @@ def time_workload(moe, name: str, steps: int, warmup: int, dev, stream, peaks, p
         if ev is not None:
             ev[4].record(stream)
 
+    def fwd():
+        moe.moe_forward(L, d["x"], d["w_router"], d["corr_bias"], d["w_gate_up"], d["w_down"],
+                        wsgu, wsd, out, ws, stream=stream)
+
+    # the step through moe_forward (timed as a whole), then the op chain
+    # with events between the ops (breakdown and the expert GEMMs' time)
     for _ in range(warmup):
-        step()
+        fwd()
     torch.cuda.synchronize(dev)
     moe.read_device_status(ws, stream)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index or 0) as clk:
         torch.cuda.synchronize(dev)
+        e0.record(stream)
         for i in range(steps):
-            step(evs[i])
+            fwd()
+        e1.record(stream)
         torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    for _ in range(warmup):
+        step()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    for i in range(steps):
+        step(evs[i])
+    torch.cuda.synchronize(dev)
     moe.read_device_status(ws, stream)
-    ms = evs[0][0].elapsed_time(evs[-1][4]) / steps
     op_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i in range(4)]
     counts = (off[1:] - off[:-1]).cpu()
     touched = int((counts > 0).sum()) + S
@@ -372,7 +390,8 @@ def time_workload(moe, name: str, steps: int, warmup: int, dev, stream, peaks, p
     res = {"ms_per_step": ms, "tokens_per_s": T / (ms / 1e3),
            "tflops": mw.flops(w)["total"] / (ms / 1e3) / 1e12,
            "op_ms": {"route": op_ms[0], "permute": op_ms[1], "expert_ffn": op_ms[2],
-                     "combine": op_ms[3]},
+                     "combine": op_ms[3],
+                     "op_chain_step": evs[0][0].elapsed_time(evs[-1][4]) / steps},
            "expert_gemms": roof,
            "step_hbm": {"algorithmic_bytes": sb, "achieved_gbs": sb / (ms / 1e3) / 1e9,
                         "frac": sb / (ms / 1e3) / 1e9 / hbm_peak},
@@ -444,19 +463,32 @@ def gpu_arm(args, world, rank, local):
         if ev is not None:
             ev[4].record(st)
 
+    def fwd(st=None):
+        """One step through the one-call API (moe_forward / moe_forward_prenorm),
+        inputs resident on the device: the headline step."""
+        st = stream if st is None else st
+        if args.prenorm:
+            moe.moe_forward_prenorm(L, d["x"], nw, mw.RMS_NORM_EPS, d["w_router"], d["corr_bias"],
+                                    d["w_gate_up"], d["w_down"], wsgu, wsd, out, ws, stream=st)
+        else:
+            moe.moe_forward(L, d["x"], d["w_router"], d["corr_bias"], d["w_gate_up"], d["w_down"],
+                            wsgu, wsd, out, ws, stream=st)
+
+    # the headline step: moe_forward, or the op chain in the row-gathering
+    # mode (which moe_forward does not use)
+    headline = (lambda st=None: step(st=st)) if args.gather_rows else fwd
     for _ in range(args.warmup):
-        step()
+        headline()
     torch.cuda.synchronize(dev)
     moe.read_device_status(ws, stream)
     graph = None
     if args.graph:
-        # the whole op chain of one step captured once and replayed (the
-        # per-op events stay outside: op_ms then has only the total)
+        # one step captured once and replayed
         graph = torch.cuda.CUDAGraph()
         cap = torch.cuda.Stream(dev)
         cap.wait_stream(stream)
         with torch.cuda.graph(graph, stream=cap):
-            step(st=cap)
+            headline(st=cap)
         torch.cuda.synchronize(dev)
         # the replay must do the step's work: from a zeroed output it gives the
         # eager step's bits
@@ -465,37 +497,46 @@ def gpu_arm(args, world, rank, local):
         torch.cuda.synchronize(dev)
         replayed = out.clone()
         out.zero_()
-        step()
+        headline()
         torch.cuda.synchronize(dev)
         if not (torch.equal(replayed, out) and bool(replayed.abs().sum() > 0)):
             raise RuntimeError("the captured graph does not reproduce the eager step")
 
     # ---- timed region: K steps, inputs (weights 9.7 GB at the default
     # workload) far larger than the 126 MB L2, so no flush is needed between steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize(dev)
+        e_start.record(stream)
         for i in range(args.steps):
             if graph is None:
-                step(evs[i])
+                headline()
             else:
-                evs[i][5 if args.prenorm else 0].record(stream)
                 graph.replay()
-                evs[i][4].record(stream)
+        e_end.record(stream)
         torch.cuda.synchronize(dev)
         barrier(world)
     clocks = clk.summary()
     moe.read_device_status(ws, stream)
+    ms_step = max_over_ranks(e_start.elapsed_time(e_end) / args.steps, world)
+
+    # ---- the same steps as the op chain with CUDA events between the ops:
+    # the per-op breakdown and the expert GEMMs' own time (for the roofline)
+    for _ in range(args.warmup):
+        step()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    moe.read_device_status(ws, stream)
+    op_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(4)]
+    norm_ms = (sum(e[5].elapsed_time(e[0]) for e in evs) / args.steps) if args.prenorm else None
     first = 5 if args.prenorm else 0
-    total_ms = evs[0][first].elapsed_time(evs[-1][4])
-    if graph is None:
-        op_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(4)]
-        norm_ms = (sum(e[5].elapsed_time(e[0]) for e in evs) / args.steps) if args.prenorm else None
-    else:
-        op_ms = [float("nan")] * 4
-        norm_ms = float("nan") if args.prenorm else None
-    ms_step = max_over_ranks(total_ms / args.steps, world)
+    chain_ms = evs[0][first].elapsed_time(evs[-1][4]) / args.steps
 
     # ---- end to end through the public one-call API with host buffers: every
     # step copies its input from pinned host memory and its output back.  Two
@@ -551,9 +592,7 @@ def gpu_arm(args, world, rank, local):
     if rank == 0:
         peaks, peak_src = load_peaks()
         fl = mw.flops(w)
-        # per-op times need the events between ops; a graph replay has only the
-        # step's: the roofline then charges the expert flops with the whole step
-        ffn_ms = op_ms[2] if graph is None else ms_step
+        ffn_ms = op_ms[2]          # the expert GEMMs' own time (op chain)
         counts = (off[1:] - off[:-1]).cpu()
         touched = int((counts > 0).sum()) + S
         roof = gemm_roofline(w, ffn_ms, touched, peaks, peak_src)
@@ -576,9 +615,12 @@ def gpu_arm(args, world, rank, local):
                                            "rows rounded to fp16" if L.down_f16 else w.dtype),
                        "l2": "inputs larger than L2 (expert weights %.1f GB)" % (mw.weight_bytes(w) / 1e9)},
             "tflops": world * fl["total"] / (ms_step / 1e3) / 1e12,
-            "op_ms": {"route": op_ms[0], "permute": op_ms[1], "expert_ffn": op_ms[2], "combine": op_ms[3]},
-            "roofline": {"kernel": ("grouped expert GEMMs (gate_up + down launches of moe_expert_ffn)"
-                                    if graph is None else "whole step (one CUDA graph replay)"),
+            "op_ms": {"route": op_ms[0], "permute": op_ms[1], "expert_ffn": op_ms[2], "combine": op_ms[3],
+                      "op_chain_step": chain_ms},
+            "step": ("moe_forward_prenorm" if args.prenorm else "moe_forward") if not args.gather_rows
+                    else "op chain (moe_route, moe_permute, moe_expert_ffn, moe_combine)",
+            "roofline": {"kernel": "grouped expert GEMMs (gate_up + down launches of moe_expert_ffn, "
+                                   "timed in the op chain)",
                          **roof},
             "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
@@ -591,21 +633,22 @@ def gpu_arm(args, world, rank, local):
         }
         if graph is not None:
             line["config"]["graph"] = True
-            del line["op_ms"]
         if args.gather_rows:
             line["config"]["a_rows"] = "gathered from x by the gate_up GEMM (no x_perm copy)"
-            line["gpu_launches"] -= args.steps          # no row-gather launch in the permute
+            # the op chain: no row-gather launch in the permute, and the shared
+            # experts inside the expert call (no side-stream launches)
+            side = 2 if (S and w.dtype == "bf16") else 0
+            line["gpu_launches"] -= args.steps * (1 + side)
         if args.prenorm:
             # the block: post_attention_layernorm, then the layer
             el_x = 2 if w.dtype == "bf16" else 4
             nb = 2 * T * H * el_x
             line["config"]["block"] = "rmsnorm prologue + layer"
-            if graph is None:
-                line["op_ms"]["rmsnorm"] = norm_ms
-                line["rmsnorm_roofline"] = {"bound": "hbm", "achieved": nb / (norm_ms / 1e3) / 1e9,
-                                            "peak": hbm_peak, "unit": "GB/s",
-                                            "frac": nb / (norm_ms / 1e3) / 1e9 / hbm_peak,
-                                            "algorithmic_bytes": nb}
+            line["op_ms"]["rmsnorm"] = norm_ms
+            line["rmsnorm_roofline"] = {"bound": "hbm", "achieved": nb / (norm_ms / 1e3) / 1e9,
+                                        "peak": hbm_peak, "unit": "GB/s",
+                                        "frac": nb / (norm_ms / 1e3) / 1e9 / hbm_peak,
+                                        "algorithmic_bytes": nb}
         if world == 1 and not args.no_per_config and w.name == DEFAULT_WORKLOAD and graph is None:
             # the task's other workloads, timed in this run with the same
             # step counts (one GPU only: the replicas time the default one)

@@ -350,9 +350,10 @@ moe_status_t moe_dense_workspace_size(const moe_dense_desc_t* desc, size_t* byte
 /*
  * moe_dense_mlp — InklingDenseMLP.forward.  bf16 layers run both projections
  * on the tcgen05 tensor cores (bf16 operands, fp32 accumulation; h rounded
- * to bf16, y kept fp32 and rounded once into out); fp32 layers run them in
- * fp32 on the CUDA cores.  Workspace as for the MoE layer: initialise its
- * status word once with moe_workspace_init().
+ * to bf16, y kept fp32 and rounded once into out); MOE_BF16_F16DOWN layers
+ * round h to fp16 and take w_down in fp16 (the down projection's operands);
+ * fp32 layers run them in fp32 on the CUDA cores.  Workspace as for the MoE
+ * layer: initialise its status word once with moe_workspace_init().
  */
 moe_status_t moe_dense_mlp(const moe_dense_desc_t* desc, const void* x, const void* w_gate_up,
                            const void* w_down, void* out, void* workspace, size_t workspace_bytes,

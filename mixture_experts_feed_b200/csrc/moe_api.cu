@@ -2,6 +2,7 @@
 // checks, workspace layout and the order of launches.  Every step of the
 // layer runs in this library's kernels; there is no host compute path.
 #include <atomic>
+#include <mutex>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -176,13 +177,13 @@ moe_status_t permute_impl(const Layer& L, const int32_t* topk_idx, const uint8_t
                                     num_sms(), stream));
 }
 
-moe_status_t ffn_impl(const Layer& L, const void* x, const void* x_perm, const int32_t* offsets,
-                      const int32_t* perm_slot, const float* topk_w, const float* gamma,
-                      const void* wgu, const void* wd, const void* wsgu, const void* wsd,
-                      void* y_routed, void* y_shared, void* ws, cudaStream_t stream) {
-  const WsLayout w = ws_layout(L);
-  void* h = region<void>(ws, w.h);
-  int32_t* status = region<int32_t>(ws, w.status);
+// The expert GEMMs of `L` with the activated rows in `h` (routed rows first,
+// then S x T shared rows) and the status word at `status`.
+moe_status_t ffn_launch(const Layer& L, const void* x, const void* x_perm, const int32_t* offsets,
+                        const int32_t* perm_slot, const float* topk_w, const float* gamma,
+                        const void* wgu, const void* wd, const void* wsgu, const void* wsd,
+                        void* y_routed, void* y_shared, void* h, int32_t* status,
+                        cudaStream_t stream) {
   if (L.dtype == MOE_BF16) {
     bool map_error = false;
     const cudaError_t e = launch_expert_ffn_bf16(L, x, x_perm, offsets, perm_slot, topk_w, gamma,
@@ -196,8 +197,56 @@ moe_status_t ffn_impl(const Layer& L, const void* x, const void* x_perm, const i
                                            num_sms(), stream));
 }
 
+moe_status_t ffn_impl(const Layer& L, const void* x, const void* x_perm, const int32_t* offsets,
+                      const int32_t* perm_slot, const float* topk_w, const float* gamma,
+                      const void* wgu, const void* wd, const void* wsgu, const void* wsd,
+                      void* y_routed, void* y_shared, void* ws, cudaStream_t stream) {
+  const WsLayout w = ws_layout(L);
+  return ffn_launch(L, x, x_perm, offsets, perm_slot, topk_w, gamma, wgu, wd, wsgu, wsd, y_routed,
+                    y_shared, region<void>(ws, w.h), region<int32_t>(ws, w.status), stream);
+}
+
+// The side stream of moe_forward on each device, with its fork and join
+// events: created on first use (no device memory), kept for the life of the
+// process.  A mutex orders the fork/join sequences of calls from several host
+// threads, so that each record/wait pair of one call is not interleaved
+// with another call's.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxSideDevices = 64;
+SideStream g_side[kMaxSideDevices];
+std::mutex g_side_mutex;
+
+// Returns the side stream of the current device (nullptr if it cannot be made).
+SideStream* side_stream() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxSideDevices) return nullptr;
+  SideStream& ss = g_side[dev];
+  if (ss.stream == nullptr) {
+    cudaStream_t st = nullptr;
+    cudaEvent_t f = nullptr, j = nullptr;
+    if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess)
+      return nullptr;
+    ss.fork = f;
+    ss.join = j;
+    ss.stream = st;
+  }
+  return &ss;
+}
+
 // moe_forward with an optional RMSNorm prologue (norm_weight != null): the
 // normalised input goes to the workspace and feeds every later step.
+//
+// bf16 layers with shared experts overlap them with the permutation: after
+// the router, a fork to the side stream runs the shared experts' GEMMs (they
+// need the gammas, not the permutation) while the caller's stream runs the
+// permutation and the routed experts' GEMMs; the join comes before the
+// combine.  The shared experts write their own activated rows (after the
+// routed rows in h) and y_shared, so the two streams share no buffer.
 moe_status_t forward_checked(const moe_layer_desc_t* desc, const void* x, const void* norm_weight,
                              float norm_eps, const float* w_router, const float* corr_bias,
                              const void* w_gate_up, const void* w_down, const void* ws_gate_up,
@@ -229,12 +278,39 @@ moe_status_t forward_checked(const moe_layer_desc_t* desc, const void* x, const 
   void* y_routed = region<void>(workspace, w.y_routed);
   void* y_shared = region<void>(workspace, w.y_shared);
   MOE_TRY(route_impl(L, x, w_router, corr_bias, tw, ti, sg, workspace, s));
+  SideStream* side = (L.dtype == MOE_BF16 && L.S > 0) ? side_stream() : nullptr;
+  if (side != nullptr) {
+    std::lock_guard<std::mutex> lock(g_side_mutex);
+    MOE_TRY(cuda_status(cudaEventRecord(side->fork, s)));
+    MOE_TRY(cuda_status(cudaStreamWaitEvent(side->stream, side->fork, 0)));
+    // the shared groups alone (E = 0, k = 0), their h rows after the routed ones
+    Layer Ls = L;
+    Ls.E = 0;
+    Ls.k = 0;
+    void* h_shared = static_cast<uint8_t*>(region<void>(workspace, w.h)) +
+                     static_cast<size_t>(L.T) * L.k * L.I * 2;
+    bool map_error = false;
+    const cudaError_t e = launch_expert_ffn_bf16(Ls, x, x, nullptr, nullptr, nullptr, sg, nullptr,
+                                                 nullptr, ws_gate_up, ws_down, h_shared, y_shared,
+                                                 y_shared, region<int32_t>(workspace, w.status),
+                                                 num_sms(), side->stream, &map_error);
+    if (map_error) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(cuda_status(e));
+    MOE_TRY(cuda_status(cudaEventRecord(side->join, side->stream)));
+  }
   // the permuted copy of x: the GEMM's A tiles are then whole TMA boxes (the
   // row-gathering mode, x_perm = null, issues one TMA per 4 rows and runs
   // slower once tiles are full)
   MOE_TRY(permute_impl(L, ti, padding_mask, x, offsets, perm_slot, inv_perm, x_perm, workspace, s));
-  MOE_TRY(ffn_impl(L, x, x_perm, offsets, perm_slot, tw, sg, w_gate_up, w_down, ws_gate_up,
-                   ws_down, y_routed, y_shared, workspace, s));
+  Layer Lr = L;
+  if (side != nullptr) Lr.S = 0;   // the routed groups only: the shared ones run on the side stream
+  MOE_TRY(ffn_launch(Lr, x, x_perm, offsets, perm_slot, tw, sg, w_gate_up, w_down, ws_gate_up,
+                     ws_down, y_routed, y_shared, region<void>(workspace, w.h),
+                     region<int32_t>(workspace, w.status), s));
+  if (side != nullptr) {
+    std::lock_guard<std::mutex> lock(g_side_mutex);
+    MOE_TRY(cuda_status(cudaStreamWaitEvent(s, side->join, 0)));
+  }
   return cuda_status(launch_combine(L, y_routed, y_shared, inv_perm, out,
                                     region<int32_t>(workspace, w.status), num_sms(), s));
 }
@@ -541,8 +617,9 @@ int32_t moe_forward_kernel_count(const moe_layer_desc_t* desc) {
   // router: (bf16: split + tensor-core logits | fp32: logits) + top-k (plus
   // a partial-logit sum when K is split 4 or more ways); permute: chunk
   // counts, chunk scan, scatter, row gather; experts: gate_up + down (bf16
-  // with T > 128: CTA-pair launch + single-CTA launch each); combine.
-  const int experts = L.dtype == MOE_BF16 ? (L.T > 128 ? 4 : 2) : 2;
+  // with T > 128: CTA-pair launch + single-CTA launch each; bf16 with shared
+  // experts: their gate_up + down on the side stream too); combine.
+  const int experts = L.dtype == MOE_BF16 ? (L.T > 128 ? 4 : 2) + (L.S > 0 ? 2 : 0) : 2;
   return (L.dtype == MOE_BF16 ? 2 : 1) + router_topk_launches(router_ksplit(L)) + 4 + experts + 1;
 }
 

@@ -525,7 +525,8 @@ def test_down_weight_conversion():
     g = torch.Generator().manual_seed(9)
     t = (torch.randn(4096, generator=g) * 0.02).to(torch.bfloat16)
     t[:5] = torch.tensor([1e-9, 3e-7, 7e4, -1e6, float("nan")]).to(torch.bfloat16)
-    t[5:9] = torch.tensor([0.0, -0.0, 2.0 ** -14, 65504.0]).to(torch.bfloat16)
+    # 65280 is the largest bf16 value below 65504 (65504 itself rounds to 65536 in bf16)
+    t[5:9] = torch.tensor([0.0, -0.0, 2.0 ** -14, 65280.0]).to(torch.bfloat16)
     count = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = moe.convert_bf16_to_f16(t.cuda(), nonfinite=count)
     torch.cuda.synchronize()
