@@ -253,36 +253,36 @@ def reference_arm(args, world, rank):
 
 
 # ----------------------------------------------------------------- GPU arm
-def expert_ffn_bytes(w, touched: int) -> int:
+def expert_ffn_bytes(w, touched: int, yel: int = 4) -> int:
     """Algorithmic bytes of moe_expert_ffn: the weights of every group with
     rows (routed experts with a nonzero count, every shared expert) once, the
     routed A rows (x_perm) and shared A rows (x) read once, h written and read
-    once in the dtype, the fp32 down rows written once."""
+    once (2 bytes), the down rows written once (``yel`` bytes: 4 fp32, 2 fp16)."""
     el = 2 if w.dtype == "bf16" else 4
     rows = w.T * (w.k + w.S)
-    return touched * 3 * w.H * w.I * el + rows * (w.H * el + 2 * w.I * el + 4 * w.H)
+    return touched * 3 * w.H * w.I * el + rows * (w.H * el + 2 * w.I * el + yel * w.H)
 
 
-def step_bytes(w, touched: int) -> int:
+def step_bytes(w, touched: int, yel: int = 4) -> int:
     """Algorithmic bytes of one layer step: the expert call's bytes, plus the
     fp32 router bank and bias, x read by the router and the shared experts'
-    row gather, x_perm written, the fp32 rows read back by the combine and
+    row gather, x_perm written, the down rows read back by the combine and
     the output written."""
     el = 2 if w.dtype == "bf16" else 4
     router = 4 * (w.E + w.S) * w.H + 4 * w.E + w.T * w.H * el
     permute = w.T * w.k * w.H * el
-    combine = 4 * w.T * (w.k + w.S) * w.H + w.T * w.H * el
-    return expert_ffn_bytes(w, touched) + router + permute + combine
+    combine = yel * w.T * (w.k + w.S) * w.H + w.T * w.H * el
+    return expert_ffn_bytes(w, touched, yel) + router + permute + combine
 
 
-def gemm_roofline(w, ffn_ms: float, touched: int, peaks, peak_src: str):
+def gemm_roofline(w, ffn_ms: float, touched: int, peaks, peak_src: str, yel: int = 4):
     """Roofline of the expert GEMMs (the four launches of moe_expert_ffn):
     tensor-bound against the measured burst bf16 peak (the calls are timed in
     a region of well under a second), or HBM-bound against the measured copy
     bandwidth when their flops per algorithmic byte fall below the ridge."""
     fl = mw.flops(w)
     ffn_flops = fl["routed"] + fl["shared"]
-    ffn_bytes = expert_ffn_bytes(w, touched)
+    ffn_bytes = expert_ffn_bytes(w, touched, yel)
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
@@ -332,8 +332,8 @@ def time_workload(moe, name: str, steps: int, warmup: int, dev, stream, peaks, p
     ps = torch.empty(T * k, dtype=torch.int32, device=dev)
     ip = torch.empty(T * k, dtype=torch.int32, device=dev)
     xp = torch.empty(T * k, H, dtype=L.dtype, device=dev)
-    yr = torch.empty(T * k, H, dtype=torch.float32, device=dev)
-    ys = torch.empty(S * T, H, dtype=torch.float32, device=dev) if S else None
+    yr = torch.empty(T * k, H, dtype=L.y_dtype, device=dev)
+    ys = torch.empty(S * T, H, dtype=L.y_dtype, device=dev) if S else None
     out = torch.empty(T, H, dtype=L.dtype, device=dev)
     wsgu, wsd = (d["ws_gate_up"], d["ws_down"]) if S else (None, None)
 
@@ -384,9 +384,10 @@ def time_workload(moe, name: str, steps: int, warmup: int, dev, stream, peaks, p
     op_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i in range(4)]
     counts = (off[1:] - off[:-1]).cpu()
     touched = int((counts > 0).sum()) + S
-    roof = gemm_roofline(w, op_ms[2], touched, peaks, peak_src)
+    yel = 2 if L.down_f16 else 4
+    roof = gemm_roofline(w, op_ms[2], touched, peaks, peak_src, yel)
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    sb = step_bytes(w, touched)
+    sb = step_bytes(w, touched, yel)
     res = {"ms_per_step": ms, "tokens_per_s": T / (ms / 1e3),
            "tflops": mw.flops(w)["total"] / (ms / 1e3) / 1e12,
            "op_ms": {"route": op_ms[0], "permute": op_ms[1], "expert_ffn": op_ms[2],
@@ -429,8 +430,8 @@ def gpu_arm(args, world, rank, local):
     # the permuted copy of x, as moe_forward makes it (--gather-rows: none;
     # the gate_up GEMM then gathers the routed rows of x itself)
     xp = None if args.gather_rows else torch.empty(T * k, H, dtype=L.dtype, device=dev)
-    yr = torch.empty(T * k, H, dtype=torch.float32, device=dev)
-    ys = torch.empty(S * T, H, dtype=torch.float32, device=dev) if S else None
+    yr = torch.empty(T * k, H, dtype=L.y_dtype, device=dev)
+    ys = torch.empty(S * T, H, dtype=L.y_dtype, device=dev) if S else None
     out = torch.empty(T, H, dtype=L.dtype, device=dev)
     out_host = torch.empty(T, H, dtype=L.dtype).pin_memory()
     wsgu = d.get("ws_gate_up") if S else None
@@ -595,14 +596,15 @@ def gpu_arm(args, world, rank, local):
         ffn_ms = op_ms[2]          # the expert GEMMs' own time (op chain)
         counts = (off[1:] - off[:-1]).cpu()
         touched = int((counts > 0).sum()) + S
-        roof = gemm_roofline(w, ffn_ms, touched, peaks, peak_src)
+        yel = 2 if L.down_f16 else 4
+        roof = gemm_roofline(w, ffn_ms, touched, peaks, peak_src, yel)
         # the captured bytes are those of the launches reading x_perm; the
         # row-gathering mode reads x instead and has no capture
         traffic, traffic_src = traffic_of(w.name)
         roof["traffic"] = None if args.gather_rows else traffic
         roof["traffic_source"] = None if args.gather_rows or traffic is None else traffic_src
         hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-        sb = step_bytes(w, touched)
+        sb = step_bytes(w, touched, yel)
         tokens_s = world * T / (ms_step / 1e3)
         line = {
             "metric": METRIC, "value": tokens_s, "unit": "tokens/s", "n_gpus": world,
@@ -611,8 +613,8 @@ def gpu_arm(args, world, rank, local):
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02^2) weights, random init)",
             "config": {"workload": w.name, "T": T, "H": H, "E": E, "k": k, "S": S, "I": w.I,
                        "route_scale": w.route_scale, "parallelism": f"replicas x{world}",
-                       "down_projection": ("fp16: weights copied once from bf16 (exact), activated "
-                                           "rows rounded to fp16" if L.down_f16 else w.dtype),
+                       "down_projection": ("fp16: weights copied once from bf16, activated rows "
+                                           "and expert output rows in fp16" if L.down_f16 else w.dtype),
                        "l2": "inputs larger than L2 (expert weights %.1f GB)" % (mw.weight_bytes(w) / 1e9)},
             "tflops": world * fl["total"] / (ms_step / 1e3) / 1e12,
             "op_ms": {"route": op_ms[0], "permute": op_ms[1], "expert_ffn": op_ms[2], "combine": op_ms[3],

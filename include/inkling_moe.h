@@ -36,8 +36,8 @@
  *       ws_gate_up [S, 2I, H], ws_down [S, H, I]   (shared experts)
  *     x, the expert weights, x_perm and out share `dtype` (MOE_BF16_F16DOWN:
  *     bf16, with w_down and ws_down fp16); the expert output rows
- *     y_routed / y_shared are fp32 in every dtype (they are summed in fp32
- *     and rounded once, in moe_combine).
+ *     y_routed / y_shared are fp32 (MOE_BF16_F16DOWN: fp16); moe_combine
+ *     sums them in fp32 and rounds once.
  *   - Sizes: T = num_tokens, H = hidden, E = n_routed, k = top_k,
  *     S = n_shared, I = intermediate.  Limits: 1 <= k <= min(E, 16),
  *     E <= 1024, S <= 8, H % 64 == 0, I % 64 == 0, T <= 2^26,
@@ -79,16 +79,19 @@ typedef enum {
  *   MOE_BF16_F16DOWN  x, out, the router input and the gate_up weights bf16,
  *                     as MOE_BF16; the down projections' weights (w_down,
  *                     ws_down) fp16, and the activated rows h rounded to
- *                     fp16, 8 times finer than bf16.  The fp16 weights are
+ *                     fp16, 8 times finer than bf16; the expert output rows
+ *                     y are stored in fp16 too (half the bytes of fp32).
+ *                     The fp16 weights are
  *                     the checkpoint's bf16 values copied once with
  *                     moe_convert_bf16_to_f16 (exact for |w| in [2^-17, 65504]
  *                     and zero; smaller values change by at most 2^-25).
  *                     With bf16 h the rounding of h adds up to
  *                     about 1% of the output's RMS to the error of the final
  *                     bf16 rounding (1.7% of RMS when outputs reach 6 x RMS);
- *                     with fp16 h it adds about 0.1%.  An h value at or beyond
- *                     65520 in magnitude (an fp16 infinity) is recorded in the
- *                     workspace status word (MOE_ERR_DEVICE_CHECK).
+ *                     with fp16 h and fp16 y rows about 0.1–0.2%.  An h or y
+ *                     value at or beyond 65520 in magnitude (an fp16
+ *                     infinity) is recorded in the workspace status word
+ *                     (MOE_ERR_DEVICE_CHECK).
  */
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_BF16_F16DOWN = 2 } moe_dtype_t;
 
@@ -190,7 +193,7 @@ moe_status_t moe_permute_noalloc(const moe_layer_desc_t* desc, const int32_t* to
  * and for shared expert s and token t (weight shared_gamma[t*S+s]) the same
  * with x[t] and ws_*[s] into y_shared[s*T + t].  The activated rows are
  * rounded to dtype (MOE_BF16_F16DOWN: fp16) before the down projection; y
- * rows are written in fp32.
+ * rows are written in fp32 (MOE_BF16_F16DOWN: fp16).
  * x_perm may be NULL: the gate_up GEMM then reads row r straight from
  * x[perm_slot[r] / k] (bf16: TMA gathers of 4 rows into the tile), with the
  * same results bit for bit and without the [T*k, H] copy (memory saved:
@@ -201,7 +204,8 @@ moe_status_t moe_permute_noalloc(const moe_layer_desc_t* desc, const int32_t* to
  *   expert-parallel rank receives are (moe_ep_dispatch_prep).
  *   x [T,H], x_perm [T*k,H] or NULL, expert_offsets, perm_slot, topk_w [T*k],
  *   shared_gamma [T*S] (NULL iff S == 0), weights as above,
- *   y_routed [T*k, H] fp32 out (rows < off[E] written), y_shared [S*T, H] fp32 out.
+ *   y_routed [T*k, H] out (rows < off[E] written), y_shared [S*T, H] out: fp32
+ *   (MOE_BF16_F16DOWN: fp16).
  */
 moe_status_t moe_expert_ffn(const moe_layer_desc_t* desc, const void* x, const void* x_perm,
                             const int32_t* expert_offsets, const int32_t* perm_slot,
@@ -220,7 +224,8 @@ moe_status_t moe_expert_ffn(const moe_layer_desc_t* desc, const void* x, const v
  * accumulation, activated rows rounded to dtype, y rows fp32).  It serves a
  * rank whose routed experts run elsewhere (expert parallelism).  S >= 1.
  *   x [T,H] dtype, shared_gamma [T,S] fp32, ws_gate_up [S,2I,H],
- *   ws_down [S,H,I], y_shared [S*T,H] fp32 out; workspace as moe_workspace_size.
+ *   ws_down [S,H,I], y_shared [S*T,H] out (fp32; MOE_BF16_F16DOWN: fp16);
+ *   workspace as moe_workspace_size.
  */
 moe_status_t moe_shared_ffn(const moe_layer_desc_t* desc, const void* x, const float* shared_gamma,
                             const void* ws_gate_up, const void* ws_down, void* y_shared,
@@ -254,7 +259,7 @@ moe_status_t moe_ep_dispatch_prep(const moe_layer_desc_t* desc, const int32_t* e
  * moe_combine — InklingMoE.forward recombination:
  *   out[t] = sum_s y_shared[s*T + t] + sum_{j<k, inv_perm[t*k+j] >= 0} y_routed[inv_perm[t*k+j]]
  * summed in fp32 in that fixed order, rounded once to dtype.  y_routed and
- * y_shared are fp32; out [T, H] has `dtype`.
+ * y_shared are fp32 (MOE_BF16_F16DOWN: fp16); out [T, H] has `dtype`.
  */
 moe_status_t moe_combine(const moe_layer_desc_t* desc, const void* y_routed, const void* y_shared,
                          const int32_t* inv_perm, void* out, void* workspace,

@@ -125,6 +125,11 @@ class Layer:
         """dtype of w_down / ws_down."""
         return torch.float16 if self.down_f16 else self.dtype
 
+    @property
+    def y_dtype(self) -> torch.dtype:
+        """dtype of the expert output rows y_routed / y_shared."""
+        return torch.float16 if self.down_f16 else torch.float32
+
     @staticmethod
     def from_workload(w, down_f16: bool = False) -> "Layer":
         return Layer(w.T, w.H, w.E, w.k, w.S, w.I, w.torch_dtype, w.route_scale, w.global_scale,
@@ -279,8 +284,8 @@ def moe_expert_ffn(layer: Layer, x, x_perm, expert_offsets, perm_slot, topk_w, s
     _expect(w_down, "w_down", (L.E, L.H, L.I), L.down_dtype)
     _expect(ws_gate_up, "ws_gate_up", (L.S, 2 * L.I, L.H), L.dtype, allow_none=L.S == 0)
     _expect(ws_down, "ws_down", (L.S, L.H, L.I), L.down_dtype, allow_none=L.S == 0)
-    _expect(y_routed, "y_routed", (L.T * L.k, L.H), torch.float32)
-    _expect(y_shared, "y_shared", (L.S * L.T, L.H), torch.float32, allow_none=L.S == 0)
+    _expect(y_routed, "y_routed", (L.T * L.k, L.H), L.y_dtype)
+    _expect(y_shared, "y_shared", (L.S * L.T, L.H), L.y_dtype, allow_none=L.S == 0)
     _check(LIB.moe_expert_ffn(ctypes.byref(L.desc()), _ptr(x), _ptr(x_perm), _ptr(expert_offsets),
                               _ptr(perm_slot), _ptr(topk_w), _ptr(shared_gamma), _ptr(w_gate_up),
                               _ptr(w_down), _ptr(ws_gate_up), _ptr(ws_down), _ptr(y_routed),
@@ -296,7 +301,7 @@ def moe_shared_ffn(layer: Layer, x, shared_gamma, ws_gate_up, ws_down, y_shared,
     _expect(shared_gamma, "shared_gamma", (L.T, L.S), torch.float32)
     _expect(ws_gate_up, "ws_gate_up", (L.S, 2 * L.I, L.H), L.dtype)
     _expect(ws_down, "ws_down", (L.S, L.H, L.I), L.down_dtype)
-    _expect(y_shared, "y_shared", (L.S * L.T, L.H), torch.float32)
+    _expect(y_shared, "y_shared", (L.S * L.T, L.H), L.y_dtype)
     _check(LIB.moe_shared_ffn(ctypes.byref(L.desc()), _ptr(x), _ptr(shared_gamma),
                               _ptr(ws_gate_up), _ptr(ws_down), _ptr(y_shared), ws.data_ptr(),
                               ws.numel(), _stream(stream)), "moe_shared_ffn")
@@ -324,8 +329,8 @@ def moe_ep_dispatch_prep(layer: Layer, expert_offsets, perm_slot, topk_w, row_w,
 
 def moe_combine(layer: Layer, y_routed, y_shared, inv_perm, out, ws, stream=None):
     L = layer
-    _expect(y_routed, "y_routed", (L.T * L.k, L.H), torch.float32)
-    _expect(y_shared, "y_shared", (L.S * L.T, L.H), torch.float32, allow_none=L.S == 0)
+    _expect(y_routed, "y_routed", (L.T * L.k, L.H), L.y_dtype)
+    _expect(y_shared, "y_shared", (L.S * L.T, L.H), L.y_dtype, allow_none=L.S == 0)
     _expect(inv_perm, "inv_perm", (L.T * L.k,), torch.int32)
     _expect(out, "out", (L.T, L.H), L.dtype)
     _check(LIB.moe_combine(ctypes.byref(L.desc()), _ptr(y_routed), _ptr(y_shared), _ptr(inv_perm),

@@ -2,13 +2,15 @@
 // InklingMoE.forward):
 //   out[t] = sum_s y_shared[s*T + t] + sum_j y_routed[inv_perm[t*k + j]]
 // in fp32, in that fixed order (shared s ascending, then choices j
-// ascending), rounded once to the output dtype.  The rows are fp32.  The routing weights are
+// ascending), rounded once to the output dtype.  The rows are fp32, or fp16
+// for MOE_BF16_F16DOWN layers (widened exactly before the sum).  The routing weights are
 // already folded into the rows (inkling_swiglu multiplies silu(g)*u by them),
 // so the sum is unweighted.  One block per token; 16-byte vector loads and
 // stores along the hidden dim, coalesced across the block.  HBM-bound.
 #include <algorithm>
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -18,7 +20,7 @@
 namespace moe {
 namespace {
 
-// acc[0..V) += 4*V/4 consecutive fp32 values (V = 8 or 4)
+// acc[0..V) += V consecutive fp32 values (V = 8 or 4)
 template <int V>
 __device__ __forceinline__ void add_vec(float (&acc)[V], const float* p) {
 #pragma unroll
@@ -28,6 +30,19 @@ __device__ __forceinline__ void add_vec(float (&acc)[V], const float* p) {
     acc[4 * i + 1] += q.y;
     acc[4 * i + 2] += q.z;
     acc[4 * i + 3] += q.w;
+  }
+}
+
+// acc[0..8) += 8 consecutive fp16 values (one 16-byte load), each widened
+// exactly to fp32
+__device__ __forceinline__ void add_vec(float (&acc)[8], const __half* p) {
+  const uint4 q = __ldcs(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+    acc[2 * i] += f.x;
+    acc[2 * i + 1] += f.y;
   }
 }
 
@@ -44,9 +59,10 @@ __device__ __forceinline__ void store_vec(float* p, const float (&acc)[4]) {
   *reinterpret_cast<float4*>(p) = make_float4(acc[0], acc[1], acc[2], acc[3]);
 }
 
-template <typename TY>
+// TY: output dtype; TR: expert row dtype (fp32, or fp16 with bf16 output)
+template <typename TY, typename TR>
 __global__ void __launch_bounds__(256)
-    combine_kernel(const float* __restrict__ y_routed, const float* __restrict__ y_shared,
+    combine_kernel(const TR* __restrict__ y_routed, const TR* __restrict__ y_shared,
                    const int32_t* __restrict__ inv_perm, TY* __restrict__ out, int64_t T, int H,
                    int k, int S, int64_t rows_cap, int32_t* status) {
   constexpr int V = 16 / sizeof(TY);   // one 16-byte output store per vector
@@ -86,12 +102,16 @@ cudaError_t launch_combine(const Layer& L, const void* y_routed, const void* y_s
   const unsigned grid =
       static_cast<unsigned>(std::min<int64_t>(L.T, static_cast<int64_t>(num_sms) * 8));
   const int64_t cap = L.T * L.k;
-  if (L.dtype == MOE_BF16)
-    combine_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+  if (L.dtype == MOE_BF16 && L.y_f16)
+    combine_kernel<__nv_bfloat16, __half><<<grid, 256, 0, stream>>>(
+        static_cast<const __half*>(y_routed), static_cast<const __half*>(y_shared), inv_perm,
+        static_cast<__nv_bfloat16*>(out), L.T, L.H, L.k, L.S, cap, status);
+  else if (L.dtype == MOE_BF16)
+    combine_kernel<__nv_bfloat16, float><<<grid, 256, 0, stream>>>(
         static_cast<const float*>(y_routed), static_cast<const float*>(y_shared), inv_perm,
         static_cast<__nv_bfloat16*>(out), L.T, L.H, L.k, L.S, cap, status);
   else
-    combine_kernel<float><<<grid, 256, 0, stream>>>(
+    combine_kernel<float, float><<<grid, 256, 0, stream>>>(
         static_cast<const float*>(y_routed), static_cast<const float*>(y_shared), inv_perm,
         static_cast<float*>(out), L.T, L.H, L.k, L.S, cap, status);
   return cudaGetLastError();

@@ -17,7 +17,7 @@ enum DeviceCode : int32_t {
   DEV_OK = 0,
   DEV_BAD_EXPERT_ID = 0x101,   // topk_idx outside [0, E)
   DEV_BAD_ROW = 0x102,         // inv_perm / perm_slot outside its range
-  DEV_H_OVERFLOW = 0x103,      // an activated row value beyond the fp16 range (fp16 down projections)
+  DEV_F16_OVERFLOW = 0x103,    // an activated value or expert output beyond the fp16 range
   DEV_WAIT_TIMEOUT = 0x201,    // a pipeline wait ran past its time limit
 };
 

@@ -103,7 +103,8 @@ template <int MODE, bool PAIR_> struct Tile {
 struct alignas(64) GemmParams {
   CUtensorMap tmA[2];   // A operand of routed (0) and shared (1) groups: 2-D [rows, K]
   CUtensorMap tmB[2];   // weights of routed (0) and shared (1) groups: 3-D [G][N][K]
-  CUtensorMap tmY[2];   // kDown: fp32 output rows of routed (0) and shared (1) groups, box 32 x 32
+  CUtensorMap tmY[2];   // kDown: output rows of routed (0) and shared (1) groups: fp32, box
+                        // 32 rows x 32 columns, or fp16, box 32 x 64 (128 bytes a row either way)
   const int32_t* offsets;     // [E+1]
   const int32_t* perm_slot;   // [rows] slot of each permuted row (kGateUp weights)
   const float* topk_w;        // [T*k]
@@ -121,6 +122,7 @@ struct alignas(64) GemmParams {
   int gather_k;               // kGateUp: > 0 = routed A rows are gathered from x (tmA[0] over
                               // [T, H], box one row high): row r reads x[perm_slot[r] / gather_k]
   int f16;                    // kGateUp: h written in fp16; kDown: A (h) and B (weights) fp16
+  int y_f16;                  // kDown: output rows in fp16 (tmY boxes 32 rows x 64 columns)
   int64_t split_stride;       // kRouter: elements between partial outputs
 };
 
@@ -165,6 +167,28 @@ __device__ __forceinline__ void store_rows_f32(float* st, const uint32_t (&v)[32
     const float4 val = *reinterpret_cast<const float4*>(st + rr * STAGE_LD + sub_col);
     if (rr < rows_left)
       *reinterpret_cast<float4*>(out + (row0 + rr) * ld + col0 + sub_col) = val;
+  }
+  __syncwarp();
+}
+
+// The same for 32 rows x 64 fp16 columns (32 packed words a lane: 128 bytes
+// of its row), staged with a 36-word row stride.
+__device__ __forceinline__ void store_rows_f16(uint32_t* st, const uint32_t (&w)[32], int lane,
+                                               uint16_t* out, int64_t row0, int rows_left,
+                                               int64_t ld, int col0) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    *reinterpret_cast<uint4*>(st + lane * STAGE_LD + 4 * q) =
+        make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  __syncwarp();
+  const int sub_row = lane >> 3;          // 0..3
+  const int sub_col = (lane & 7) * 4;     // word offset 0..28 (8 fp16 each 4 words)
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int rr = it * 4 + sub_row;
+    const uint4 val = *reinterpret_cast<const uint4*>(st + rr * STAGE_LD + sub_col);
+    if (rr < rows_left)
+      *reinterpret_cast<uint4*>(out + (row0 + rr) * ld + col0 + 2 * sub_col) = val;
   }
   __syncwarp();
 }
@@ -515,6 +539,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       const uint32_t t_row = t_lane + static_cast<uint32_t>(acc * BN);
       const int n_here = min(bn, p.N - n * bn);
+      if (MODE == kDown && p.y_f16) {
+        // fp16 output rows: two 32-column chunks make one 128-byte row
+        // segment (n_here is a multiple of 64: H % 64 == 0); each 32-row slab
+        // goes through the swizzled staging box and one TMA store, as below
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; c += 2) {
+          const int col0 = n * bn + c * 32;
+          if (c * 32 >= n_here) break;             // warp-uniform
+          uint32_t v[32], v2[32], pk[32];
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * 32), v);
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 1) * 32), v2);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            pk[i] = pack_f16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]), h_overflow);
+            pk[16 + i] = pack_f16x2(__uint_as_float(v2[2 * i]), __uint_as_float(v2[2 * i + 1]), h_overflow);
+          }
+          if (lane == 0) bulk_wait_group_read0();
+          __syncwarp();
+          if (rows_left >= 32) {
+            uint8_t* box = reinterpret_cast<uint8_t*>(st);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ (lane & 7)) * 16)) =
+                  make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&p.tmY[gi.src], box, col0,
+                           static_cast<int32_t>(gi.out_row0 + row0 + quarter * 32));
+              bulk_commit_group();
+            }
+          } else {
+            store_rows_f16(reinterpret_cast<uint32_t*>(st), pk, lane,
+                           static_cast<uint16_t*>(p.out[gi.src]), gi.out_row0 + row0 + quarter * 32,
+                           rows_left, p.ld_out, col0);
+          }
+        }
+      } else {
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         const int col0 = n * bn + c * 32;
@@ -571,6 +634,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -579,8 +643,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       ++it;
     }
-    if (MODE == kGateUp && __any_sync(0xffffffffu, h_overflow) && lane == 0)
-      record_status(p.status, DEV_H_OVERFLOW);
+    if (MODE != kRouter && __any_sync(0xffffffffu, h_overflow) && lane == 0)
+      record_status(p.status, DEV_F16_OVERFLOW);
     // the warp's TMA stores complete before the block (and its shared memory) goes
     if (MODE == kDown && lane == 0) bulk_wait_group0();
   }
@@ -627,14 +691,15 @@ static bool encode_a(CUtensorMap* m, const void* base, int64_t rows, int K, int 
 
 // 2-D fp32 map over [rows, H] (H contiguous), box [32 rows, 32 columns],
 // 128B swizzle: the down projection's output rows, written by TMA stores.
-static bool encode_y(CUtensorMap* m, void* base, int64_t rows, int H) {
+static bool encode_y(CUtensorMap* m, void* base, int64_t rows, int H, bool f16 = false) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(H) * 4};
-  cuuint32_t box[2] = {32, 32};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(H) * (f16 ? 2 : 4)};
+  cuuint32_t box[2] = {f16 ? 64u : 32u, 32};   // 128 bytes a row
   cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+  return enc(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base,
+             dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -764,8 +829,9 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   // output maps: routed rows [T*k, H]; shared rows [S*T, H], or one partial
   // [T, H] per K split when the down projection splits K (the dense layer)
   const int64_t shared_rows = L.T * static_cast<int64_t>(L.S > tiling.down_ksplit ? L.S : tiling.down_ksplit);
-  if (ok && L.S > 0) ok = encode_y(&d.tmY[1], y_shared, shared_rows, L.H);
-  if (ok && routed) ok = encode_y(&d.tmY[0], y_routed, Rk, L.H);
+  const bool y_f16 = L.y_f16 && tiling.down_ksplit == 1;   // K-split partials stay fp32
+  if (ok && L.S > 0) ok = encode_y(&d.tmY[1], y_shared, shared_rows, L.H, y_f16);
+  if (ok && routed) ok = encode_y(&d.tmY[0], y_routed, Rk, L.H, y_f16);
   if (!routed) d.tmY[0] = d.tmY[1];
   if (L.S == 0) d.tmY[1] = d.tmY[0];
   if (!ok) { *map_error = true; return cudaErrorInvalidValue; }
@@ -781,6 +847,7 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   d.split_stride = L.T * static_cast<int64_t>(L.H);   // partial rows of the shared groups
   d.bn = 256;
   d.f16 = f16 ? 1 : 0;
+  d.y_f16 = y_f16 ? 1 : 0;
   e = pairs ? launch_mode<kDown, true>(d, num_sms, stream) : cudaSuccess;
   if (e == cudaSuccess && singles) e = launch_mode<kDown, false>(d, num_sms, stream);
   return e;

@@ -16,6 +16,9 @@ struct Layer {
   // MOE_BF16_F16DOWN layers: the down projections' weights are fp16 and the
   // activated rows h are rounded to fp16 (dtype is MOE_BF16)
   bool down_f16 = false;
+  // the expert output rows y_routed / y_shared are fp16 (MOE_BF16_F16DOWN MoE
+  // layers); else fp32.  The dense layer keeps fp32 rows (its K-split partials).
+  bool y_f16 = false;
 };
 
 // moe_api.cu: SM count of the current device (cached per device), and the

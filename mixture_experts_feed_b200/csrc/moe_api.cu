@@ -67,8 +67,9 @@ WsLayout ws_layout(const Layer& L) {
   w.inv_perm = take(Rk * 4);
   w.x_perm = take(Rk * L.H * elt);
   w.h = take(Rh * L.I * elt);
-  w.y_routed = take(Rk * L.H * 4);   // expert output rows stay fp32
-  w.y_shared = take(T * L.S * L.H * 4);
+  const size_t yel = L.y_f16 ? 2 : 4;   // expert output rows: fp32, or fp16
+  w.y_routed = take(Rk * L.H * yel);
+  w.y_shared = take(T * L.S * L.H * yel);
   w.x_norm = take(T * L.H * elt);    // moe_forward_prenorm: the normalised input
   w.total = off;
   return w;
@@ -96,6 +97,7 @@ moe_status_t check_desc(const moe_layer_desc_t* d, Layer* L) {
   L->I = d->intermediate;
   L->dtype = d->dtype == MOE_F32 ? MOE_F32 : MOE_BF16;
   L->down_f16 = d->dtype == MOE_BF16_F16DOWN;
+  L->y_f16 = L->down_f16;
   L->route_scale = d->route_scale;
   L->global_scale = d->global_scale;
   return MOE_OK;

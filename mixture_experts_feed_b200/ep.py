@@ -33,7 +33,7 @@ module holds the exchanges and their host-side bookkeeping only):
 Per rank and per step the exchange moves, for R_out rows sent and R_in rows
 received: ``R_out*(H*dtype + 4)`` bytes out and ``R_in*(H*dtype + 4)`` in for
 the rows and weights, and ``4*H`` bytes a row each way for the fp32 results
-(the layer keeps expert outputs in fp32 until the final rounding).
+(``2*H`` with fp16 down projections, whose expert output rows are fp16).
 
 The results equal the one-GPU layer's up to the order of rows inside the
 expert GEMM tiles, which does not change any row's arithmetic.
@@ -193,14 +193,15 @@ class ExpertParallelMoE:
         # 5: the local experts over the received rows (already grouped, in slot order)
         Ll = self.ops.Layer(R_in, H, El, 1, 0, self.I, self.dtype, self.route_scale,
                             self.global_scale, self.down_f16)
-        y_in = torch.empty(R_in, H, dtype=torch.float32, device=dev)
+        y_dtype = torch.float16 if self.down_f16 else torch.float32   # the expert output rows
+        y_in = torch.empty(R_in, H, dtype=y_dtype, device=dev)
         if R_in > 0:
             off_loc = torch.tensor(loc_off, dtype=torch.int32).to(dev)
             ws_loc = ops.new_workspace(Ll, device=dev)
             ops.moe_expert_ffn(Ll, x_in, x_in, off_loc, None, w_in, None, w["w_gate_up"],
                                w["w_down"], None, None, y_in, None, ws_loc)
         # 6: the output rows back into this rank's permuted order
-        yr = torch.empty(T * k, H, dtype=torch.float32, device=dev)
+        yr = torch.empty(T * k, H, dtype=y_dtype, device=dev)
         sends, recvs = [], []
         for s in range(W):
             for e in range(El):
@@ -216,7 +217,7 @@ class ExpertParallelMoE:
         # 7: shared experts on this rank's tokens, then the fixed-order combine
         ys = None
         if S:
-            ys = torch.empty(S * T, H, dtype=torch.float32, device=dev)
+            ys = torch.empty(S * T, H, dtype=y_dtype, device=dev)
             ops.moe_shared_ffn(L, x, sg, w["ws_gate_up"], w["ws_down"], ys, ws)
         out = torch.empty(T, H, dtype=self.dtype, device=dev)
         ops.moe_combine(L, yr, ys, ip, out, ws)

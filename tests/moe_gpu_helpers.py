@@ -61,8 +61,8 @@ def run_chain(L: moe.Layer, d: Dict[str, torch.Tensor], padding_mask: Optional[t
         "perm_slot": torch.full((T * k,), -7, dtype=torch.int32, device=dev),
         "inv_perm": torch.full((T * k,), -7, dtype=torch.int32, device=dev),
         "x_perm": torch.empty(T * k, H, dtype=L.dtype, device=dev),
-        "y_routed": torch.empty(T * k, H, dtype=torch.float32, device=dev),
-        "y_shared": torch.empty(S * T, H, dtype=torch.float32, device=dev) if S else None,
+        "y_routed": torch.empty(T * k, H, dtype=L.y_dtype, device=dev),
+        "y_shared": torch.empty(S * T, H, dtype=L.y_dtype, device=dev) if S else None,
         "out": torch.empty(T, H, dtype=L.dtype, device=dev),
     }
     pm = None if padding_mask is None else padding_mask.to(dev, torch.uint8).contiguous()

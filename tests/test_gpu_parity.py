@@ -544,11 +544,17 @@ def test_down_weight_conversion():
         moe.prepare_down_weights(t.cuda())
 
 
-def test_fp16_activation_overflow_is_reported():
-    """With fp16 down projections an activated value beyond the fp16 range is
-    recorded in the status word (0x103), not passed on silently."""
+@pytest.mark.parametrize("where", ["h", "y"])
+def test_fp16_overflow_is_reported(where):
+    """With fp16 down projections an activated value (h) or an expert output
+    (y) beyond the fp16 range is recorded in the status word (0x103), not
+    passed on silently."""
     w, inputs = small_case(64, 128, 8, 2, 1, 64)
-    inputs["w_gate_up"] = (inputs["w_gate_up"].float() * 3000.0).to(torch.bfloat16)
+    if where == "h":
+        inputs["w_gate_up"] = (inputs["w_gate_up"].float() * 3000.0).to(torch.bfloat16)
+    else:   # down weights of about 2000: finite in fp16, outputs far beyond 65504
+        for n in ("w_down", "ws_down"):
+            inputs[n] = (inputs[n].float() * 1e5).clamp(-6e4, 6e4).to(torch.bfloat16)
     L = moe.Layer.from_workload(w, down_f16=True)
     d = to_device(inputs, down_f16=True)
     ws = moe.new_workspace(L)
