@@ -552,7 +552,9 @@ def test_fp16_overflow_is_reported(where):
     w, inputs = small_case(64, 128, 8, 2, 1, 64)
     if where == "h":
         inputs["w_gate_up"] = (inputs["w_gate_up"].float() * 3000.0).to(torch.bfloat16)
-    else:   # down weights of about 2000: finite in fp16, outputs far beyond 65504
+    else:   # activated rows of tens, down weights of about 2000 (both finite in fp16):
+            # outputs far beyond 65504
+        inputs["w_gate_up"] = (inputs["w_gate_up"].float() * 30.0).to(torch.bfloat16)
         for n in ("w_down", "ws_down"):
             inputs[n] = (inputs[n].float() * 1e5).clamp(-6e4, 6e4).to(torch.bfloat16)
     L = moe.Layer.from_workload(w, down_f16=True)
