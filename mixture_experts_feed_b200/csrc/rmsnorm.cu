@@ -15,7 +15,8 @@
 // rmsnorm_rows_kernel: a team of TPR threads (32..256, one to eight warps)
 // per row, each thread holding up to four 16-byte vectors of its row in
 // registers.  Every vector of the row is loaded at once (one HBM read per
-// element, all of a row's loads in flight together), each thread adds its
+// element, all of a row's loads in flight together, and the next row's
+// issued before this row's reduction), each thread adds its
 // squares into fp64 partials per element position, the warps reduce by a
 // butterfly and the row's warps' sums are added in warp order through shared
 // memory (a fixed order: the same sum on every run), and the thread scales
@@ -92,6 +93,16 @@ struct Bf16Row {
       acc[2 * i + 1] = fma(b, b, acc[2 * i + 1]);
     }
   }
+  // acc[i & 1] += square of element i
+  __device__ static void sumsq2(const Vec& q, double (&acc)[2]) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const double a = __uint_as_float(w[i] << 16), b = __uint_as_float(w[i] & 0xFFFF0000u);
+      acc[0] = fma(a, a, acc[0]);
+      acc[1] = fma(b, b, acc[1]);
+    }
+  }
   // bf16 bits of p * inv (p = x * weight, exact in fp32)
   __device__ static uint32_t one(float p, float inv32, double inv) {
     const float y32 = p * inv32;
@@ -123,6 +134,12 @@ struct F32Row {
     acc[1] = fma(static_cast<double>(q.y), q.y, acc[1]);
     acc[2] = fma(static_cast<double>(q.z), q.z, acc[2]);
     acc[3] = fma(static_cast<double>(q.w), q.w, acc[3]);
+  }
+  __device__ static void sumsq2(const Vec& q, double (&acc)[2]) {
+    acc[0] = fma(static_cast<double>(q.x), q.x, acc[0]);
+    acc[1] = fma(static_cast<double>(q.y), q.y, acc[1]);
+    acc[0] = fma(static_cast<double>(q.z), q.z, acc[0]);
+    acc[1] = fma(static_cast<double>(q.w), q.w, acc[1]);
   }
   __device__ static Vec scale(const Vec& q, const Vec& g, float, double inv) {
     return make_float4(__double2float_rn(static_cast<double>(q.x) * g.x * inv),
@@ -184,9 +201,11 @@ __global__ void __launch_bounds__(kThreads)
 
 // Row-resident variant: TPR = 1 << tpr_log2 threads per row (32..256), each
 // holding VPT vectors; 256 / TPR rows per block.  The loop over row groups
-// is uniform across the block (every thread reaches every barrier).
+// is uniform across the block (every thread reaches every barrier).  The
+// next row group's vectors are loaded before the current group's block
+// reduction, so that each block keeps two rows' loads in flight.
 template <typename R, int VPT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)
     rmsnorm_rows_kernel(const void* x_, const void* __restrict__ w_, void* out_, int64_t T, int H,
                         double eps, int tpr_log2) {
   using Vec = typename R::Vec;
@@ -202,28 +221,33 @@ __global__ void __launch_bounds__(kThreads)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int wpr = tpr >> 5;                              // warps per row
   const int first_warp = r_in_b * wpr;
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * rpb; base < T;
-       base += static_cast<int64_t>(gridDim.x) * rpb) {
+  const int64_t step = static_cast<int64_t>(gridDim.x) * rpb;
+  auto load_row = [&](int64_t t, Vec (&buf)[VPT]) {
+    if (t >= T) return;
+    const Vec* row = x + t * nv;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = t_in_r + j * tpr;
+      if (v < nv) buf[j] = row[v];
+    }
+  };
+  Vec buf[VPT];
+  int64_t base = static_cast<int64_t>(blockIdx.x) * rpb;
+  load_row(base + r_in_b, buf);
+  for (; base < T; base += step) {
     const int64_t t = base + r_in_b;
     const bool live = t < T;
-    const Vec* row = x + (live ? t : 0) * nv;
-    Vec buf[VPT];
+    Vec nxt[VPT];
+    load_row(base + step + r_in_b, nxt);                 // in flight during this row's reduction
+    // two fp64 partial sums a thread (element positions even / odd), added
+    // in a fixed order
+    double part[2] = {0.0, 0.0};
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
       const int v = t_in_r + j * tpr;
-      if (live && v < nv) buf[j] = row[v];
+      if (live && v < nv) R::sumsq2(buf[j], part);
     }
-    double part[R::V];
-#pragma unroll
-    for (int i = 0; i < R::V; ++i) part[i] = 0.0;
-#pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-      const int v = t_in_r + j * tpr;
-      if (live && v < nv) R::sumsq(buf[j], part);
-    }
-    double acc = 0.0;
-#pragma unroll
-    for (int i = 0; i < R::V; ++i) acc += part[i];
+    double acc = part[0] + part[1];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) s_part[warp] = acc;
@@ -241,6 +265,8 @@ __global__ void __launch_bounds__(kThreads)
         if (v < nv) orow[v] = R::scale(buf[j], w[v], inv32, inv);
       }
     }
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) buf[j] = nxt[j];
   }
 }
 
@@ -256,7 +282,7 @@ cudaError_t launch_rows(int64_t T, int H, double eps, const void* x, const void*
   const int vpt = (nv + tpr - 1) / tpr;
   const int rpb = kThreads / tpr;
   const int64_t blocks = (T + rpb - 1) / rpb;
-  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(blocks, static_cast<int64_t>(num_sms) * 8));
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(blocks, static_cast<int64_t>(num_sms) * 4));
   switch (vpt) {
     case 1: rmsnorm_rows_kernel<R, 1><<<grid, kThreads, 0, stream>>>(x, weight, out, T, H, eps, tpr_log2); break;
     case 2: rmsnorm_rows_kernel<R, 2><<<grid, kThreads, 0, stream>>>(x, weight, out, T, H, eps, tpr_log2); break;
