@@ -551,11 +551,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * 32), v);
           tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 1) * 32), v2);
           tmem_ld_wait();
+          bool ovf = false;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            pk[i] = pack_f16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]), h_overflow);
-            pk[16 + i] = pack_f16x2(__uint_as_float(v2[2 * i]), __uint_as_float(v2[2 * i + 1]), h_overflow);
+            pk[i] = pack_f16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]), ovf);
+            pk[16 + i] = pack_f16x2(__uint_as_float(v2[2 * i]), __uint_as_float(v2[2 * i + 1]), ovf);
           }
+          // only rows of the group count: rows past its end hold whatever the
+          // A operand's rows beyond the group held, and are never stored
+          if (valid && ovf) h_overflow = true;
           if (lane == 0) bulk_wait_group_read0();
           __syncwarp();
           if (rows_left >= 32) {

@@ -131,6 +131,7 @@ class ExpertParallelMoE:
         self.down_f16 = self.w["w_down"].dtype == torch.float16   # fp16 down projections
         self.route_scale, self.global_scale = route_scale, global_scale
         self.last_counts = None       # (rows sent per destination, rows received per source)
+        self._ws = []                 # the workspaces of the last call (status words)
 
     def layer(self, T: int) -> Layer:
         return self.ops.Layer(T, self.H, self.E, self.k, self.S, self.I, self.dtype,
@@ -195,9 +196,11 @@ class ExpertParallelMoE:
                             self.global_scale, self.down_f16)
         y_dtype = torch.float16 if self.down_f16 else torch.float32   # the expert output rows
         y_in = torch.empty(R_in, H, dtype=y_dtype, device=dev)
+        self._ws = [ws]
         if R_in > 0:
             off_loc = torch.tensor(loc_off, dtype=torch.int32).to(dev)
             ws_loc = ops.new_workspace(Ll, device=dev)
+            self._ws.append(ws_loc)
             ops.moe_expert_ffn(Ll, x_in, x_in, off_loc, None, w_in, None, w["w_gate_up"],
                                w["w_down"], None, None, y_in, None, ws_loc)
         # 6: the output rows back into this rank's permuted order
@@ -222,6 +225,16 @@ class ExpertParallelMoE:
         out = torch.empty(T, H, dtype=self.dtype, device=dev)
         ops.moe_combine(L, yr, ys, ip, out, ws)
         return out
+
+
+def read_device_status(layer: "ExpertParallelMoE") -> int:
+    """Read and clear the status words of the workspaces of the layer's last
+    call (raises the binding's MoEError when a kernel recorded a problem)."""
+    from . import read_device_status as _read
+    code = 0
+    for ws in layer._ws:
+        code = code or _read(ws)
+    return code
 
 
 def _exclusive_scan(v: Sequence[int]) -> List[int]:

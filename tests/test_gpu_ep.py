@@ -24,7 +24,7 @@ pytestmark = pytest.mark.gpu
 
 
 def run_ranks(inputs, world, T_rank, E, k, S, route_scale, pm=None):
-    from mixture_experts_feed_b200.ep import ExpertParallelMoE
+    from mixture_experts_feed_b200.ep import ExpertParallelMoE, read_device_status
     shared = LoopbackComm(world)
     outs, counts, errs = [None] * world, [None] * world, []
 
@@ -37,6 +37,7 @@ def run_ranks(inputs, world, T_rank, E, k, S, route_scale, pm=None):
             m = None if pm is None else pm[r * T_rank:(r + 1) * T_rank]
             o = layer(x, padding_mask=m)
             torch.cuda.synchronize()
+            assert read_device_status(layer) == 0
             outs[r], counts[r] = o.cpu(), layer.last_counts
         except BaseException as e:    # noqa: BLE001 - reported below
             errs.append((r, e))

@@ -567,3 +567,21 @@ def test_fp16_overflow_is_reported(where):
     with pytest.raises(moe.MoEError) as ei:
         moe.read_device_status(ws)
     assert ei.value.device_code == 0x103
+
+
+@pytest.mark.parametrize("shape", [(300, 256, 12, 3, 2, 320, "bf16"), (1100, 256, 16, 2, 1, 128, "bf16")],
+                         ids=["T300", "T1100"])
+def test_stale_workspace_is_harmless(shape):
+    """A workspace whose every byte is 0xFF (NaN in bf16 and fp16) before the
+    call: the rows past each group's end that the tiles load from it are
+    never stored and raise no overflow flag; the outputs equal those computed
+    with a zeroed workspace, bit for bit (fp16 down projections)."""
+    w, inputs = small_case(*shape)
+    L = moe.Layer.from_workload(w, down_f16=True)
+    d = to_device(inputs, down_f16=True)
+    outs = []
+    for fill in (0x00, 0xFF):
+        ws = torch.full((moe.workspace_size(L),), fill, dtype=torch.uint8, device="cuda")
+        moe.LIB.moe_workspace_init(ws.data_ptr(), ws.numel(), None)
+        outs.append(run_forward(L, d, ws=ws)["out"])      # asserts a clean status word
+    assert torch.equal(outs[0], outs[1])
