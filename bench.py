@@ -275,7 +275,27 @@ def step_bytes(w, touched: int, yel: int = 4) -> int:
     return expert_ffn_bytes(w, touched, yel) + router + permute + combine
 
 
-def gemm_roofline(w, ffn_ms: float, touched: int, peaks, peak_src: str, yel: int = 4):
+def groupwise_bound_ms(w, counts, peaks, yel: int = 4) -> float:
+    """The expert GEMMs' floor group by group: each group (routed expert with
+    rows, every shared expert) takes at least max(its flops / the burst bf16
+    peak, its bytes / the measured HBM bandwidth), with bytes its weights
+    once plus, per row, the A row, h written and read and the down row
+    written.  Groups with few rows are bound by their weights' bytes, so this
+    floor lies above the aggregate flop floor."""
+    P = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])) * 1e12
+    BW = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])) * 1e9
+    el = 2 if w.dtype == "bf16" else 4
+    t = 0.0
+    for r in list(counts) + [w.T] * w.S:
+        if r > 0:
+            fl = 6.0 * r * w.H * w.I
+            by = 3 * w.H * w.I * el + r * (w.H * el + 2 * w.I * el + yel * w.H)
+            t += max(fl / P, by / BW)
+    return t * 1e3
+
+
+def gemm_roofline(w, ffn_ms: float, touched: int, peaks, peak_src: str, yel: int = 4,
+                  counts=None):
     """Roofline of the expert GEMMs (the four launches of moe_expert_ffn):
     tensor-bound against the measured burst bf16 peak (the calls are timed in
     a region of well under a second), or HBM-bound against the measured copy
@@ -299,6 +319,10 @@ def gemm_roofline(w, ffn_ms: float, touched: int, peaks, peak_src: str, yel: int
     roof["algorithmic_bytes"] = ffn_bytes
     roof["algorithmic_flops"] = ffn_flops
     roof["touched_groups"] = touched
+    if counts is not None:
+        gb = groupwise_bound_ms(w, counts, peaks, yel)
+        roof["groupwise_bound_ms"] = gb
+        roof["frac_of_groupwise_bound"] = gb / ffn_ms
     return roof
 
 
@@ -385,7 +409,7 @@ def time_workload(moe, name: str, steps: int, warmup: int, dev, stream, peaks, p
     counts = (off[1:] - off[:-1]).cpu()
     touched = int((counts > 0).sum()) + S
     yel = 2 if L.down_f16 else 4
-    roof = gemm_roofline(w, op_ms[2], touched, peaks, peak_src, yel)
+    roof = gemm_roofline(w, op_ms[2], touched, peaks, peak_src, yel, counts.tolist())
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     sb = step_bytes(w, touched, yel)
     res = {"ms_per_step": ms, "tokens_per_s": T / (ms / 1e3),
@@ -597,7 +621,7 @@ def gpu_arm(args, world, rank, local):
         counts = (off[1:] - off[:-1]).cpu()
         touched = int((counts > 0).sum()) + S
         yel = 2 if L.down_f16 else 4
-        roof = gemm_roofline(w, ffn_ms, touched, peaks, peak_src, yel)
+        roof = gemm_roofline(w, ffn_ms, touched, peaks, peak_src, yel, counts.tolist())
         # the captured bytes are those of the launches reading x_perm; the
         # row-gathering mode reads x instead and has no capture
         traffic, traffic_src = traffic_of(w.name)

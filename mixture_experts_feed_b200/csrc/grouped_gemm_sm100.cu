@@ -6,14 +6,16 @@
 //   kGateUp: the accumulator columns interleave gate and up channels
 //            ([g0, u0, g1, u1, ...], the fused gate_up_proj layout of the
 //            Inkling layers page, inkling_swiglu); the epilogue writes
-//            h = w * silu(g) * u in bf16, w the row's routing weight (routed
+//            h = w * silu(g) * u in bf16, or in fp16 when the down
+//            projection runs in fp16, w the row's routing weight (routed
 //            rows: topk_w of the row's slot; shared rows: the token's gamma,
 //            or one uniform weight when no gamma is given: the dense layer,
 //            run as a single shared group, passes its global_scale).
-//   kDown:   the epilogue writes D in fp32 (the down projection); the rows
-//            stay fp32 until the recombination rounds the layer output once
-//            (rounding them to bf16 as well would put a correct pipeline at
-//            about 2% of the output RMS, the edge of the 2e-2 bound).
+//   kDown:   bf16 x bf16, or fp16 x fp16 (fp16 h against an fp16 copy of the
+//            weights); the epilogue writes D in fp32, or fp16 with fp16
+//            operands, and the recombination sums the rows in fp32 and
+//            rounds the layer output once (bf16 rows would put a correctly
+//            rounded pipeline beyond the 2e-2 x RMS bound).
 //   kRouter: router logits z = x @ Wr^T, the fp32 router bank split exactly
 //            into three bf16 parts (W = W0 + W1 + W2) so that every product
 //            is exact.  The tensor-core accumulator loses about one fp32 ulp
