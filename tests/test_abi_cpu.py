@@ -251,3 +251,30 @@ def test_ep_partition():
     assert partition(128, 8, 3) == (48, 16)
     with pytest.raises(ValueError):
         partition(10, 4, 0)
+
+
+def test_convert_host_checks():
+    """moe_convert_bf16_to_f16: n a multiple of 8, both buffers present and
+    16-byte aligned; n = 0 does nothing."""
+    fake = 1 << 20
+    assert moe.LIB.moe_convert_bf16_to_f16(12, fake, fake, None, None) == 1       # n % 8
+    assert moe.LIB.moe_convert_bf16_to_f16(-8, fake, fake, None, None) == 1
+    assert moe.LIB.moe_convert_bf16_to_f16(16, None, fake, None, None) == 1
+    assert moe.LIB.moe_convert_bf16_to_f16(16, fake, fake + 2, None, None) == 1   # misaligned
+    assert moe.LIB.moe_convert_bf16_to_f16(0, None, None, None, None) == 0
+
+
+def test_layer_codes():
+    """The binding's layer dtypes map onto moe_dtype_t; fp16 down projections
+    exist for bf16 layers only."""
+    assert moe.Layer(4, 64, 4, 1, 0, 64, torch.bfloat16).desc().dtype == moe.MOE_BF16
+    assert moe.Layer(4, 64, 4, 1, 0, 64, torch.bfloat16, down_f16=True).desc().dtype == moe.MOE_BF16_F16DOWN
+    assert moe.Layer(4, 64, 4, 1, 0, 64, torch.float32).desc().dtype == moe.MOE_F32
+    with pytest.raises(ValueError):
+        moe.Layer(4, 64, 4, 1, 0, 64, torch.float32, down_f16=True).desc()
+    L = moe.Layer(4, 64, 4, 1, 0, 64, torch.bfloat16, down_f16=True)
+    assert L.down_dtype == torch.float16 and L.y_dtype == torch.float16
+    # the workspace of a fp16-down layer holds fp16 expert rows: smaller
+    Lb = moe.Layer(512, 256, 8, 2, 1, 128, torch.bfloat16)
+    Lf = moe.Layer(512, 256, 8, 2, 1, 128, torch.bfloat16, down_f16=True)
+    assert moe.workspace_size(Lf) < moe.workspace_size(Lb)
