@@ -33,19 +33,6 @@ __device__ __forceinline__ void add_vec(float (&acc)[V], const float* p) {
   }
 }
 
-// acc[0..8) += 8 consecutive fp16 values (one 16-byte load), each widened
-// exactly to fp32
-__device__ __forceinline__ void add_vec(float (&acc)[8], const __half* p) {
-  const uint4 q = __ldcs(reinterpret_cast<const uint4*>(p));
-  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
-    acc[2 * i] += f.x;
-    acc[2 * i + 1] += f.y;
-  }
-}
-
 __device__ __forceinline__ void store_vec(__nv_bfloat16* p, const float (&acc)[8]) {
   uint4 q;
   q.x = pack_bf16x2(acc[0], acc[1]);
@@ -59,7 +46,7 @@ __device__ __forceinline__ void store_vec(float* p, const float (&acc)[4]) {
   *reinterpret_cast<float4*>(p) = make_float4(acc[0], acc[1], acc[2], acc[3]);
 }
 
-// TY: output dtype; TR: expert row dtype (fp32, or fp16 with bf16 output)
+// TY: output dtype; TR: expert row dtype (fp32)
 template <typename TY, typename TR>
 __global__ void __launch_bounds__(256)
     combine_kernel(const TR* __restrict__ y_routed, const TR* __restrict__ y_shared,
@@ -94,6 +81,77 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// fp16 rows into bf16 output: the same sums in the same order, with more of
+// each thread's loads in flight (a row segment of 8 fp16 values is 16 bytes,
+// half of the fp32 kernel's): each thread takes two vectors, and the rows
+// are loaded in batches of 8 before they are added.
+constexpr int kRowBatch = 8;
+__global__ void __launch_bounds__(256)
+    combine_f16rows_kernel(const __half* __restrict__ y_routed, const __half* __restrict__ y_shared,
+                           const int32_t* __restrict__ inv_perm, __nv_bfloat16* __restrict__ out,
+                           int64_t T, int H, int k, int S, int64_t rows_cap, int32_t* status) {
+  __shared__ const __half* s_src[32];   // the token's rows: S shared, then k routed (or null)
+  const int nv = H / 8;
+  const int n = S + k;
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    if (threadIdx.x < n) {
+      const int i = threadIdx.x;
+      const __half* src = nullptr;
+      if (i < S) {
+        src = y_shared + (static_cast<int64_t>(i) * T + t) * H;
+      } else {
+        int r = inv_perm[t * k + (i - S)];
+        if (r >= rows_cap) {
+          record_status(status, DEV_BAD_ROW);
+          r = -1;
+        }
+        if (r >= 0) src = y_routed + static_cast<int64_t>(r) * H;
+      }
+      s_src[i] = src;
+    }
+    __syncthreads();
+    for (int v = threadIdx.x; v < nv; v += 2 * blockDim.x) {
+      const int v2 = v + blockDim.x;
+      const bool two = v2 < nv;
+      float acc[8], acc2[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = acc2[i] = 0.0f;
+      for (int i0 = 0; i0 < n; i0 += kRowBatch) {
+        uint4 q[kRowBatch], q2[kRowBatch];
+#pragma unroll
+        for (int u = 0; u < kRowBatch; ++u) {
+          const __half* src = i0 + u < n ? s_src[i0 + u] : nullptr;
+          if (src != nullptr) {
+            q[u] = __ldcs(reinterpret_cast<const uint4*>(src) + v);
+            if (two) q2[u] = __ldcs(reinterpret_cast<const uint4*>(src) + v2);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kRowBatch; ++u) {
+          if (i0 + u < n && s_src[i0 + u] != nullptr) {   // rows in order; skipped rows add nothing
+            const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+            const uint32_t w2[4] = {q2[u].x, q2[u].y, q2[u].z, q2[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
+              acc[2 * e] += f.x;
+              acc[2 * e + 1] += f.y;
+              if (two) {
+                const float2 g = __half22float2(*reinterpret_cast<const __half2*>(&w2[e]));
+                acc2[2 * e] += g.x;
+                acc2[2 * e + 1] += g.y;
+              }
+            }
+          }
+        }
+      }
+      store_vec(out + t * H + static_cast<int64_t>(v) * 8, acc);
+      if (two) store_vec(out + t * H + static_cast<int64_t>(v2) * 8, acc2);
+    }
+    __syncthreads();
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_combine(const Layer& L, const void* y_routed, const void* y_shared,
@@ -103,7 +161,7 @@ cudaError_t launch_combine(const Layer& L, const void* y_routed, const void* y_s
       static_cast<unsigned>(std::min<int64_t>(L.T, static_cast<int64_t>(num_sms) * 8));
   const int64_t cap = L.T * L.k;
   if (L.dtype == MOE_BF16 && L.y_f16)
-    combine_kernel<__nv_bfloat16, __half><<<grid, 256, 0, stream>>>(
+    combine_f16rows_kernel<<<grid, 256, 0, stream>>>(
         static_cast<const __half*>(y_routed), static_cast<const __half*>(y_shared), inv_perm,
         static_cast<__nv_bfloat16*>(out), L.T, L.H, L.k, L.S, cap, status);
   else if (L.dtype == MOE_BF16)
