@@ -50,15 +50,15 @@ import moe_workloads as mw  # noqa: E402
 METRIC = "Inkling MoE-layer tokens/s and TFLOP/s (% of B200 bf16 peak / % HBM BW), 1 GPU"
 DEFAULT_WORKLOAD = "bf16-T8192-H6144-E128k8S1-I2048"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes of the expert GEMMs of one step (the routed experts' four
-# grouped-GEMM launches and the shared experts' two) on these workloads: ncu
-# dram__bytes_read.sum + dram__bytes_write.sum, one pass, summed over the
-# launches.  A capture constant, not a
+# DRAM bytes of one moe_expert_ffn call (its four grouped-GEMM launches) on
+# these workloads: ncu dram__bytes_read.sum + dram__bytes_write.sum, one pass,
+# summed over the launches.  A capture constant, not a
 # measurement of this run: each entry names its capture.  An entry is removed
 # when the kernels change, until it is captured again.
 NCU_TRAFFIC_BYTES = {
-    "bf16-T8192-H6144-E128k8S1-I2048": (16286890496, "ncu capture of 2026-12-03 (the six expert-GEMM "
-                                        "launches of one moe_forward step, fp16 down projections), "
+    "bf16-T8192-H6144-E128k8S1-I2048": (18046190848, "ncu capture of 2026-12-03 (the four launches of "
+                                        "one moe_expert_ffn call of the op chain, fp16 down "
+                                        "projections; box-to-box spread 13-18 GB), "
                                         "profiles/traffic_expert_gemms_bf16-T8192-H6144-E128k8S1-I2048.md"),
 }
 # The other workloads the benchmark spec states, timed in the same run as the default
