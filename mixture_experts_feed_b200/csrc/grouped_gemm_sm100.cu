@@ -25,7 +25,9 @@
 //            epilogue warps add the chain sums in fp32 registers with
 //            round-to-nearest adds.  fp32 logits out.  One group (all T
 //            tokens), N = E + S, 160-column tiles (E + S = 129 in one tile,
-//            257 in two).
+//            257 in two).  The parts run chunk by chunk over K (part 2, 1, 0
+//            of one 1024-deep chunk, then the next), so the three reads of
+//            an x block come from L2.
 //
 // The expert modes run on CTA pairs (clusters of two SMs, tcgen05
 // cta_group::2): a pair computes a 256-row x 256-column tile with M=256
@@ -70,6 +72,23 @@ constexpr int A_BYTES = BM * BK * 2;
 constexpr int NUM_THREADS = 192;
 // kRouter: K blocks per tensor-core accumulation chain (128-deep chains)
 constexpr int ROUTER_CHAIN = 2;
+// kRouter: K blocks per chunk.  The three weight parts run chunk by chunk
+// (part 2, 1, 0 over one chunk of K, then the next chunk), so each CTA reads
+// a 128 x 1024 block of x three times while it is still in L2 instead of
+// streaming x from HBM once per part.
+constexpr int ROUTER_CHUNK = 16;
+
+// kRouter: the K block and weight part of step kt of a CTA's 3 * k_blocks
+// steps (chunk-major; a last, shorter chunk when k_blocks is not a multiple
+// of ROUTER_CHUNK).
+__device__ __forceinline__ void router_step(int kt, int k_blocks, int& kb, int& part) {
+  const int full = k_blocks / ROUTER_CHUNK;
+  const int c = kt / (3 * ROUTER_CHUNK);
+  const int size = c < full ? ROUTER_CHUNK : k_blocks - full * ROUTER_CHUNK;
+  const int r = kt - c * 3 * ROUTER_CHUNK;
+  part = 2 - r / size;
+  kb = c * ROUTER_CHUNK + r % size;
+}
 
 enum Mode { kGateUp = 0, kDown = 1, kRouter = 2 };
 
@@ -340,9 +359,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int got = 1;
         if (lane == 0) got = mbar_wait(&empty[stage], phase ^ 1u, s_abort, p.status) ? 1 : 0;
         if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
-        // router: part 2 (smallest) first, then 1, then 0
-        const int kb = MODE == kRouter ? kt % k_blocks : kt;
-        const int slice = MODE == kRouter ? 2 - kt / k_blocks : gi.b_idx;
+        // router: per chunk of K, part 2 (smallest) first, then 1, then 0
+        int kb = kt, slice = gi.b_idx;
+        if (MODE == kRouter) router_step(kt, k_blocks, kb, slice);
         uint8_t* a_dst = stage_a(stage);
         if (PAIR) {
           // both CTAs' bytes complete on the rank-0 CTA's barrier
