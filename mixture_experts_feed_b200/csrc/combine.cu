@@ -81,73 +81,78 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// fp16 rows into bf16 output: the same sums in the same order, with more of
-// each thread's loads in flight (a row segment of 8 fp16 values is 16 bytes,
-// half of the fp32 kernel's): each thread takes two vectors, and the rows
-// are loaded in batches of 8 before they are added.
-constexpr int kRowBatch = 8;
+// fp16 rows into bf16 output: the same sums in the same order.  Each thread
+// takes VPT vectors of 8 values (VPT * blockDim vectors per pass; one pass
+// for H <= VPT * 2048), so a thread keeps VPT * kRowBatch 16-byte loads in
+// flight, and the next token's row pointers are read while the current
+// token is summed, so no dependent index load stalls the block between
+// tokens.  Four rows a batch keep registers for two blocks an SM.
+constexpr int kRowBatch = 4;
+template <int VPT>
 __global__ void __launch_bounds__(256)
     combine_f16rows_kernel(const __half* __restrict__ y_routed, const __half* __restrict__ y_shared,
                            const int32_t* __restrict__ inv_perm, __nv_bfloat16* __restrict__ out,
                            int64_t T, int H, int k, int S, int64_t rows_cap, int32_t* status) {
-  __shared__ const __half* s_src[32];   // the token's rows: S shared, then k routed (or null)
+  __shared__ const __half* s_src[2][32];   // a token's rows: S shared, then k routed (or null)
   const int nv = H / 8;
   const int n = S + k;
-  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-    if (threadIdx.x < n) {
-      const int i = threadIdx.x;
-      const __half* src = nullptr;
-      if (i < S) {
-        src = y_shared + (static_cast<int64_t>(i) * T + t) * H;
-      } else {
-        int r = inv_perm[t * k + (i - S)];
-        if (r >= rows_cap) {
-          record_status(status, DEV_BAD_ROW);
-          r = -1;
-        }
-        if (r >= 0) src = y_routed + static_cast<int64_t>(r) * H;
-      }
-      s_src[i] = src;
+  auto row_of = [&](int64_t t, int i) -> const __half* {
+    if (i < S) return y_shared + (static_cast<int64_t>(i) * T + t) * H;
+    int r = inv_perm[t * k + (i - S)];
+    if (r >= rows_cap) {
+      record_status(status, DEV_BAD_ROW);
+      r = -1;
     }
-    __syncthreads();
-    for (int v = threadIdx.x; v < nv; v += 2 * blockDim.x) {
-      const int v2 = v + blockDim.x;
-      const bool two = v2 < nv;
-      float acc[8], acc2[8];
+    return r >= 0 ? y_routed + static_cast<int64_t>(r) * H : nullptr;
+  };
+  int buf = 0;
+  if (threadIdx.x < n && blockIdx.x < T) s_src[0][threadIdx.x] = row_of(blockIdx.x, threadIdx.x);
+  __syncthreads();
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    const int64_t tn = t + gridDim.x;
+    const __half* nxt = nullptr;   // this thread's row of the next token
+    if (threadIdx.x < n && tn < T) nxt = row_of(tn, threadIdx.x);
+    for (int base = 0; base < nv; base += VPT * blockDim.x) {
+      float acc[VPT][8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = acc2[i] = 0.0f;
+      for (int j = 0; j < VPT; ++j)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[j][i] = 0.0f;
       for (int i0 = 0; i0 < n; i0 += kRowBatch) {
-        uint4 q[kRowBatch], q2[kRowBatch];
+        uint4 q[kRowBatch][VPT];
 #pragma unroll
         for (int u = 0; u < kRowBatch; ++u) {
-          const __half* src = i0 + u < n ? s_src[i0 + u] : nullptr;
-          if (src != nullptr) {
-            q[u] = __ldcs(reinterpret_cast<const uint4*>(src) + v);
-            if (two) q2[u] = __ldcs(reinterpret_cast<const uint4*>(src) + v2);
+          const __half* src = i0 + u < n ? s_src[buf][i0 + u] : nullptr;
+#pragma unroll
+          for (int j = 0; j < VPT; ++j) {
+            const int v = base + threadIdx.x + j * blockDim.x;
+            if (src != nullptr && v < nv) q[u][j] = __ldcs(reinterpret_cast<const uint4*>(src) + v);
           }
         }
 #pragma unroll
         for (int u = 0; u < kRowBatch; ++u) {
-          if (i0 + u < n && s_src[i0 + u] != nullptr) {   // rows in order; skipped rows add nothing
-            const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
-            const uint32_t w2[4] = {q2[u].x, q2[u].y, q2[u].z, q2[u].w};
+          if (i0 + u < n && s_src[buf][i0 + u] != nullptr) {   // rows in order; skipped rows add nothing
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
-              acc[2 * e] += f.x;
-              acc[2 * e + 1] += f.y;
-              if (two) {
-                const float2 g = __half22float2(*reinterpret_cast<const __half2*>(&w2[e]));
-                acc2[2 * e] += g.x;
-                acc2[2 * e + 1] += g.y;
+            for (int j = 0; j < VPT; ++j) {
+              const uint32_t w[4] = {q[u][j].x, q[u][j].y, q[u][j].z, q[u][j].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
+                acc[j][2 * e] += f.x;
+                acc[j][2 * e + 1] += f.y;
               }
             }
           }
         }
       }
-      store_vec(out + t * H + static_cast<int64_t>(v) * 8, acc);
-      if (two) store_vec(out + t * H + static_cast<int64_t>(v2) * 8, acc2);
+#pragma unroll
+      for (int j = 0; j < VPT; ++j) {
+        const int v = base + threadIdx.x + j * blockDim.x;
+        if (v < nv) store_vec(out + t * H + static_cast<int64_t>(v) * 8, acc[j]);
+      }
     }
+    if (threadIdx.x < n) s_src[buf ^ 1][threadIdx.x] = nxt;
+    buf ^= 1;
     __syncthreads();
   }
 }
@@ -160,11 +165,22 @@ cudaError_t launch_combine(const Layer& L, const void* y_routed, const void* y_s
   const unsigned grid =
       static_cast<unsigned>(std::min<int64_t>(L.T, static_cast<int64_t>(num_sms) * 8));
   const int64_t cap = L.T * L.k;
-  if (L.dtype == MOE_BF16 && L.y_f16)
-    combine_f16rows_kernel<<<grid, 256, 0, stream>>>(
-        static_cast<const __half*>(y_routed), static_cast<const __half*>(y_shared), inv_perm,
-        static_cast<__nv_bfloat16*>(out), L.T, L.H, L.k, L.S, cap, status);
-  else if (L.dtype == MOE_BF16)
+  if (L.dtype == MOE_BF16 && L.y_f16) {
+    // vectors a thread: the fewest that cover the row in one pass of 256
+    // threads, at most 4 (longer rows take several passes)
+    const int nv = L.H / 8;
+    const auto* yr = static_cast<const __half*>(y_routed);
+    const auto* ys = static_cast<const __half*>(y_shared);
+    auto* o = static_cast<__nv_bfloat16*>(out);
+    if (nv <= 256)
+      combine_f16rows_kernel<1><<<grid, 256, 0, stream>>>(yr, ys, inv_perm, o, L.T, L.H, L.k, L.S, cap, status);
+    else if (nv <= 512)
+      combine_f16rows_kernel<2><<<grid, 256, 0, stream>>>(yr, ys, inv_perm, o, L.T, L.H, L.k, L.S, cap, status);
+    else if (nv <= 768)
+      combine_f16rows_kernel<3><<<grid, 256, 0, stream>>>(yr, ys, inv_perm, o, L.T, L.H, L.k, L.S, cap, status);
+    else
+      combine_f16rows_kernel<4><<<grid, 256, 0, stream>>>(yr, ys, inv_perm, o, L.T, L.H, L.k, L.S, cap, status);
+  } else if (L.dtype == MOE_BF16)
     combine_kernel<__nv_bfloat16, float><<<grid, 256, 0, stream>>>(
         static_cast<const float*>(y_routed), static_cast<const float*>(y_shared), inv_perm,
         static_cast<__nv_bfloat16*>(out), L.T, L.H, L.k, L.S, cap, status);
