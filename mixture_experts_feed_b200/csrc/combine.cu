@@ -81,22 +81,24 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// fp16 rows into bf16 output: the same sums in the same order.  Each thread
-// takes VPT vectors of 8 values (VPT * blockDim vectors per pass; one pass
-// for H <= VPT * 2048), so a thread keeps VPT * kRowBatch 16-byte loads in
-// flight, and the next token's row pointers are read while the current
-// token is summed, so no dependent index load stalls the block between
-// tokens.  Four rows a batch keep registers for two blocks an SM.
-constexpr int kRowBatch = 4;
-template <int VPT>
+// Rows of TR (fp16, or fp32) into bf16 output: the same sums in the same
+// order.  A vector is 8 values (one 16-byte load of fp16, two of fp32); each
+// thread takes VPT vectors (VPT * blockDim vectors per pass; one pass for
+// H <= VPT * 2048), so it keeps VPT * kRowBatch vectors of loads in flight,
+// and the next token's row pointers are read while the current token is
+// summed, so no dependent index load stalls the block between tokens.  The
+// row batch (4 fp16 rows, 2 fp32 rows) keeps registers for two blocks an SM.
+template <typename TR, int VPT>
 __global__ void __launch_bounds__(256)
-    combine_f16rows_kernel(const __half* __restrict__ y_routed, const __half* __restrict__ y_shared,
-                           const int32_t* __restrict__ inv_perm, __nv_bfloat16* __restrict__ out,
-                           int64_t T, int H, int k, int S, int64_t rows_cap, int32_t* status) {
-  __shared__ const __half* s_src[2][32];   // a token's rows: S shared, then k routed (or null)
+    combine_rows_kernel(const TR* __restrict__ y_routed, const TR* __restrict__ y_shared,
+                        const int32_t* __restrict__ inv_perm, __nv_bfloat16* __restrict__ out,
+                        int64_t T, int H, int k, int S, int64_t rows_cap, int32_t* status) {
+  constexpr int kRowBatch = sizeof(TR) == 2 ? 4 : 2;
+  constexpr int LPV = sizeof(TR) == 2 ? 1 : 2;   // 16-byte loads per vector of 8 values
+  __shared__ const TR* s_src[2][32];   // a token's rows: S shared, then k routed (or null)
   const int nv = H / 8;
   const int n = S + k;
-  auto row_of = [&](int64_t t, int i) -> const __half* {
+  auto row_of = [&](int64_t t, int i) -> const TR* {
     if (i < S) return y_shared + (static_cast<int64_t>(i) * T + t) * H;
     int r = inv_perm[t * k + (i - S)];
     if (r >= rows_cap) {
@@ -110,7 +112,7 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
     const int64_t tn = t + gridDim.x;
-    const __half* nxt = nullptr;   // this thread's row of the next token
+    const TR* nxt = nullptr;   // this thread's row of the next token
     if (threadIdx.x < n && tn < T) nxt = row_of(tn, threadIdx.x);
     for (int base = 0; base < nv; base += VPT * blockDim.x) {
       float acc[VPT][8];
@@ -119,14 +121,18 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[j][i] = 0.0f;
       for (int i0 = 0; i0 < n; i0 += kRowBatch) {
-        uint4 q[kRowBatch][VPT];
+        uint4 q[kRowBatch][VPT][LPV];
 #pragma unroll
         for (int u = 0; u < kRowBatch; ++u) {
-          const __half* src = i0 + u < n ? s_src[buf][i0 + u] : nullptr;
+          const TR* src = i0 + u < n ? s_src[buf][i0 + u] : nullptr;
 #pragma unroll
           for (int j = 0; j < VPT; ++j) {
             const int v = base + threadIdx.x + j * blockDim.x;
-            if (src != nullptr && v < nv) q[u][j] = __ldcs(reinterpret_cast<const uint4*>(src) + v);
+            if (src != nullptr && v < nv) {
+#pragma unroll
+              for (int l = 0; l < LPV; ++l)
+                q[u][j][l] = __ldcs(reinterpret_cast<const uint4*>(src) + static_cast<int64_t>(v) * LPV + l);
+            }
           }
         }
 #pragma unroll
@@ -134,12 +140,22 @@ __global__ void __launch_bounds__(256)
           if (i0 + u < n && s_src[buf][i0 + u] != nullptr) {   // rows in order; skipped rows add nothing
 #pragma unroll
             for (int j = 0; j < VPT; ++j) {
-              const uint32_t w[4] = {q[u][j].x, q[u][j].y, q[u][j].z, q[u][j].w};
+              if (sizeof(TR) == 2) {
+                const uint32_t w[4] = {q[u][j][0].x, q[u][j][0].y, q[u][j][0].z, q[u][j][0].w};
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
-                acc[j][2 * e] += f.x;
-                acc[j][2 * e + 1] += f.y;
+                for (int e = 0; e < 4; ++e) {
+                  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
+                  acc[j][2 * e] += f.x;
+                  acc[j][2 * e + 1] += f.y;
+                }
+              } else {
+#pragma unroll
+                for (int l = 0; l < LPV; ++l) {
+                  acc[j][4 * l + 0] += __uint_as_float(q[u][j][l].x);
+                  acc[j][4 * l + 1] += __uint_as_float(q[u][j][l].y);
+                  acc[j][4 * l + 2] += __uint_as_float(q[u][j][l].z);
+                  acc[j][4 * l + 3] += __uint_as_float(q[u][j][l].w);
+                }
               }
             }
           }
@@ -157,6 +173,23 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// bf16 output from rows of TR: vectors a thread sized to cover the row in
+// one pass of 256 threads, at most 4 (longer rows take several passes)
+template <typename TR>
+void launch_rows(unsigned grid, cudaStream_t stream, const TR* yr, const TR* ys,
+                 const int32_t* inv_perm, __nv_bfloat16* o, const Layer& L, int64_t cap,
+                 int32_t* status) {
+  const int nv = L.H / 8;
+  if (nv <= 256)
+    combine_rows_kernel<TR, 1><<<grid, 256, 0, stream>>>(yr, ys, inv_perm, o, L.T, L.H, L.k, L.S, cap, status);
+  else if (nv <= 512)
+    combine_rows_kernel<TR, 2><<<grid, 256, 0, stream>>>(yr, ys, inv_perm, o, L.T, L.H, L.k, L.S, cap, status);
+  else if (nv <= 768)
+    combine_rows_kernel<TR, 3><<<grid, 256, 0, stream>>>(yr, ys, inv_perm, o, L.T, L.H, L.k, L.S, cap, status);
+  else
+    combine_rows_kernel<TR, 4><<<grid, 256, 0, stream>>>(yr, ys, inv_perm, o, L.T, L.H, L.k, L.S, cap, status);
+}
+
 }  // namespace
 
 cudaError_t launch_combine(const Layer& L, const void* y_routed, const void* y_shared,
@@ -165,25 +198,13 @@ cudaError_t launch_combine(const Layer& L, const void* y_routed, const void* y_s
   const unsigned grid =
       static_cast<unsigned>(std::min<int64_t>(L.T, static_cast<int64_t>(num_sms) * 8));
   const int64_t cap = L.T * L.k;
-  if (L.dtype == MOE_BF16 && L.y_f16) {
-    // vectors a thread: the fewest that cover the row in one pass of 256
-    // threads, at most 4 (longer rows take several passes)
-    const int nv = L.H / 8;
-    const auto* yr = static_cast<const __half*>(y_routed);
-    const auto* ys = static_cast<const __half*>(y_shared);
-    auto* o = static_cast<__nv_bfloat16*>(out);
-    if (nv <= 256)
-      combine_f16rows_kernel<1><<<grid, 256, 0, stream>>>(yr, ys, inv_perm, o, L.T, L.H, L.k, L.S, cap, status);
-    else if (nv <= 512)
-      combine_f16rows_kernel<2><<<grid, 256, 0, stream>>>(yr, ys, inv_perm, o, L.T, L.H, L.k, L.S, cap, status);
-    else if (nv <= 768)
-      combine_f16rows_kernel<3><<<grid, 256, 0, stream>>>(yr, ys, inv_perm, o, L.T, L.H, L.k, L.S, cap, status);
-    else
-      combine_f16rows_kernel<4><<<grid, 256, 0, stream>>>(yr, ys, inv_perm, o, L.T, L.H, L.k, L.S, cap, status);
-  } else if (L.dtype == MOE_BF16)
-    combine_kernel<__nv_bfloat16, float><<<grid, 256, 0, stream>>>(
-        static_cast<const float*>(y_routed), static_cast<const float*>(y_shared), inv_perm,
-        static_cast<__nv_bfloat16*>(out), L.T, L.H, L.k, L.S, cap, status);
+  auto* o = static_cast<__nv_bfloat16*>(out);
+  if (L.dtype == MOE_BF16 && L.y_f16)
+    launch_rows(grid, stream, static_cast<const __half*>(y_routed),
+                static_cast<const __half*>(y_shared), inv_perm, o, L, cap, status);
+  else if (L.dtype == MOE_BF16)
+    launch_rows(grid, stream, static_cast<const float*>(y_routed),
+                static_cast<const float*>(y_shared), inv_perm, o, L, cap, status);
   else
     combine_kernel<float, float><<<grid, 256, 0, stream>>>(
         static_cast<const float*>(y_routed), static_cast<const float*>(y_shared), inv_perm,
