@@ -47,7 +47,9 @@
  *     Its first 256 bytes hold a sticky device status word; zero them once
  *     with moe_workspace_init() before first use.  Kernels that detect a bad
  *     index or a stalled pipeline record it there instead of faulting;
- *     moe_read_device_status() reads and clears it.
+ *     moe_read_device_status() reads and clears it.  Bytes 64..71 of that
+ *     region are the expert GEMMs' tile counters, which every call that uses
+ *     them zeroes itself on its stream.
  *   - Calls sharing one workspace must be ordered on one stream.
  */
 #ifndef INKLING_MOE_H

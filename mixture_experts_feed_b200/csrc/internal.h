@@ -49,6 +49,14 @@ cudaError_t launch_permute(const Layer& L, const int32_t* topk_idx, const uint8_
 int64_t permute_chunk_slots(int64_t slots);
 int64_t permute_chunks(int64_t slots);
 
+// The workspace's status region: its first 256 bytes.  Byte 0 holds the
+// sticky device status word; bytes kTileCounterOffset .. +7 hold the tile
+// counters of the gate_up pair launch's dynamic schedule (two int32: one for
+// a call with routed groups, one for a call of shared groups alone), which
+// each call zeroes on its stream before its launches.
+constexpr size_t kStatusBytes = 256;
+constexpr size_t kTileCounterOffset = 64;
+
 // grouped_gemm_sm100.cu (bf16, tcgen05)
 // Tile shape choices of one expert-FFN call: the n-tile width of the
 // single-CTA gate_up launch (256 or 128) and the K splits of the down

@@ -16,7 +16,6 @@ namespace moe {
 namespace {
 
 constexpr int kVersion = 1;
-constexpr size_t kStatusBytes = 256;
 constexpr size_t kRegionAlign = 1024;
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }

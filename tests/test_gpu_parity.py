@@ -569,6 +569,29 @@ def test_fp16_overflow_is_reported(where):
     assert ei.value.device_code == 0x103
 
 
+def test_drawn_tile_schedule_long_k():
+    """H >= 4096: the gate_up CTA-pair launch draws its tiles from a counter
+    in the workspace's status region, which each call zeroes itself.  With
+    that counter (and its neighbour, the shared-experts-only call's) left at
+    garbage before the call, the layer matches the oracle on every token
+    (both the one-call path, whose shared groups run on a second stream, and
+    the op chain), twice in a row on the same workspace, bit for bit."""
+    w, inputs = small_case(700, 4096, 8, 2, 1, 256, seed=23)
+    L = moe.Layer.from_workload(w, down_f16=True)
+    d = to_device(inputs, down_f16=True)
+    ws = moe.new_workspace(L)
+    outs = []
+    for _ in range(2):
+        ws[64:72].fill_(0x7F)          # the two tile counters: large garbage
+        f = run_forward(L, d, ws=ws)   # asserts a clean status word
+        outs.append(f["out"])
+    assert torch.equal(outs[0], outs[1])
+    stats, _ = check_all(w, inputs, f)
+    r = run_chain(L, d)
+    assert torch.equal(r["out"], outs[0])
+    print(f"drawn schedule, H=4096: {stats}")
+
+
 @pytest.mark.parametrize("shape", [(300, 256, 12, 3, 2, 320, "bf16"), (1100, 256, 16, 2, 1, 128, "bf16")],
                          ids=["T300", "T1100"])
 def test_stale_workspace_is_harmless(shape):
