@@ -49,7 +49,10 @@
 //   warps 2..5  epilogue: tcgen05.ld this CTA's accumulator rows (warp w
 //               reads TMEM lanes 32*(w%4) .. +31), fused math, global stores.
 // The two accumulators let the epilogue of one tile (or, for kRouter, one K
-// chain) overlap the MMAs of the next.  All waits are bounded
+// chain) overlap the MMAs of the next.  Tiles go to the CTAs (CTA pairs) in
+// a fixed order, or, when the launch is given a tile counter (the gate_up
+// pair launch with long K), as the rank-0 producer draws them, handed to
+// the other roles through a tile queue in shared memory.  All waits are bounded
 // (sm100_ptx.cuh); on a timeout every role stops, the status word records it
 // and TMEM is released.  No TMA load uses cluster multicast.
 #include <atomic>
