@@ -569,6 +569,18 @@ def test_fp16_overflow_is_reported(where):
     assert ei.value.device_code == 0x103
 
 
+@pytest.mark.parametrize("down_f16", [False, True], ids=["fp32-rows", "fp16-rows"])
+def test_combine_rows_longer_than_one_pass(down_f16):
+    """H = 9216: the combine's 256 threads take four 8-value vectors each and
+    still need a second, partial pass over the row (1152 vectors), for fp32
+    and fp16 expert rows alike."""
+    w, inputs = small_case(70, 9216, 4, 2, 1, 128, seed=29)
+    L = moe.Layer.from_workload(w, down_f16=down_f16)
+    r = run_chain(L, to_device(inputs, down_f16=down_f16))
+    stats, _ = check_all(w, inputs, r)
+    print(f"H=9216 combine ({'fp16' if down_f16 else 'fp32'} rows): {stats}")
+
+
 def test_drawn_tile_schedule_long_k():
     """H >= 4096: the gate_up CTA-pair launch draws its tiles from a counter
     in the workspace's status region, which each call zeroes itself.  With
