@@ -69,10 +69,11 @@ def test_dense_workloads(name, down_f16):
     del d
     # every token (7.4 TFLOP in fp64 at the model's sizes: seconds on the host cores)
     ref = oracle.dense_mlp(inputs["x"], inputs["w_gate_up"], inputs["w_down"], w.global_scale)
-    # the plain 2e-2 x RMS bound at the model's sizes; the small shapes get half
-    # a bf16 ulp of the exact value on top (their outputs reach 5 x RMS, where
-    # the final rounding alone costs 2^-8 x 5 = 2% of RMS)
-    rel = check_output(out, ref, w.torch_dtype, f"{name} out", strict=w.H >= 2048)
+    # the plain 2e-2 x RMS bound at the model's sizes and in the fp16-down mode;
+    # the small shapes with bf16 activated rows get half a bf16 ulp of the
+    # exact value on top (their outputs reach 5 x RMS, where the final rounding
+    # alone costs 2^-8 x 5 = 2% of RMS; measured 2.10% at H=512)
+    rel = check_output(out, ref, w.torch_dtype, f"{name} out", strict=w.H >= 2048 or down_f16)
     print(f"{name} ({'fp16' if down_f16 else 'bf16'} down): all {w.T} tokens, max|err|/RMS = {rel:.4f}")
 
 
