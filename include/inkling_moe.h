@@ -258,6 +258,57 @@ moe_status_t moe_ep_dispatch_prep(const moe_layer_desc_t* desc, const int32_t* e
                                   void* stream);
 
 /*
+ * moe_ep_dispatch_p2p — the dispatch of expert parallelism over peer memory
+ * (NVLink between the GPUs of a node; same layers-page passages as
+ * moe_ep_dispatch_prep).  Rank r's permuted rows go straight from x into
+ * the receive buffers of the ranks that own their experts, each with its
+ * routing weight: for permuted row i of expert e (offsets[e] <= i <
+ * offsets[e+1]), owner d = e / El (El = E / n_ranks) and
+ *   dst_x[d][dst_base[e] + i - offsets[e]] = x[perm_slot[i] / k]   (H values)
+ *   dst_w[d][dst_base[e] + i - offsets[e]] = topk_w[perm_slot[i]]
+ * dst_base[e] is the row of d's receive buffers where this rank's rows of
+ * expert e start (the caller computes it from every rank's counts).  No
+ * x_perm copy is made (moe_permute may be called with x_perm = NULL).
+ *   desc: this rank's layer (T its tokens, E all routed experts);
+ *   x [T,H] dtype (16-byte aligned), topk_w [T*k] fp32, perm_slot [T*k],
+ *   expert_offsets [E+1] (from moe_permute), dst_base [E] int32 — device;
+ *   dst_x, dst_w: device arrays of n_ranks pointers, valid in this process
+ *   (this rank's own buffers, or peers' mapped by CUDA IPC), each buffer
+ *   dst_rows rows of H dtype values (dst_x) or fp32 (dst_w).  A destination
+ *   row outside [0, dst_rows) or a bad slot is recorded in the status word at
+ *   the head of `workspace` (>= 256 bytes) and that row is skipped.
+ * The kernel only stores; before any rank reads its receive buffers the
+ * caller orders every rank's dispatch before that read (an all-reduce over
+ * the ranks on the same stream, or a host barrier).  E % n_ranks != 0, or a
+ * null or misaligned pointer: MOE_ERR_INVALID_ARG.
+ */
+moe_status_t moe_ep_dispatch_p2p(const moe_layer_desc_t* desc, const void* x, const float* topk_w,
+                                 const int32_t* perm_slot, const int32_t* expert_offsets,
+                                 const int32_t* dst_base, int32_t n_ranks, void* const* dst_x,
+                                 float* const* dst_w, int64_t dst_rows, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/*
+ * moe_ep_return_p2p — the return of expert parallelism over peer memory.  A
+ * rank's received rows are ordered by local expert el, then by source rank s
+ * (run el * n_ranks + s); after moe_expert_ffn its output row i of run j goes
+ * back to the source's y rows at the row's place in the source's permuted
+ * order:
+ *   dst_y[s][src_base[j] + i - run_start[j]] = y_in[i]   (H values)
+ *   desc: the layer (H, E, dtype; the rows are fp16 for MOE_BF16_F16DOWN,
+ *   else fp32); y_in [rows_in, H]; run_start [E + 1] int32 ascending with
+ *   run_start[E] == rows_in, src_base [E] int32 (for run el*n_ranks + s:
+ *   source s's expert_offsets[first + el]) — device; dst_y: device array of
+ *   n_ranks pointers to buffers of dst_rows rows.  A destination row outside
+ *   [0, dst_rows), or run_start[E] != rows_in, is recorded in the status word
+ *   and the row (or the call) skipped.  Ordering as for moe_ep_dispatch_p2p.
+ */
+moe_status_t moe_ep_return_p2p(const moe_layer_desc_t* desc, const void* y_in, int64_t rows_in,
+                               const int32_t* run_start, const int32_t* src_base, int32_t n_ranks,
+                               void* const* dst_y, int64_t dst_rows, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/*
  * moe_combine — InklingMoE.forward recombination:
  *   out[t] = sum_s y_shared[s*T + t] + sum_{j<k, inv_perm[t*k+j] >= 0} y_routed[inv_perm[t*k+j]]
  * summed in fp32 in that fixed order, rounded once to dtype.  y_routed and

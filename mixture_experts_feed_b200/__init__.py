@@ -75,6 +75,10 @@ LIB.moe_shared_ffn.argtypes = [_DESC, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _
 LIB.moe_shared_ffn_kernel_count.restype = ctypes.c_int32
 LIB.moe_shared_ffn_kernel_count.argtypes = [_DESC]
 LIB.moe_ep_dispatch_prep.argtypes = [_DESC, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+LIB.moe_ep_dispatch_p2p.argtypes = [_DESC, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _P,
+                                    ctypes.c_int64, _P, ctypes.c_size_t, _P]
+LIB.moe_ep_return_p2p.argtypes = [_DESC, _P, ctypes.c_int64, _P, _P, ctypes.c_int32, _P,
+                                  ctypes.c_int64, _P, ctypes.c_size_t, _P]
 LIB.moe_convert_bf16_to_f16.argtypes = [ctypes.c_int64, _P, _P, _P, _P]
 LIB.moe_forward.argtypes = [_DESC] + [_P] * 13 + [ctypes.c_size_t, _P]
 LIB.moe_selftest_wait_timeout.argtypes = [_P, ctypes.c_size_t, ctypes.c_uint32, _P]
@@ -96,7 +100,8 @@ for _f in ("moe_workspace_size", "moe_workspace_init", "moe_read_device_status",
            "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_selftest_wait_timeout", "moe_dense_workspace_size", "moe_dense_mlp",
            "moe_rmsnorm", "moe_forward_prenorm", "moe_dense_mlp_prenorm", "moe_shared_ffn",
-           "moe_ep_dispatch_prep", "moe_convert_bf16_to_f16"):
+           "moe_ep_dispatch_prep", "moe_ep_dispatch_p2p", "moe_ep_return_p2p",
+           "moe_convert_bf16_to_f16"):
     getattr(LIB, _f).restype = ctypes.c_int
 
 
@@ -325,6 +330,51 @@ def moe_ep_dispatch_prep(layer: Layer, expert_offsets, perm_slot, topk_w, row_w,
     _check(LIB.moe_ep_dispatch_prep(ctypes.byref(L.desc()), _ptr(expert_offsets), _ptr(perm_slot),
                                     _ptr(topk_w), _ptr(row_w), _ptr(expert_counts), ws.data_ptr(),
                                     ws.numel(), _stream(stream)), "moe_ep_dispatch_prep")
+
+
+def _ptr_table(ptrs, n: int, what: str) -> None:
+    if (not isinstance(ptrs, torch.Tensor) or ptrs.dtype != torch.int64 or ptrs.numel() != n
+            or not ptrs.is_cuda or not ptrs.is_contiguous()):
+        raise ValueError(f"{what} must be a contiguous int64 CUDA tensor of {n} device pointers")
+
+
+def moe_ep_dispatch_p2p(layer: Layer, x, topk_w, perm_slot, expert_offsets, dst_base, n_ranks: int,
+                        dst_x, dst_w, dst_rows: int, ws, stream=None):
+    """Every permuted row of this rank, with its weight, stored straight into
+    the receive buffers of the rank that owns its expert (``dst_x`` /
+    ``dst_w``: int64 CUDA tensors of ``n_ranks`` device pointers, buffers of
+    ``dst_rows`` rows; ``dst_base [E]``: where this rank's rows of each expert
+    start there)."""
+    L = layer
+    _expect(x, "x", (L.T, L.H), L.dtype)
+    if topk_w.numel() != L.T * L.k or topk_w.dtype != torch.float32 or not topk_w.is_contiguous():
+        raise ValueError("topk_w must be a contiguous fp32 tensor of T*k entries")
+    _expect(perm_slot, "perm_slot", (L.T * L.k,), torch.int32)
+    _expect(expert_offsets, "expert_offsets", (L.E + 1,), torch.int32)
+    _expect(dst_base, "dst_base", (L.E,), torch.int32)
+    _ptr_table(dst_x, n_ranks, "dst_x")
+    _ptr_table(dst_w, n_ranks, "dst_w")
+    _check(LIB.moe_ep_dispatch_p2p(ctypes.byref(L.desc()), _ptr(x), _ptr(topk_w), _ptr(perm_slot),
+                                   _ptr(expert_offsets), _ptr(dst_base), n_ranks, _ptr(dst_x),
+                                   _ptr(dst_w), dst_rows, ws.data_ptr(), ws.numel(),
+                                   _stream(stream)), "moe_ep_dispatch_p2p")
+
+
+def moe_ep_return_p2p(layer: Layer, y_in, rows_in: int, run_start, src_base, n_ranks: int, dst_y,
+                      dst_rows: int, ws, stream=None):
+    """Every received output row stored straight into its source's y rows
+    (``dst_y``: int64 CUDA tensor of ``n_ranks`` device pointers to buffers of
+    ``dst_rows`` rows); runs ordered by local expert, then source."""
+    L = layer
+    if y_in.dtype != L.y_dtype or y_in.dim() != 2 or y_in.shape[1] != L.H or y_in.shape[0] < rows_in \
+            or not y_in.is_contiguous():
+        raise ValueError(f"y_in must be a contiguous [>= {rows_in}, {L.H}] {L.y_dtype} tensor")
+    _expect(run_start, "run_start", (L.E + 1,), torch.int32)
+    _expect(src_base, "src_base", (L.E,), torch.int32)
+    _ptr_table(dst_y, n_ranks, "dst_y")
+    _check(LIB.moe_ep_return_p2p(ctypes.byref(L.desc()), _ptr(y_in), rows_in, _ptr(run_start),
+                                 _ptr(src_base), n_ranks, _ptr(dst_y), dst_rows, ws.data_ptr(),
+                                 ws.numel(), _stream(stream)), "moe_ep_return_p2p")
 
 
 def moe_combine(layer: Layer, y_routed, y_shared, inv_perm, out, ws, stream=None):

@@ -9,7 +9,8 @@ them the exchange logic runs on CPU ranks over gloo.
 process on one GPU.  Every exchange is host-synchronised: each rank's stream
 is synchronised before its tensors are posted and after its copies, and the
 ranks meet at a barrier between posting and copying.  No kernel ever waits on
-another rank's kernel.
+another rank's kernel.  For the peer-memory transport it also hands out the
+other threads' buffer addresses (all on the one GPU) and a host barrier.
 """
 from __future__ import annotations
 
@@ -136,6 +137,28 @@ class _RankComm:
                                    f"unreceived messages from {peer}")
         self._sync()
         self.s.barrier.wait()
+
+    # the peer-memory transport: all ranks' buffers live on the one GPU, so a
+    # rank's "peer" pointers are the other threads' tensors' addresses
+    def all_gather(self, out, inp):
+        self._sync()
+        self.s.box[("ag", self.rank)] = inp
+        self.s.barrier.wait()
+        for src in range(self.world):
+            out[src].copy_(self.s.box[("ag", src)])
+        self._sync()
+        self.s.barrier.wait()
+
+    def device_barrier(self, device):
+        self._sync()
+        self.s.barrier.wait()
+
+    def peer_pointers(self, tensors):
+        self.s.box[("pp", self.rank)] = [t.data_ptr() for t in tensors]
+        self.s.barrier.wait()
+        out = [[self.s.box[("pp", src)][i] for src in range(self.world)] for i in range(len(tensors))]
+        self.s.barrier.wait()
+        return out
 
 
 def rank_weights(inputs: dict, E: int, world: int, rank: int) -> dict:

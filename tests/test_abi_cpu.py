@@ -236,6 +236,31 @@ def test_new_entry_points_host_checks():
     assert moe.LIB.moe_ep_dispatch_prep(d1, fake, fake, fake, fake, fake, fake, 100, None) == 1
 
 
+def test_peer_memory_entry_points_host_checks():
+    """moe_ep_dispatch_p2p and moe_ep_return_p2p reject bad arguments on the
+    host (fake aligned pointers are never touched)."""
+    fake, big = 1 << 20, 1 << 40
+    L = moe.Layer(64, 128, 8, 2, 1, 64)
+    d = ctypes.byref(L.desc())
+    ok = [fake, fake, fake, fake, fake]                       # x, topk_w, perm_slot, offsets, dst_base
+    for i in range(5):
+        args = list(ok)
+        args[i] = None
+        assert moe.LIB.moe_ep_dispatch_p2p(d, *args, 2, fake, fake, 100, fake, 4096, None) == 1
+    assert moe.LIB.moe_ep_dispatch_p2p(d, fake + 8, *ok[1:], 2, fake, fake, 100, fake, 4096, None) == 1
+    assert moe.LIB.moe_ep_dispatch_p2p(d, *ok, 3, fake, fake, 100, fake, 4096, None) == 1   # 8 % 3
+    assert moe.LIB.moe_ep_dispatch_p2p(d, *ok, 2, None, fake, 100, fake, 4096, None) == 1
+    assert moe.LIB.moe_ep_dispatch_p2p(d, *ok, 2, fake, fake, 100, fake, 100, None) == 1   # workspace
+    assert moe.LIB.moe_ep_return_p2p(d, fake, 10, None, fake, 2, fake, 100, fake, 4096, None) == 1
+    assert moe.LIB.moe_ep_return_p2p(d, fake, 10, fake, fake, 0, fake, 100, fake, 4096, None) == 1
+    assert moe.LIB.moe_ep_return_p2p(d, fake + 8, 10, fake, fake, 2, fake, 100, fake, 4096, None) == 1
+    assert moe.LIB.moe_ep_return_p2p(d, fake, -1, fake, fake, 2, fake, 100, fake, 4096, None) == 1
+    assert moe.LIB.moe_ep_return_p2p(d, None, 0, fake, fake, 2, fake, 100, fake, 4096, None) == 0
+    L0 = moe.Layer(0, 128, 8, 2, 1, 64)
+    assert moe.LIB.moe_ep_dispatch_p2p(ctypes.byref(L0.desc()), *ok, 2, fake, fake, 100, fake, 4096,
+                                       None) == 0          # T = 0: nothing launched
+
+
 def test_expert_ffn_needs_a_row_map_or_a_copy():
     """moe_expert_ffn takes perm_slot = NULL only when x_perm is given (rows
     already in slot order); with neither the rows cannot be found."""

@@ -23,7 +23,7 @@ from moe_gpu_helpers import check_output, run_forward, to_device
 pytestmark = pytest.mark.gpu
 
 
-def run_ranks(inputs, world, T_rank, E, k, S, route_scale, pm=None):
+def run_ranks(inputs, world, T_rank, E, k, S, route_scale, pm=None, transport="exchange", calls=1):
     from mixture_experts_feed_b200.ep import ExpertParallelMoE, read_device_status
     shared = LoopbackComm(world)
     outs, counts, errs = [None] * world, [None] * world, []
@@ -32,12 +32,17 @@ def run_ranks(inputs, world, T_rank, E, k, S, route_scale, pm=None):
         try:
             torch.cuda.set_device(0)
             layer = ExpertParallelMoE(rank_weights(inputs, E, world, r), E, k, S, route_scale,
-                                      comm=shared.bind(r), device="cuda")
+                                      comm=shared.bind(r), device="cuda", transport=transport)
             x = inputs["x"][r * T_rank:(r + 1) * T_rank].cuda()
             m = None if pm is None else pm[r * T_rank:(r + 1) * T_rank]
             o = layer(x, padding_mask=m)
             torch.cuda.synchronize()
             assert read_device_status(layer) == 0
+            for _ in range(calls - 1):     # again, into the buffers of the first call
+                again = layer(x, padding_mask=m)
+                torch.cuda.synchronize()
+                assert read_device_status(layer) == 0
+                assert torch.equal(again, o)
             outs[r], counts[r] = o.cpu(), layer.last_counts
         except BaseException as e:    # noqa: BLE001 - reported below
             errs.append((r, e))
@@ -61,10 +66,15 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("transport", ["exchange", "p2p"])
 @pytest.mark.parametrize("case", CASES, ids=[f"W{c[0]}-T{c[1]}-H{c[2]}-E{c[3]}k{c[4]}S{c[5]}-I{c[6]}"
                                              + ("-skew" if c[7] else "") + ("-down-f16" if c[8] else "")
                                              for c in CASES])
-def test_ep_virtual_ranks(case):
+def test_ep_virtual_ranks(case, transport):
+    """``exchange``: rows and results travel as grouped sends and receives.
+    ``p2p``: moe_ep_dispatch_p2p and moe_ep_return_p2p store them straight
+    into the other ranks' buffers (here all on the one GPU), twice in a row
+    into the same buffers."""
     world, T_rank, H, E, k, S, I, skew, down_f16 = case
     w = mw.tiny(T=T_rank * world, H=H, E=E, k=k, S=S, I=I, dtype="bf16", route_scale=2.5, seed=23)
     inputs = mw.generate(w, threads=4)
@@ -76,7 +86,8 @@ def test_ep_virtual_ranks(case):
     if down_f16:   # the ranks hold the exact fp16 copies of the down weights
         rank_inputs["w_down"] = inputs["w_down"].to(torch.float16)
         rank_inputs["ws_down"] = inputs["ws_down"].to(torch.float16)
-    out_ep, counts = run_ranks(rank_inputs, world, T_rank, E, k, S, w.route_scale, pm=pm)
+    out_ep, counts = run_ranks(rank_inputs, world, T_rank, E, k, S, w.route_scale, pm=pm,
+                               transport=transport, calls=2 if transport == "p2p" else 1)
     if skew:
         assert all(sum(counts[r][1]) == 0 for r in range(1, world))
     L = __import__("mixture_experts_feed_b200").Layer.from_workload(w, down_f16=down_f16)
@@ -85,5 +96,5 @@ def test_ep_virtual_ranks(case):
     ref = oracle.moe_forward_workload(inputs, w, padding_mask=pm,
                                       given_topk_idx=one["topk_idx"].to(torch.int64))
     rel = check_output(out_ep, ref["out"], torch.bfloat16, "expert-parallel out", strict=False)
-    print(f"W={world}: rows sent {[sum(c[0]) for c in counts]}, received "
+    print(f"W={world} {transport}: rows sent {[sum(c[0]) for c in counts]}, received "
           f"{[sum(c[1]) for c in counts]}; max|out - oracle|/RMS = {rel:.4f}")
