@@ -88,9 +88,11 @@ def load_peaks():
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """nvidia-smi clock / throttle samples while the timed region runs."""
+    """nvidia-smi clock / throttle samples, every 20 ms, kept when they fall
+    inside the timed region (``mark_start`` / ``mark_end`` give its host-time
+    bounds; each sample carries nvidia-smi's timestamp)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -98,6 +100,13 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
@@ -105,7 +114,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", str(self.gpu), "-lms", "100"],
+                 "-i", str(self.gpu), "-lms", "20"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except (OSError, FileNotFoundError):
@@ -128,23 +137,31 @@ class ClockSampler:
         rows = []
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                rows.append((float(parts[1]), float(parts[2]), parts[4:9]))
+                stamp, frac = (parts[0].split(".") + ["0"])[:2]
+                t = time.mktime(time.strptime(stamp, "%Y/%m/%d %H:%M:%S")) + float("0." + frac)
+                rows.append((t, float(parts[2]), float(parts[3]), parts[5:10]))
             except ValueError:
                 continue
         os.unlink(self.path)
-        if not rows:
+        inside = [r for r in rows if self.t0 is not None and self.t1 is not None
+                  and self.t0 <= r[0] <= self.t1]
+        window = "timed region"
+        if not inside:   # a region shorter than the sampling gap: the samples nearest to it
+            inside = sorted(rows, key=lambda r: abs(r[0] - ((self.t0 or 0) + (self.t1 or 0)) / 2))[:2]
+            window = "nearest samples"
+        if not inside:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         seen = set()
-        for _, _, flags in rows:
+        for _, _, _, flags in inside:
             for n, v in zip(names, flags[1:]):
                 if v.lower() == "active":
                     seen.add(n)
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": sorted(seen), "samples": len(rows)}
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": sorted(seen), "samples": len(inside), "window": window}
 
 
 # ------------------------------------------------------------- distributed
@@ -387,11 +404,13 @@ def time_workload(moe, name: str, steps: int, warmup: int, dev, stream, peaks, p
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index or 0) as clk:
         torch.cuda.synchronize(dev)
+        clk.mark_start()
         e0.record(stream)
         for i in range(steps):
             fwd()
         e1.record(stream)
         torch.cuda.synchronize(dev)
+        clk.mark_end()
     ms = e0.elapsed_time(e1) / steps
     for _ in range(warmup):
         step()
@@ -529,6 +548,7 @@ def gpu_arm(args, world, rank, local):
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize(dev)
+        clk.mark_start()
         e_start.record(stream)
         for i in range(args.steps):
             if graph is None:
@@ -537,6 +557,7 @@ def gpu_arm(args, world, rank, local):
                 graph.replay()
         e_end.record(stream)
         torch.cuda.synchronize(dev)
+        clk.mark_end()
         barrier(world)
     clocks = clk.summary()
     moe.read_device_status(ws, stream)
@@ -755,11 +776,13 @@ def dense_gpu_arm(args, world, rank, local):
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize(dev)
+        clk.mark_start()
         e0.record(stream)
         for _ in range(args.steps):
             step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
+        clk.mark_end()
         barrier(world)
     clocks = clk.summary()
     moe.read_device_status(ws, stream)
