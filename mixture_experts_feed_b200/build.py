@@ -26,7 +26,7 @@ LIB = os.path.join(PKG, "libinklingmoe.so")
 
 SOURCES = ["moe_api.cu", "router.cu", "permute.cu", "permute_noalloc.cu",
            "grouped_gemm_sm100.cu", "grouped_gemm_simt.cu", "combine.cu", "rmsnorm.cu",
-           "selftest.cu", "expert_parallel.cu", "weights.cu"]
+           "selftest.cu", "expert_parallel.cu", "weights.cu", "swiglu.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
                      "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

@@ -971,10 +971,40 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   g.bn = tiling.gate_up_bn;
   g.gather_k = gather ? L.k : 0;
   g.f16 = L.down_f16 ? 1 : 0;   // h in fp16 for fp16 down projections
-  g.tile_counter = gate_up_counter;
-  cudaError_t e = pairs ? launch_mode<kGateUp, true>(g, num_sms, stream) : cudaSuccess;
-  g.tile_counter = nullptr;
-  if (e == cudaSuccess && singles) e = launch_mode<kGateUp, false>(g, num_sms, stream);
+  cudaError_t e = cudaSuccess;
+  if (tiling.gate_up_ksplit > 1) {
+    // The dense layer with few tokens: gate_up as a plain GEMM with its K
+    // split (the kDown mode's fp32 partial stores: split s at rows s * T of
+    // gate_up_part [ks * T, 2I]), then the SwiGLU over the partials.  More
+    // tiles than the n-tiles alone give fill the SMs in whole waves.
+    const int ks = tiling.gate_up_ksplit;
+    if (L.E != 0 || L.S != 1 || pairs || tiling.gate_up_part == nullptr) return cudaErrorInvalidValue;
+    GemmParams q{};
+    ok = encode_a(&q.tmA[0], x, L.T, L.H) &&
+         encode_b(&q.tmB[0], ws_gate_up, 1, 2 * L.I, L.H, BROWS) &&
+         encode_y(&q.tmY[0], tiling.gate_up_part, L.T * static_cast<int64_t>(ks), 2 * L.I);
+    if (!ok) { *map_error = true; return cudaErrorInvalidValue; }
+    q.tmA[1] = q.tmA[0];
+    q.tmB[1] = q.tmB[0];
+    q.tmY[1] = q.tmY[0];
+    q.out[0] = q.out[1] = tiling.gate_up_part;
+    q.status = status;
+    q.T = L.T; q.a1_base = 0; q.a1_stride = L.T;
+    q.E = 0; q.S = 1; q.K = L.H; q.N = 2 * L.I; q.ld_out = 2 * L.I;
+    q.rows_cap = 0;
+    q.ksplit = ks;
+    q.split_stride = L.T * static_cast<int64_t>(2 * L.I);
+    q.bn = 256;
+    e = launch_mode<kDown, false>(q, num_sms, stream);
+    if (e == cudaSuccess)
+      e = launch_swiglu_partials(tiling.gate_up_part, ks, L.T, L.I, L.global_scale, L.down_f16,
+                                 h, status, num_sms, stream);
+  } else {
+    g.tile_counter = gate_up_counter;
+    e = pairs ? launch_mode<kGateUp, true>(g, num_sms, stream) : cudaSuccess;
+    g.tile_counter = nullptr;
+    if (e == cudaSuccess && singles) e = launch_mode<kGateUp, false>(g, num_sms, stream);
+  }
   if (e != cudaSuccess) return e;
 
   // ---------------- down: h [rows, I] x [H, I]^T -> y [rows, H] (fp32)

@@ -59,13 +59,22 @@ constexpr size_t kTileCounterOffset = 64;
 
 // grouped_gemm_sm100.cu (bf16, tcgen05)
 // Tile shape choices of one expert-FFN call: the n-tile width of the
-// single-CTA gate_up launch (256 or 128) and the K splits of the down
-// projection (its split s writes partial rows at y_shared + s * T * H; the
-// caller sums them).  The MoE layer uses the defaults.
+// single-CTA gate_up launch (256 or 128), the K splits of the gate_up
+// projection (the dense layer with few tokens: split s writes its raw fp32
+// accumulators at gate_up_part + s * T * 2I, and launch_swiglu_partials
+// adds them and forms h), and the K splits of the down projection (split s
+// writes partial rows at y_shared + s * T * H; the caller sums them).  The
+// MoE layer uses the defaults.
 struct FfnTiling {
   int gate_up_bn = 256;
+  int gate_up_ksplit = 1;
+  float* gate_up_part = nullptr;   // [gate_up_ksplit][T][2I] when gate_up_ksplit > 1
   int down_ksplit = 1;
 };
+// swiglu.cu: h[t][j] = w * silu(g) * u from the K-split partials of gate_up
+cudaError_t launch_swiglu_partials(const float* part, int ksplit, int64_t T, int I, float w,
+                                   bool f16, void* h, int32_t* status, int num_sms,
+                                   cudaStream_t stream);
 cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_perm,
                                    const int32_t* offsets, const int32_t* perm_slot,
                                    const float* topk_w, const float* gamma, const void* w_gate_up,

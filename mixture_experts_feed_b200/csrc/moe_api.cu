@@ -321,7 +321,7 @@ moe_status_t forward_checked(const moe_layer_desc_t* desc, const void* x, const 
 // T tokens (E = 0, S = 1) whose per-token weight is global_scale, then the
 // recombination with k = 0 rounds y into out.
 struct DenseWs {
-  size_t status, h, y, x_norm, total;
+  size_t status, h, y, gu_part, x_norm, total;
 };
 
 // Tile choices of the dense layer on the tensor cores (functions of the
@@ -341,7 +341,21 @@ FfnTiling dense_tiling(const Layer& L) {
   };
   if (L.T <= 128) {   // every tile on the single-CTA launch
     const int64_t t256 = mt * ((2 * L.I + 255) / 256), t128 = mt * ((2 * L.I + 127) / 128);
-    if (t256 < 4 * kTilingSms && waves_eff(t128) > waves_eff(t256) + 0.05) t.gate_up_bn = 128;
+    double best = waves_eff(t256);
+    if (t256 < 4 * kTilingSms && waves_eff(t128) > best + 0.05) {
+      t.gate_up_bn = 128;
+      best = waves_eff(t128);
+    }
+    // or split gate_up's K (256-wide tiles, each split a fresh accumulation,
+    // at least 16 K blocks a split) when that fills the waves better still
+    for (int ks = 2; ks <= 4 && t256 < 4 * kTilingSms; ++ks) {
+      if (L.H / 64 / ks < 16) break;
+      if (waves_eff(t256 * ks) > best + 0.05) {
+        best = waves_eff(t256 * ks);
+        t.gate_up_ksplit = ks;
+        t.gate_up_bn = 256;
+      }
+    }
   }
   const int64_t down_tiles = mt * ((L.H + 255) / 256);   // m-tiles x n-tiles (either launch)
   if (down_tiles < kTilingSms) {
@@ -387,7 +401,10 @@ DenseWs dense_ws_layout(const Layer& L) {
   const size_t T = static_cast<size_t>(L.T);
   w.status = take(kStatusBytes);
   w.h = take(T * L.I * elt);
-  w.y = take(T * L.H * 4 * dense_tiling(L).down_ksplit);   // one partial per K split
+  const FfnTiling tiling = dense_tiling(L);
+  w.y = take(T * L.H * 4 * tiling.down_ksplit);   // one partial per K split
+  // gate_up's K-split accumulators (fp32, [ks][T][2I]) when its K is split
+  w.gu_part = take(tiling.gate_up_ksplit > 1 ? T * 2 * L.I * 4 * tiling.gate_up_ksplit : 0);
   w.x_norm = take(T * L.H * elt);    // moe_dense_mlp_prenorm: the normalised input
   w.total = off;
   return w;
@@ -415,7 +432,8 @@ moe_status_t dense_checked(const moe_dense_desc_t* desc, const void* x, const vo
     x = xn;
   }
   // one shared group: the routed operands are never read (E = 0, k = 0)
-  const FfnTiling tiling = dense_tiling(L);
+  FfnTiling tiling = dense_tiling(L);
+  tiling.gate_up_part = region<float>(workspace, w.gu_part);
   if (L.dtype == MOE_BF16) {
     bool map_error = false;
     const cudaError_t e = launch_expert_ffn_bf16(L, x, x, nullptr, nullptr, nullptr, nullptr,
@@ -652,8 +670,9 @@ int32_t moe_dense_kernel_count(const moe_dense_desc_t* desc) {
   Layer L;
   if (check_dense(desc, &L) != MOE_OK || L.T == 0) return 0;
   // gate_up + down (one launch each: the one group's tiles are all CTA-pair
-  // or all single-CTA tiles), then the rounding pass
-  return 3;
+  // or all single-CTA tiles; a K-split gate_up adds its SwiGLU pass), then
+  // the rounding pass
+  return L.dtype == MOE_BF16 && dense_tiling(L).gate_up_ksplit > 1 ? 4 : 3;
 }
 
 int32_t moe_dense_prenorm_kernel_count(const moe_dense_desc_t* desc) {

@@ -42,6 +42,7 @@ SMALL = [
     (1, 128, 64, "bf16", 1.0),          # a single token
     (129, 128, 192, "bf16", 1.0),       # 2 m-tiles, the second one row
     (64, 256, 1024, "bf16", 1.0),       # decode-shaped: 128-wide gate_up tiles, down split 4 ways
+    (16, 4096, 2048, "bf16", 0.75),     # decode-shaped, long K: gate_up's K split 4 ways + SwiGLU pass
     (96, 128, 192, "f32", 1.0),         # fp32 layer (CUDA cores)
     (77, 192, 128, "f32", 1.5),
 ]
