@@ -159,6 +159,34 @@ def test_padding_mask():
     assert torch.equal(f["out"], r["out"])
 
 
+@pytest.mark.parametrize("route_scale,global_scale", [(8.0, 0.5), (1.0, 2.0)])
+def test_route_and_global_scales(route_scale, global_scale):
+    """Other scales than the workloads' 2.5 x 1: the weights of every token
+    sum to route_scale * global_scale and the output meets the bar."""
+    w = mw.tiny(T=200, H=256, E=16, k=4, S=2, I=128, dtype="bf16", route_scale=route_scale,
+                global_scale=global_scale, seed=41)
+    inputs = mw.generate(w, threads=4)
+    L = moe.Layer.from_workload(w, down_f16=True)
+    r = run_forward(L, to_device(inputs, down_f16=True))
+    check_all(w, inputs, r)
+    tot = r["topk_w"].double().sum(1) + r["shared_gamma"].double().sum(1)
+    assert torch.allclose(tot, torch.full_like(tot, route_scale * global_scale), rtol=1e-5)
+
+
+def test_every_token_padded():
+    """A batch whose every token is padding: no routed rows at all, the
+    shared experts alone make the output."""
+    w, inputs = small_case(150, 256, 12, 3, 2, 128)
+    pm = torch.ones(w.T, dtype=torch.bool)
+    L = moe.Layer.from_workload(w)
+    r = run_chain(L, to_device(inputs), padding_mask=pm)
+    assert int(r["offsets"][-1]) == 0
+    assert bool((r["inv_perm"] == -1).all())
+    check_all(w, inputs, r, padding_mask=pm)
+    f = run_forward(L, to_device(inputs), padding_mask=pm)
+    assert torch.equal(f["out"], r["out"])
+
+
 def test_deterministic_bitwise():
     w, inputs = small_case(700, 256, 24, 4, 1, 192)
     L = moe.Layer.from_workload(w)
