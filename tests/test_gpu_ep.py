@@ -63,6 +63,7 @@ CASES = [
     (2, 256, 256, 16, 4, 1, 192, False, False),
     (4, 128, 256, 16, 2, 2, 128, False, True),
     (4, 128, 128, 16, 2, 1, 64, True, True),    # every row to rank 0's experts: ranks 1-3 receive none
+    (8, 64, 128, 16, 2, 1, 64, False, True),    # eight ranks of two experts each
 ]
 
 
