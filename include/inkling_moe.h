@@ -322,11 +322,12 @@ moe_status_t moe_combine(const moe_layer_desc_t* desc, const void* y_routed, con
  * moe_forward — InklingMoE.forward in one call: moe_route, moe_permute,
  * moe_expert_ffn, moe_combine with every intermediate in `workspace`
  * (including the permuted copy x_perm [T*k, H]).  For bf16 layers with
- * shared experts the shared experts' GEMMs run on a second stream the
- * library keeps for each device (created, with two events, on the first such
- * call; no device memory), forked from `stream` after the router and joined
- * back before the combine, so that they overlap the permutation and the
- * routed experts' GEMMs.  The call stays asynchronous on `stream` and can be
+ * shared experts the shared experts' gate_up GEMM runs on a second stream
+ * the library keeps for each device (created, with two events, on the first
+ * such call; no device memory), forked from `stream` after the router so that
+ * it overlaps the permutation and the routed experts' gate_up, and joined
+ * back before the down projection, which covers the routed and the shared
+ * experts in the same launches.  The call stays asynchronous on `stream` and can be
  * captured in a CUDA graph (the fork and join are captured with it).  Calls
  * from several host threads share that second stream, in call order.
  *   out [T, H] dtype.  topk_w, topk_idx, shared_gamma are optional outputs

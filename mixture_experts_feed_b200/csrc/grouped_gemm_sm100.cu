@@ -927,6 +927,9 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   // launches only the kind of CTA that has tiles)
   const bool pairs = L.T > BM && (L.E > 0 || group_paired(static_cast<int>((L.T + BM - 1) / BM)));
   const bool singles = L.E > 0 || !pairs;
+  // tiling.part: both projections, or one of them (a caller that splits the
+  // two around a join of streams)
+  const bool do_gate_up = tiling.part != 2, do_down = tiling.part != 1;
   // The gate_up pair launch with long K (H >= 4096) draws its tiles from a
   // counter (the dynamic schedule of the kernel): its clusters then stay on
   // a narrow window of consecutive tiles, whose A rows and weight strips L2
@@ -938,7 +941,7 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   // groups alone, E == 0, takes the next one, so that it can run on another
   // stream beside a call of the routed groups) and is zeroed here.
   int* gate_up_counter = nullptr;
-  if (status != nullptr && pairs && L.H >= 4096) {
+  if (status != nullptr && pairs && L.H >= 4096 && do_gate_up) {
     gate_up_counter = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(status) + kTileCounterOffset) +
                       (L.E == 0 ? 1 : 0);
     const cudaError_t e = cudaMemsetAsync(gate_up_counter, 0, sizeof(int), stream);
@@ -972,7 +975,9 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   g.gather_k = gather ? L.k : 0;
   g.f16 = L.down_f16 ? 1 : 0;   // h in fp16 for fp16 down projections
   cudaError_t e = cudaSuccess;
-  if (tiling.gate_up_ksplit > 1) {
+  if (!do_gate_up) {
+    // the activated rows are already in h
+  } else if (tiling.gate_up_ksplit > 1) {
     // The dense layer with few tokens: gate_up as a plain GEMM with its K
     // split (the kDown mode's fp32 partial stores: split s at rows s * T of
     // gate_up_part [ks * T, 2I]), then the SwiGLU over the partials.  More
@@ -1005,7 +1010,7 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
     g.tile_counter = nullptr;
     if (e == cudaSuccess && singles) e = launch_mode<kGateUp, false>(g, num_sms, stream);
   }
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || !do_down) return e;
 
   // ---------------- down: h [rows, I] x [H, I]^T -> y [rows, H] (fp32)
   GemmParams d{};

@@ -66,6 +66,7 @@ constexpr size_t kTileCounterOffset = 64;
 // writes partial rows at y_shared + s * T * H; the caller sums them).  The
 // MoE layer uses the defaults.
 struct FfnTiling {
+  int part = 0;                    // 0: gate_up and down; 1: gate_up only; 2: down only
   int gate_up_bn = 256;
   int gate_up_ksplit = 1;
   float* gate_up_part = nullptr;   // [gate_up_ksplit][T][2I] when gate_up_ksplit > 1

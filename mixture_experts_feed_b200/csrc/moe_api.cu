@@ -280,21 +280,25 @@ moe_status_t forward_checked(const moe_layer_desc_t* desc, const void* x, const 
   void* y_shared = region<void>(workspace, w.y_shared);
   MOE_TRY(route_impl(L, x, w_router, corr_bias, tw, ti, sg, workspace, s));
   SideStream* side = (L.dtype == MOE_BF16 && L.S > 0) ? side_stream() : nullptr;
+  int32_t* status = region<int32_t>(workspace, w.status);
+  void* h = region<void>(workspace, w.h);
   if (side != nullptr) {
     std::lock_guard<std::mutex> lock(g_side_mutex);
     MOE_TRY(cuda_status(cudaEventRecord(side->fork, s)));
     MOE_TRY(cuda_status(cudaStreamWaitEvent(side->stream, side->fork, 0)));
-    // the shared groups alone (E = 0, k = 0), their h rows after the routed ones
+    // the shared groups' gate_up alone (E = 0, k = 0), their h rows after
+    // the routed ones
     Layer Ls = L;
     Ls.E = 0;
     Ls.k = 0;
-    void* h_shared = static_cast<uint8_t*>(region<void>(workspace, w.h)) +
-                     static_cast<size_t>(L.T) * L.k * L.I * 2;
+    void* h_shared = static_cast<uint8_t*>(h) + static_cast<size_t>(L.T) * L.k * L.I * 2;
+    FfnTiling gate_up_only;
+    gate_up_only.part = 1;
     bool map_error = false;
     const cudaError_t e = launch_expert_ffn_bf16(Ls, x, x, nullptr, nullptr, nullptr, sg, nullptr,
                                                  nullptr, ws_gate_up, ws_down, h_shared, y_shared,
-                                                 y_shared, region<int32_t>(workspace, w.status),
-                                                 num_sms(), side->stream, &map_error);
+                                                 y_shared, status, num_sms(), side->stream,
+                                                 &map_error, gate_up_only);
     if (map_error) return MOE_ERR_INVALID_ARG;
     MOE_TRY(cuda_status(e));
     MOE_TRY(cuda_status(cudaEventRecord(side->join, side->stream)));
@@ -303,17 +307,34 @@ moe_status_t forward_checked(const moe_layer_desc_t* desc, const void* x, const 
   // row-gathering mode, x_perm = null, issues one TMA per 4 rows and runs
   // slower once tiles are full)
   MOE_TRY(permute_impl(L, ti, padding_mask, x, offsets, perm_slot, inv_perm, x_perm, workspace, s));
-  Layer Lr = L;
-  if (side != nullptr) Lr.S = 0;   // the routed groups only: the shared ones run on the side stream
-  MOE_TRY(ffn_launch(Lr, x, x_perm, offsets, perm_slot, tw, sg, w_gate_up, w_down, ws_gate_up,
-                     ws_down, y_routed, y_shared, region<void>(workspace, w.h),
-                     region<int32_t>(workspace, w.status), s));
-  if (side != nullptr) {
-    std::lock_guard<std::mutex> lock(g_side_mutex);
-    MOE_TRY(cuda_status(cudaStreamWaitEvent(s, side->join, 0)));
+  if (side == nullptr) {
+    MOE_TRY(ffn_launch(L, x, x_perm, offsets, perm_slot, tw, sg, w_gate_up, w_down, ws_gate_up,
+                       ws_down, y_routed, y_shared, h, status, s));
+  } else {
+    // the routed groups' gate_up; then, once the shared gate_up has joined,
+    // one down projection over all groups (routed and shared rows of h)
+    Layer Lr = L;
+    Lr.S = 0;
+    FfnTiling gate_up_only, down_only;
+    gate_up_only.part = 1;
+    down_only.part = 2;
+    bool map_error = false;
+    cudaError_t e = launch_expert_ffn_bf16(Lr, x, x_perm, offsets, perm_slot, tw, sg, w_gate_up,
+                                           w_down, ws_gate_up, ws_down, h, y_routed, y_shared,
+                                           status, num_sms(), s, &map_error, gate_up_only);
+    if (map_error) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(cuda_status(e));
+    {
+      std::lock_guard<std::mutex> lock(g_side_mutex);
+      MOE_TRY(cuda_status(cudaStreamWaitEvent(s, side->join, 0)));
+    }
+    e = launch_expert_ffn_bf16(L, x, x_perm, offsets, perm_slot, tw, sg, w_gate_up, w_down,
+                               ws_gate_up, ws_down, h, y_routed, y_shared, status, num_sms(), s,
+                               &map_error, down_only);
+    if (map_error) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(cuda_status(e));
   }
-  return cuda_status(launch_combine(L, y_routed, y_shared, inv_perm, out,
-                                    region<int32_t>(workspace, w.status), num_sms(), s));
+  return cuda_status(launch_combine(L, y_routed, y_shared, inv_perm, out, status, num_sms(), s));
 }
 
 // ------------------------------------------------------------ dense layer
@@ -637,8 +658,9 @@ int32_t moe_forward_kernel_count(const moe_layer_desc_t* desc) {
   // a partial-logit sum when K is split 4 or more ways); permute: chunk
   // counts, chunk scan, scatter, row gather; experts: gate_up + down (bf16
   // with T > 128: CTA-pair launch + single-CTA launch each; bf16 with shared
-  // experts: their gate_up + down on the side stream too); combine.
-  const int experts = L.dtype == MOE_BF16 ? (L.T > 128 ? 4 : 2) + (L.S > 0 ? 2 : 0) : 2;
+  // experts: their gate_up on the side stream too, their down in the routed
+  // experts' down launches); combine.
+  const int experts = L.dtype == MOE_BF16 ? (L.T > 128 ? 4 : 2) + (L.S > 0 ? 1 : 0) : 2;
   return (L.dtype == MOE_BF16 ? 2 : 1) + router_topk_launches(router_ksplit(L)) + 4 + experts + 1;
 }
 

@@ -56,8 +56,9 @@ def test_workspace_size_covers_intermediates(w):
     need = el * (Rk * w.H + (Rk + w.S * w.T) * w.I) + 4 * (Rk + w.S * w.T) * w.H
     assert n >= need
     # bf16: gate_up and down as CTA-pair + single-CTA launches (T > 128), and
-    # with shared experts their own gate_up + down on moe_forward's side stream
-    experts = ((4 if w.T > 128 else 2) + (2 if w.S else 0)) if w.dtype == "bf16" else 2
+    # with shared experts their own gate_up on moe_forward's side stream (their
+    # down joins the routed experts' down launches)
+    experts = ((4 if w.T > 128 else 2) + (1 if w.S else 0)) if w.dtype == "bf16" else 2
     # tensor-core router: K split across ~148 CTAs when T is small; from 4
     # splits on a separate kernel sums the partial logits before the top-k
     ksplit = 1
