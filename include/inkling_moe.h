@@ -51,6 +51,12 @@
  *     region are the expert GEMMs' tile counters, which every call that uses
  *     them zeroes itself on its stream.
  *   - Calls sharing one workspace must be ordered on one stream.
+ *   - Kernels are launched with programmatic stream serialisation: a
+ *     kernel's CTAs may start while the kernel before it on the stream
+ *     (this library's or the caller's) is still finishing, but they read and
+ *     write global memory only after that kernel has completed and its
+ *     writes are visible.  Stream order is therefore exactly that of plain
+ *     launches; only the launch latency and each kernel's set-up overlap.
  */
 #ifndef INKLING_MOE_H
 #define INKLING_MOE_H

@@ -52,6 +52,8 @@ __global__ void __launch_bounds__(256)
     combine_kernel(const TR* __restrict__ y_routed, const TR* __restrict__ y_shared,
                    const int32_t* __restrict__ inv_perm, TY* __restrict__ out, int64_t T, int H,
                    int k, int S, int64_t rows_cap, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int V = 16 / sizeof(TY);   // one 16-byte output store per vector
   __shared__ int s_rows[32];
   const int nv = H / V;
@@ -93,6 +95,8 @@ __global__ void __launch_bounds__(256)
     combine_rows_kernel(const TR* __restrict__ y_routed, const TR* __restrict__ y_shared,
                         const int32_t* __restrict__ inv_perm, __nv_bfloat16* __restrict__ out,
                         int64_t T, int H, int k, int S, int64_t rows_cap, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int kRowBatch = sizeof(TR) == 2 ? 4 : 2;
   constexpr int LPV = sizeof(TR) == 2 ? 1 : 2;   // 16-byte loads per vector of 8 values
   __shared__ const TR* s_src[2][32];   // a token's rows: S shared, then k routed (or null)
@@ -176,18 +180,16 @@ __global__ void __launch_bounds__(256)
 // bf16 output from rows of TR: vectors a thread sized to cover the row in
 // one pass of 256 threads, at most 4 (longer rows take several passes)
 template <typename TR>
-void launch_rows(unsigned grid, cudaStream_t stream, const TR* yr, const TR* ys,
-                 const int32_t* inv_perm, __nv_bfloat16* o, const Layer& L, int64_t cap,
-                 int32_t* status) {
+cudaError_t launch_rows(unsigned grid, cudaStream_t stream, const TR* yr, const TR* ys,
+                        const int32_t* inv_perm, __nv_bfloat16* o, const Layer& L, int64_t cap,
+                        int32_t* status) {
   const int nv = L.H / 8;
-  if (nv <= 256)
-    combine_rows_kernel<TR, 1><<<grid, 256, 0, stream>>>(yr, ys, inv_perm, o, L.T, L.H, L.k, L.S, cap, status);
-  else if (nv <= 512)
-    combine_rows_kernel<TR, 2><<<grid, 256, 0, stream>>>(yr, ys, inv_perm, o, L.T, L.H, L.k, L.S, cap, status);
-  else if (nv <= 768)
-    combine_rows_kernel<TR, 3><<<grid, 256, 0, stream>>>(yr, ys, inv_perm, o, L.T, L.H, L.k, L.S, cap, status);
-  else
-    combine_rows_kernel<TR, 4><<<grid, 256, 0, stream>>>(yr, ys, inv_perm, o, L.T, L.H, L.k, L.S, cap, status);
+  auto* kernel = nv <= 256   ? combine_rows_kernel<TR, 1>
+                 : nv <= 512 ? combine_rows_kernel<TR, 2>
+                 : nv <= 768 ? combine_rows_kernel<TR, 3>
+                             : combine_rows_kernel<TR, 4>;
+  return launch_chained(kernel, grid, 256, 0, stream, yr, ys, inv_perm, o, L.T, L.H, L.k, L.S,
+                        cap, status);
 }
 
 }  // namespace
@@ -200,16 +202,14 @@ cudaError_t launch_combine(const Layer& L, const void* y_routed, const void* y_s
   const int64_t cap = L.T * L.k;
   auto* o = static_cast<__nv_bfloat16*>(out);
   if (L.dtype == MOE_BF16 && L.y_f16)
-    launch_rows(grid, stream, static_cast<const __half*>(y_routed),
-                static_cast<const __half*>(y_shared), inv_perm, o, L, cap, status);
-  else if (L.dtype == MOE_BF16)
-    launch_rows(grid, stream, static_cast<const float*>(y_routed),
-                static_cast<const float*>(y_shared), inv_perm, o, L, cap, status);
-  else
-    combine_kernel<float, float><<<grid, 256, 0, stream>>>(
-        static_cast<const float*>(y_routed), static_cast<const float*>(y_shared), inv_perm,
-        static_cast<float*>(out), L.T, L.H, L.k, L.S, cap, status);
-  return cudaGetLastError();
+    return launch_rows(grid, stream, static_cast<const __half*>(y_routed),
+                       static_cast<const __half*>(y_shared), inv_perm, o, L, cap, status);
+  if (L.dtype == MOE_BF16)
+    return launch_rows(grid, stream, static_cast<const float*>(y_routed),
+                       static_cast<const float*>(y_shared), inv_perm, o, L, cap, status);
+  return launch_chained(combine_kernel<float, float>, grid, 256, 0, stream,
+                        static_cast<const float*>(y_routed), static_cast<const float*>(y_shared),
+                        inv_perm, static_cast<float*>(out), L.T, L.H, L.k, L.S, cap, status);
 }
 
 }  // namespace moe

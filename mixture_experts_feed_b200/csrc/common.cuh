@@ -56,4 +56,37 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi, bool& overflo
 
 __host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Programmatic dependent launch.  The layer's kernels are launched with
+// programmatic stream serialisation (launch_chained): a kernel's CTAs may
+// start while the previous kernel on the stream is still finishing, so the
+// launch latency and the kernel's own setup overlap that kernel's tail.
+// Until pdl_wait() a kernel touches no global memory other than its
+// parameters (it initialises shared-memory barriers, allocates tensor
+// memory, prefetches tensor maps); pdl_wait() returns once the previous grid
+// has completed and its writes are visible, so every read of an earlier
+// result and every global write (including writes to buffers an earlier
+// kernel reads) comes after it.  pdl_trigger() lets the next kernel be
+// scheduled once every CTA of this one has called it or exited.  Launched
+// without the attribute, pdl_wait() returns at once.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                           cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 }  // namespace moe

@@ -42,6 +42,8 @@ __global__ void __launch_bounds__(SB_THREADS) grouped_gemm_simt_kernel(const Sim
   const int n_tiles = (p.N + SB_N - 1) / SB_N;
   const int tid = threadIdx.x;
   if (tid == 0) s_bad = 0;
+  pdl_wait();
+  pdl_trigger();
   __syncthreads();
   if (tid < 32) build_tile_prefix(p.offsets, p.E, p.S, p.T, kAllTiles, SB_M, n_tiles, p.rows_cap, s_off, s_tile, &s_bad);
   __syncthreads();
@@ -159,8 +161,8 @@ cudaError_t launch_expert_ffn_f32(const Layer& L, const void* x, const void* x_p
   g.T = L.T; g.a1_base = 0; g.a1_stride = 0;
   g.E = L.E; g.S = L.S; g.K = L.H; g.N = 2 * L.I; g.ld_out = L.I;
   g.rows_cap = static_cast<int>(Rk);
-  grouped_gemm_simt_kernel<true><<<grid, SB_THREADS, tables, stream>>>(g);
-  cudaError_t e = cudaGetLastError();
+  const cudaError_t e =
+      launch_chained(grouped_gemm_simt_kernel<true>, grid, SB_THREADS, tables, stream, g);
   if (e != cudaSuccess) return e;
 
   SimtParams d{};
@@ -176,8 +178,7 @@ cudaError_t launch_expert_ffn_f32(const Layer& L, const void* x, const void* x_p
   d.T = L.T; d.a1_base = Rk; d.a1_stride = L.T;
   d.E = L.E; d.S = L.S; d.K = L.I; d.N = L.H; d.ld_out = L.H;
   d.rows_cap = static_cast<int>(Rk);
-  grouped_gemm_simt_kernel<false><<<grid, SB_THREADS, tables, stream>>>(d);
-  return cudaGetLastError();
+  return launch_chained(grouped_gemm_simt_kernel<false>, grid, SB_THREADS, tables, stream, d);
 }
 
 }  // namespace moe

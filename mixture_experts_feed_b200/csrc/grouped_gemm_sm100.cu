@@ -313,8 +313,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_relinquish();
     }
   } else if (warp == 2) {
+    pdl_wait();
     build_tile_prefix(p.offsets, p.E, p.S, p.T, SET, BM, n_tiles, p.rows_cap, s_off, s_tile, s_bad);
   }
+  // The setup above (barriers, tensor memory, tensor-map prefetch) may run
+  // while the previous kernel on the stream finishes; every global access
+  // below comes after it has completed.
+  pdl_wait();
   tc_fence_before();
   __syncthreads();
   if (PAIR) cluster_sync();   // both CTAs' barriers exist before any cross-CTA signal
@@ -492,6 +497,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok) break;
     }
+    // no more loads from this CTA: the next kernel on the stream may be
+    // scheduled (its CTAs take an SM once one of this launch's CTAs exits)
+    pdl_trigger();
     // Wait (bounded) until the last load issued on every stage has landed,
     // so that no copy still writes shared memory when the block exits.  A
     // pair's loads all complete on the rank-0 CTA's barriers; the other CTA
@@ -881,22 +889,22 @@ static cudaError_t launch_mode(const GemmParams& p, int sms, cudaStream_t stream
       }
     }
   }
-  if (!PAIR) {
-    grouped_gemm_kernel<MODE, PAIR><<<sms, NUM_THREADS, smem, stream>>>(p);
-    return cudaGetLastError();
-  }
+  // programmatic stream serialisation (see pdl_wait), and CTA pairs as
+  // clusters of two
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);   // whole pairs
+  cfg.gridDim = dim3(static_cast<unsigned>(PAIR ? (sms & ~1) : sms), 1, 1);   // whole pairs
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = PAIR ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, PAIR>, p);
 }
 

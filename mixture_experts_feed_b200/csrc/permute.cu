@@ -35,6 +35,8 @@ namespace {
 __global__ void perm_count_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ pad,
                                   int64_t T, int k, int E, int32_t* __restrict__ counts,
                                   int32_t* __restrict__ inv_perm, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int s_hist[];
   for (int i = threadIdx.x; i < E; i += blockDim.x) s_hist[i] = 0;
   __syncthreads();
@@ -62,6 +64,8 @@ __global__ void perm_count_kernel(const int32_t* __restrict__ idx, const uint8_t
 // Exclusive scan of counts[0..E) by one block of 1024 threads (E <= 1024).
 __global__ void __launch_bounds__(1024)
     perm_scan_kernel(const int32_t* __restrict__ counts, int E, int32_t* __restrict__ offsets) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int s_warp[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int v = tid < E ? counts[tid] : 0;
@@ -119,6 +123,8 @@ __device__ __forceinline__ int block_excl_scan_256(int v, int* s_warp, int& tota
 __global__ void __launch_bounds__(256)
     perm_chunk_scan_kernel(const int32_t* __restrict__ counts, int E, int n_chunks,
                            int32_t* __restrict__ offsets, int32_t* __restrict__ chunk) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int s_warp[8];
   const int e = blockIdx.x;
   int part = 0;
@@ -156,6 +162,8 @@ __global__ void __launch_bounds__(256)
                             int64_t slots, int k, int E, int64_t cs,
                             int32_t* __restrict__ counts, int32_t* __restrict__ chunk,
                             int32_t* __restrict__ inv_perm, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int s_hist[];
   for (int i = threadIdx.x; i < E; i += blockDim.x) s_hist[i] = 0;
   __syncthreads();
@@ -192,6 +200,8 @@ __global__ void __launch_bounds__(256)
                         int64_t slots, int k, int E, int64_t cs,
                         const int32_t* __restrict__ chunk, int32_t* __restrict__ perm_slot,
                         int32_t* __restrict__ inv_perm, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int s_mem[];
   int* s_cnt = s_mem;              // [8 warps][E]
   int* s_base = s_mem + 8 * E;     // [E]
@@ -240,6 +250,8 @@ __global__ void __launch_bounds__(COMPACT_THREADS)
     perm_compact_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ pad,
                         int64_t T, int k, const int32_t* __restrict__ offsets,
                         int32_t* __restrict__ perm_slot, int32_t* __restrict__ inv_perm) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int s_warp[32];
   __shared__ int s_total;
   const int e = blockIdx.x;
@@ -294,6 +306,8 @@ template <typename TX>
 __global__ void gather_rows_kernel(const TX* __restrict__ x, const int32_t* __restrict__ perm_slot,
                                    const int32_t* __restrict__ offsets, int E, int k, int H,
                                    int64_t slots, TX* __restrict__ x_perm, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   const int R = offsets[E];
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -346,34 +360,36 @@ cudaError_t launch_permute(const Layer& L, const int32_t* topk_idx, const uint8_
   if (chunk != nullptr) {
     const int64_t cs = permute_chunk_slots(slots);
     const int nc = static_cast<int>(permute_chunks(slots));
-    perm_chunk_count_kernel<<<nc, 256, sizeof(int) * L.E, stream>>>(
-        topk_idx, padding_mask, slots, L.k, L.E, cs, counts, chunk, inv_perm, status);
-    perm_chunk_scan_kernel<<<L.E, 256, 0, stream>>>(counts, L.E, nc, offsets, chunk);
-    perm_scatter_kernel<<<nc, 256, sizeof(int) * 9 * L.E, stream>>>(
-        topk_idx, padding_mask, slots, L.k, L.E, cs, chunk, perm_slot, inv_perm, status);
+    err = launch_chained(perm_chunk_count_kernel, nc, 256, sizeof(int) * L.E, stream, topk_idx,
+                         padding_mask, slots, L.k, L.E, cs, counts, chunk, inv_perm, status);
+    if (err == cudaSuccess)
+      err = launch_chained(perm_chunk_scan_kernel, L.E, 256, 0, stream, counts, L.E, nc, offsets,
+                           chunk);
+    if (err == cudaSuccess)
+      err = launch_chained(perm_scatter_kernel, nc, 256, sizeof(int) * 9 * L.E, stream, topk_idx,
+                           padding_mask, slots, L.k, L.E, cs, chunk, perm_slot, inv_perm, status);
   } else {
     const int threads = 256;
     const unsigned cgrid = static_cast<unsigned>(
         std::min<int64_t>(ceil_div(L.T, threads), static_cast<int64_t>(num_sms) * 4));
-    perm_count_kernel<<<cgrid, threads, sizeof(int) * L.E, stream>>>(topk_idx, padding_mask, L.T,
-                                                                     L.k, L.E, counts, inv_perm,
-                                                                     status);
-    perm_scan_kernel<<<1, 1024, 0, stream>>>(counts, L.E, offsets);
-    perm_compact_kernel<<<L.E, COMPACT_THREADS, 0, stream>>>(topk_idx, padding_mask, L.T, L.k,
-                                                             offsets, perm_slot, inv_perm);
+    err = launch_chained(perm_count_kernel, cgrid, threads, sizeof(int) * L.E, stream, topk_idx,
+                         padding_mask, L.T, L.k, L.E, counts, inv_perm, status);
+    if (err == cudaSuccess)
+      err = launch_chained(perm_scan_kernel, 1, 1024, 0, stream, counts, L.E, offsets);
+    if (err == cudaSuccess)
+      err = launch_chained(perm_compact_kernel, L.E, COMPACT_THREADS, 0, stream, topk_idx,
+                           padding_mask, L.T, L.k, offsets, perm_slot, inv_perm);
   }
-  if (x_perm == nullptr) return cudaGetLastError();   // rows are gathered by the consumer
+  if (err != cudaSuccess || x_perm == nullptr) return err;   // x_perm null: the consumer gathers
   const unsigned ggrid = static_cast<unsigned>(
       std::min<int64_t>(ceil_div(slots, 8), static_cast<int64_t>(num_sms) * 8));
   if (L.dtype == MOE_BF16)
-    gather_rows_kernel<__nv_bfloat16><<<ggrid, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(x), perm_slot, offsets, L.E, L.k, L.H, slots,
-        static_cast<__nv_bfloat16*>(x_perm), status);
-  else
-    gather_rows_kernel<float><<<ggrid, 256, 0, stream>>>(static_cast<const float*>(x), perm_slot,
-                                                         offsets, L.E, L.k, L.H, slots,
-                                                         static_cast<float*>(x_perm), status);
-  return cudaGetLastError();
+    return launch_chained(gather_rows_kernel<__nv_bfloat16>, ggrid, 256, 0, stream,
+                          static_cast<const __nv_bfloat16*>(x), perm_slot, offsets, L.E, L.k, L.H,
+                          slots, static_cast<__nv_bfloat16*>(x_perm), status);
+  return launch_chained(gather_rows_kernel<float>, ggrid, 256, 0, stream,
+                        static_cast<const float*>(x), perm_slot, offsets, L.E, L.k, L.H, slots,
+                        static_cast<float*>(x_perm), status);
 }
 
 }  // namespace moe

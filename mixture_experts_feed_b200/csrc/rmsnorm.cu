@@ -153,6 +153,8 @@ template <typename R>
 __global__ void __launch_bounds__(kThreads)
     rmsnorm_kernel(const void* x_, const void* __restrict__ w_, void* out_, int64_t T, int H,
                    double eps) {
+  pdl_wait();
+  pdl_trigger();
   using Vec = typename R::Vec;
   constexpr int B = RMS_BATCH;
   const Vec* x = static_cast<const Vec*>(x_);
@@ -208,6 +210,8 @@ template <typename R, int VPT>
 __global__ void __launch_bounds__(kThreads, 4)
     rmsnorm_rows_kernel(const void* x_, const void* __restrict__ w_, void* out_, int64_t T, int H,
                         double eps, int tpr_log2) {
+  pdl_wait();
+  pdl_trigger();
   using Vec = typename R::Vec;
   __shared__ double s_part[kThreads / 32];
   const Vec* x = static_cast<const Vec*>(x_);
@@ -283,13 +287,11 @@ cudaError_t launch_rows(int64_t T, int H, double eps, const void* x, const void*
   const int rpb = kThreads / tpr;
   const int64_t blocks = (T + rpb - 1) / rpb;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(blocks, static_cast<int64_t>(num_sms) * 4));
-  switch (vpt) {
-    case 1: rmsnorm_rows_kernel<R, 1><<<grid, kThreads, 0, stream>>>(x, weight, out, T, H, eps, tpr_log2); break;
-    case 2: rmsnorm_rows_kernel<R, 2><<<grid, kThreads, 0, stream>>>(x, weight, out, T, H, eps, tpr_log2); break;
-    case 3: rmsnorm_rows_kernel<R, 3><<<grid, kThreads, 0, stream>>>(x, weight, out, T, H, eps, tpr_log2); break;
-    default: rmsnorm_rows_kernel<R, 4><<<grid, kThreads, 0, stream>>>(x, weight, out, T, H, eps, tpr_log2); break;
-  }
-  return cudaGetLastError();
+  auto* kernel = vpt == 1   ? rmsnorm_rows_kernel<R, 1>
+                 : vpt == 2 ? rmsnorm_rows_kernel<R, 2>
+                 : vpt == 3 ? rmsnorm_rows_kernel<R, 3>
+                            : rmsnorm_rows_kernel<R, 4>;
+  return launch_chained(kernel, grid, kThreads, 0, stream, x, weight, out, T, H, eps, tpr_log2);
 }
 
 }  // namespace
@@ -306,11 +308,8 @@ cudaError_t launch_rmsnorm(int64_t T, int H, int dtype, float eps, const void* x
   const int64_t blocks = (T + kThreads / 32 - 1) / (kThreads / 32);
   const unsigned grid = static_cast<unsigned>(
       std::min<int64_t>(blocks, static_cast<int64_t>(num_sms) * RMS_BLOCKS_PER_SM));
-  if (dtype == MOE_BF16)
-    rmsnorm_kernel<Bf16Row><<<grid, kThreads, 0, stream>>>(x, weight, out, T, H, eps);
-  else
-    rmsnorm_kernel<F32Row><<<grid, kThreads, 0, stream>>>(x, weight, out, T, H, eps);
-  return cudaGetLastError();
+  return launch_chained(dtype == MOE_BF16 ? rmsnorm_kernel<Bf16Row> : rmsnorm_kernel<F32Row>, grid,
+                        kThreads, 0, stream, x, weight, out, T, H, static_cast<double>(eps));
 }
 
 }  // namespace moe

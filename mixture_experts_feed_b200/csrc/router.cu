@@ -58,6 +58,8 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
 // three parts is zero for every finite fp32 input of normal range.
 __global__ void router_split_kernel(const float* __restrict__ w, __nv_bfloat16* __restrict__ parts,
                                     int64_t n) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
     const float v = w[i];
@@ -77,6 +79,8 @@ __global__ void __launch_bounds__(RL_THREADS)
                          float* __restrict__ z, int64_t T, int H, int NE, int ld) {
   __shared__ __align__(16) float As[RL_BK][RL_BM + 4];
   __shared__ __align__(16) float Bs[RL_BK][RL_BN + 4];
+  pdl_wait();
+  pdl_trigger();
   const int tid = threadIdx.x;
   const int64_t m0 = static_cast<int64_t>(blockIdx.x) * RL_BM;
   const int n0 = blockIdx.y * RL_BN;
@@ -148,6 +152,8 @@ constexpr int kSumSplitsFrom = 4;
 // split count is large (few tokens): there the top-k kernel has few warps.
 __global__ void router_sum_splits_kernel(float* __restrict__ z, int ld, int ksplit, int64_t T,
                                          int NE) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t split = T * static_cast<int64_t>(ld);
   const int64_t n = T * static_cast<int64_t>(NE);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -168,6 +174,8 @@ __global__ void __launch_bounds__(TK_WARPS * 32)
                        float* __restrict__ topk_w, int32_t* __restrict__ topk_idx,
                        float* __restrict__ gamma) {
   __shared__ int s_chosen[TK_WARPS][32];
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * TK_WARPS + warp;
   if (t >= T) return;
@@ -237,8 +245,8 @@ cudaError_t launch_router_split(const Layer& L, const float* w_router, void* w_p
                                 int num_sms, cudaStream_t stream) {
   const int64_t n = static_cast<int64_t>(L.E + L.S) * L.H;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ceil_div(n, 256), num_sms * 8));
-  router_split_kernel<<<grid, 256, 0, stream>>>(w_router, static_cast<__nv_bfloat16*>(w_parts), n);
-  return cudaGetLastError();
+  return launch_chained(router_split_kernel, grid, 256, 0, stream, w_router,
+                        static_cast<__nv_bfloat16*>(w_parts), n);
 }
 
 cudaError_t launch_router_logits(const Layer& L, const void* x, const float* w_router,
@@ -246,12 +254,10 @@ cudaError_t launch_router_logits(const Layer& L, const void* x, const float* w_r
   const int NE = L.E + L.S;
   dim3 grid(static_cast<unsigned>(ceil_div(L.T, RL_BM)), static_cast<unsigned>(ceil_div(NE, RL_BN)));
   if (L.dtype == MOE_BF16)
-    router_logits_kernel<__nv_bfloat16><<<grid, RL_THREADS, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(x), w_router, logits, L.T, L.H, NE, ld);
-  else
-    router_logits_kernel<float><<<grid, RL_THREADS, 0, stream>>>(static_cast<const float*>(x),
-                                                                 w_router, logits, L.T, L.H, NE, ld);
-  return cudaGetLastError();
+    return launch_chained(router_logits_kernel<__nv_bfloat16>, grid, RL_THREADS, 0, stream,
+                          static_cast<const __nv_bfloat16*>(x), w_router, logits, L.T, L.H, NE, ld);
+  return launch_chained(router_logits_kernel<float>, grid, RL_THREADS, 0, stream,
+                        static_cast<const float*>(x), w_router, logits, L.T, L.H, NE, ld);
 }
 
 int router_topk_launches(int ksplit) { return ksplit >= kSumSplitsFrom ? 2 : 1; }
@@ -263,28 +269,26 @@ cudaError_t launch_router_topk(const Layer& L, const float* logits, int ld, int 
     const int NE = L.E + L.S;
     const int64_t n = L.T * static_cast<int64_t>(NE);
     const unsigned sgrid = static_cast<unsigned>(std::min<int64_t>(ceil_div(n, 256), 148 * 8));
-    router_sum_splits_kernel<<<sgrid, 256, 0, stream>>>(const_cast<float*>(logits), ld, ksplit,
-                                                        L.T, NE);
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch_chained(router_sum_splits_kernel, sgrid, 256, 0, stream,
+                                         const_cast<float*>(logits), ld, ksplit, L.T, NE);
     if (e != cudaSuccess) return e;
     ksplit = 1;
   }
   const unsigned grid = static_cast<unsigned>(ceil_div(L.T, TK_WARPS));
   const float scale = L.route_scale * L.global_scale;
   const int pl = static_cast<int>(ceil_div(L.E, 32));
-#define MOE_TOPK(PLV)                                                                         \
-  router_topk_kernel<PLV><<<grid, TK_WARPS * 32, 0, stream>>>(logits, ld, ksplit, corr_bias, L.T, \
-                                                              L.E, L.k,                        \
-                                                              L.S, scale, topk_w, topk_idx,     \
-                                                              shared_gamma)
-  if (pl <= 1) MOE_TOPK(1);
-  else if (pl <= 2) MOE_TOPK(2);
-  else if (pl <= 4) MOE_TOPK(4);
-  else if (pl <= 8) MOE_TOPK(8);
-  else if (pl <= 16) MOE_TOPK(16);
-  else MOE_TOPK(32);
+#define MOE_TOPK(PLV)                                                                       \
+  launch_chained(router_topk_kernel<PLV>, grid, TK_WARPS * 32, 0, stream, logits, ld, ksplit, \
+                 corr_bias, L.T, L.E, L.k, L.S, scale, topk_w, topk_idx, shared_gamma)
+  cudaError_t e;
+  if (pl <= 1) e = MOE_TOPK(1);
+  else if (pl <= 2) e = MOE_TOPK(2);
+  else if (pl <= 4) e = MOE_TOPK(4);
+  else if (pl <= 8) e = MOE_TOPK(8);
+  else if (pl <= 16) e = MOE_TOPK(16);
+  else e = MOE_TOPK(32);
 #undef MOE_TOPK
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace moe

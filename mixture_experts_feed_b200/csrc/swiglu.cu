@@ -25,6 +25,8 @@ namespace {
 __global__ void swiglu_partials_kernel(const float* __restrict__ part, int ksplit, int64_t T,
                                        int I, float w, int f16, uint16_t* __restrict__ h,
                                        int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   const int groups = I / 4;
   const int64_t n = T * groups;
   const int64_t split = T * static_cast<int64_t>(2 * I);
@@ -66,9 +68,8 @@ cudaError_t launch_swiglu_partials(const float* part, int ksplit, int64_t T, int
   const int64_t n = T * (I / 4);
   const unsigned grid = static_cast<unsigned>(
       std::max<int64_t>(1, std::min<int64_t>(ceil_div(n, 256), static_cast<int64_t>(num_sms) * 8)));
-  swiglu_partials_kernel<<<grid, 256, 0, stream>>>(part, ksplit, T, I, w, f16 ? 1 : 0,
-                                                   static_cast<uint16_t*>(h), status);
-  return cudaGetLastError();
+  return launch_chained(swiglu_partials_kernel, grid, 256, 0, stream, part, ksplit, T, I, w,
+                        f16 ? 1 : 0, static_cast<uint16_t*>(h), status);
 }
 
 }  // namespace moe
