@@ -47,11 +47,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // Two fp32 values rounded to nearest fp16; `overflow` is set when either
-// rounds to an infinity (|v| at or beyond 65520) or is not finite.
+// rounds to an infinity (|v| at or beyond 65520) or is not finite: an fp16
+// whose exponent field is all ones.  Branch-free (one per-halfword compare),
+// since epilogues pack dozens of values between two tensor-memory loads.
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi, bool& overflow) {
   const __half2 h = __floats2half2_rn(lo, hi);
-  if (__hisinf(h.x) || __hisinf(h.y) || __hisnan(h.x) || __hisnan(h.y)) overflow = true;
-  return *reinterpret_cast<const uint32_t*>(&h);
+  const uint32_t u = *reinterpret_cast<const uint32_t*>(&h);
+  overflow |= __vcmpeq2(u & 0x7C007C00u, 0x7C007C00u) != 0u;
+  return u;
 }
 
 __host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }

@@ -743,8 +743,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const float u0 = __uint_as_float(v[4 * i + 1]);
             const float g1 = __uint_as_float(v[4 * i + 2]);
             const float u1 = __uint_as_float(v[4 * i + 3]);
-            const float h0 = w * (g0 / (1.0f + __expf(-g0))) * u0;
-            const float h1 = w * (g1 / (1.0f + __expf(-g1))) * u1;
+            // silu(g) = g / (1 + e^-g) with the fast division (2 ulp): the
+            // product is rounded to bf16 or fp16 right after
+            const float h0 = w * __fdividef(g0, 1.0f + __expf(-g0)) * u0;
+            const float h1 = w * __fdividef(g1, 1.0f + __expf(-g1)) * u1;
             // fp16 down projections: h rounded to fp16 (8x finer than bf16)
             packed[i] = p.f16 ? pack_f16x2(h0, h1, h_overflow) : pack_bf16x2(h0, h1);
           }

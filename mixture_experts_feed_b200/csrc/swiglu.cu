@@ -46,7 +46,7 @@ __global__ void swiglu_partials_kernel(const float* __restrict__ part, int kspli
     const float g[4] = {a.x, a.z, b.x, b.z}, u[4] = {a.y, a.w, b.y, b.w};
     float v[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) v[q] = w * (g[q] / (1.0f + __expf(-g[q]))) * u[q];
+    for (int q = 0; q < 4; ++q) v[q] = w * __fdividef(g[q], 1.0f + __expf(-g[q])) * u[q];
     uint2 o;
     if (f16) {
       o.x = pack_f16x2(v[0], v[1], ovf);
