@@ -56,9 +56,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # measurement of this run: each entry names its capture.  An entry is removed
 # when the kernels change, until it is captured again.
 NCU_TRAFFIC_BYTES = {
-    "bf16-T8192-H6144-E128k8S1-I2048": (12650326272, "ncu capture of 2026-12-03 (the four launches of "
+    "bf16-T8192-H6144-E128k8S1-I2048": (12736334592, "ncu capture of 2026-12-03 (the four launches of "
                                         "one moe_expert_ffn call of the op chain, fp16 down "
-                                        "projections, gate_up pair tiles drawn from a counter), "
+                                        "projections, gate_up pair tiles drawn from a counter, "
+                                        "chained launches, branch-free fp16 packing), "
                                         "profiles/traffic_expert_gemms_bf16-T8192-H6144-E128k8S1-I2048.md"),
 }
 # The other workloads the benchmark spec states, timed in the same run as the default
