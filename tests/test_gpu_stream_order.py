@@ -187,3 +187,57 @@ def test_dense_calls_queued_back_to_back():
         assert moe.read_device_status(ws) == 0
         assert torch.equal(outs[0], ref["a"]) and torch.equal(outs[2], ref["a"])
         assert torch.equal(outs[1], ref["b"])
+
+
+def _replay_matches_eager(call, x_static, out, make_x):
+    """Capture call(x_static, out) in a CUDA graph, then replay it on new
+    inputs and compare each replay bitwise with the eager call."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        call(x_static, out)              # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call(x_static, out)
+    for i in range(3):
+        x_new = make_x(i)
+        x_static.copy_(x_new)
+        g.replay()
+        eager = torch.empty_like(out)
+        call(x_new, eager)
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager)
+    del g
+
+
+def test_chained_launches_in_cuda_graphs():
+    """The pre-norm layer (norm, then the side stream of moe_forward) and the
+    dense layer at T = 32 (K-split gate_up, SwiGLU pass, K-split down,
+    recombination: four chained launches) captured in CUDA graphs replay
+    with the eager calls' bits on new inputs."""
+    w, d, xb, L = _case(300, 256, 12, 3, 2, 320, "bf16")
+    gen = torch.Generator().manual_seed(36)
+    norm = (1.0 + 0.1 * torch.randn(w.H, generator=gen)).to(torch.bfloat16).cuda()
+    ws = moe.new_workspace(L)
+
+    def moe_call(x, o):
+        _forward(L, d, x, o, ws, norm)
+
+    _replay_matches_eager(moe_call, d["x"].clone(), torch.empty_like(d["x"]),
+                          lambda i: torch.randn(w.T, w.H, generator=gen).to(torch.bfloat16).cuda())
+    assert moe.read_device_status(ws) == 0
+
+    dw = mw.DenseWorkload(name="dense-bf16-T32-H4096-I1024", T=32, H=4096, I=1024, dtype="bf16",
+                          global_scale=1.0, seed=37, init_std=0.02)
+    dd = to_device(mw.generate_dense(dw, threads=4), down_f16=True)
+    DL = moe.DenseLayer.from_workload(dw, down_f16=True)
+    dws = moe.new_dense_workspace(DL)
+
+    def dense_call(x, o):
+        moe.moe_dense_mlp(DL, x, dd["w_gate_up"], dd["w_down"], o, dws)
+
+    _replay_matches_eager(dense_call, dd["x"].clone(), torch.empty_like(dd["x"]),
+                          lambda i: torch.randn(dw.T, dw.H, generator=gen).to(torch.bfloat16).cuda())
+    assert moe.read_device_status(dws) == 0
