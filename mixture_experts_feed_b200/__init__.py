@@ -200,6 +200,11 @@ def _expect(t: Optional[torch.Tensor], name: str, shape, dtype, allow_none=False
         raise ValueError(f"{name} must be contiguous")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    # the library launches on the current device: a buffer of another GPU
+    # would be read through peer memory, or fault
+    current = torch.cuda.current_device()
+    if t.device.index != current:
+        raise ValueError(f"{name} is on {t.device}, the current device is cuda:{current}")
 
 
 def workspace_size(layer: Layer) -> int:

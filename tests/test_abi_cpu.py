@@ -144,6 +144,20 @@ def test_binding_checks_shapes_on_host():
         moe.moe_combine(L, x, x, torch.zeros(8, dtype=torch.int32), x, torch.zeros(16, dtype=torch.uint8))
 
 
+def test_binding_rejects_a_buffer_of_another_device(monkeypatch):
+    """Every op launches on the current device; a tensor on another GPU is
+    rejected on the host (checked with a stand-in object: no GPU here)."""
+    from types import SimpleNamespace
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    other = SimpleNamespace(shape=(4, 128), dtype=torch.float32, is_contiguous=lambda: True,
+                            is_cuda=True, device=torch.device("cuda", 1))
+    with pytest.raises(ValueError, match="current device"):
+        moe._expect(other, "x", (4, 128), torch.float32)
+    same = SimpleNamespace(shape=(4, 128), dtype=torch.float32, is_contiguous=lambda: True,
+                           is_cuda=True, device=torch.device("cuda", 0))
+    moe._expect(same, "x", (4, 128), torch.float32)
+
+
 # ------------------------------------------------------------- dense layer
 def test_dense_desc_layout_and_sizes():
     assert ctypes.sizeof(moe.DenseDesc) == 24     # int64 + 3 x int32 + float
