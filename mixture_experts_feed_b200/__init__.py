@@ -207,6 +207,16 @@ def _expect(t: Optional[torch.Tensor], name: str, shape, dtype, allow_none=False
         raise ValueError(f"{name} is on {t.device}, the current device is cuda:{current}")
 
 
+def _wsptr(ws: torch.Tensor) -> int:
+    """Device address of a workspace (a contiguous CUDA byte tensor of the
+    current device)."""
+    if not isinstance(ws, torch.Tensor) or ws.dtype != torch.uint8 or not ws.is_contiguous():
+        raise ValueError("the workspace must be a contiguous torch.uint8 tensor")
+    if not ws.is_cuda or ws.device.index != torch.cuda.current_device():
+        raise ValueError(f"the workspace is on {ws.device}, not on the current CUDA device")
+    return ws.data_ptr()
+
+
 def workspace_size(layer: Layer) -> int:
     n = ctypes.c_size_t(0)
     _check(LIB.moe_workspace_size(ctypes.byref(layer.desc()), ctypes.byref(n)), "moe_workspace_size")
@@ -216,14 +226,14 @@ def workspace_size(layer: Layer) -> int:
 def new_workspace(layer: Layer, device=None, stream=None) -> torch.Tensor:
     """Allocate (with torch) and initialise a workspace for ``layer``."""
     ws = torch.empty(workspace_size(layer), dtype=torch.uint8, device=device or "cuda")
-    _check(LIB.moe_workspace_init(ws.data_ptr(), ws.numel(), _stream(stream)), "moe_workspace_init")
+    _check(LIB.moe_workspace_init(_wsptr(ws), ws.numel(), _stream(stream)), "moe_workspace_init")
     return ws
 
 
 def read_device_status(ws: torch.Tensor, stream=None) -> int:
     """Read and clear the device status word; raises MoEError when it is set."""
     code = ctypes.c_int32(0)
-    st = LIB.moe_read_device_status(ws.data_ptr(), _stream(stream), ctypes.byref(code))
+    st = LIB.moe_read_device_status(_wsptr(ws), _stream(stream), ctypes.byref(code))
     if st != 0:
         err = MoEError(st, f"device status 0x{code.value:x}")
         err.device_code = code.value
@@ -240,7 +250,7 @@ def moe_route(layer: Layer, x, w_router, corr_bias, topk_w, topk_idx, shared_gam
     _expect(topk_idx, "topk_idx", (L.T, L.k), torch.int32)
     _expect(shared_gamma, "shared_gamma", (L.T, L.S), torch.float32, allow_none=L.S == 0)
     _check(LIB.moe_route(ctypes.byref(L.desc()), _ptr(x), _ptr(w_router), _ptr(corr_bias),
-                         _ptr(topk_w), _ptr(topk_idx), _ptr(shared_gamma), ws.data_ptr(),
+                         _ptr(topk_w), _ptr(topk_idx), _ptr(shared_gamma), _wsptr(ws),
                          ws.numel(), _stream(stream)), "moe_route")
 
 
@@ -256,7 +266,7 @@ def moe_permute(layer: Layer, topk_idx, padding_mask, x, expert_offsets, perm_sl
     _expect(x_perm, "x_perm", (L.T * L.k, L.H), L.dtype, allow_none=True)   # None: no row copy
     _check(LIB.moe_permute(ctypes.byref(L.desc()), _ptr(topk_idx), _ptr(padding_mask), _ptr(x),
                            _ptr(expert_offsets), _ptr(perm_slot), _ptr(inv_perm), _ptr(x_perm),
-                           ws.data_ptr(), ws.numel(), _stream(stream)), "moe_permute")
+                           _wsptr(ws), ws.numel(), _stream(stream)), "moe_permute")
 
 
 def moe_permute_noalloc(layer: Layer, topk_idx, padding_mask, x, expert_offsets, perm_slot,
@@ -299,7 +309,7 @@ def moe_expert_ffn(layer: Layer, x, x_perm, expert_offsets, perm_slot, topk_w, s
     _check(LIB.moe_expert_ffn(ctypes.byref(L.desc()), _ptr(x), _ptr(x_perm), _ptr(expert_offsets),
                               _ptr(perm_slot), _ptr(topk_w), _ptr(shared_gamma), _ptr(w_gate_up),
                               _ptr(w_down), _ptr(ws_gate_up), _ptr(ws_down), _ptr(y_routed),
-                              _ptr(y_shared), ws.data_ptr(), ws.numel(), _stream(stream)),
+                              _ptr(y_shared), _wsptr(ws), ws.numel(), _stream(stream)),
            "moe_expert_ffn")
 
 
@@ -313,7 +323,7 @@ def moe_shared_ffn(layer: Layer, x, shared_gamma, ws_gate_up, ws_down, y_shared,
     _expect(ws_down, "ws_down", (L.S, L.H, L.I), L.down_dtype)
     _expect(y_shared, "y_shared", (L.S * L.T, L.H), L.y_dtype)
     _check(LIB.moe_shared_ffn(ctypes.byref(L.desc()), _ptr(x), _ptr(shared_gamma),
-                              _ptr(ws_gate_up), _ptr(ws_down), _ptr(y_shared), ws.data_ptr(),
+                              _ptr(ws_gate_up), _ptr(ws_down), _ptr(y_shared), _wsptr(ws),
                               ws.numel(), _stream(stream)), "moe_shared_ffn")
 
 
@@ -333,7 +343,7 @@ def moe_ep_dispatch_prep(layer: Layer, expert_offsets, perm_slot, topk_w, row_w,
     _expect(row_w, "row_w", (L.T * L.k,), torch.float32)
     _expect(expert_counts, "expert_counts", (L.E,), torch.int32)
     _check(LIB.moe_ep_dispatch_prep(ctypes.byref(L.desc()), _ptr(expert_offsets), _ptr(perm_slot),
-                                    _ptr(topk_w), _ptr(row_w), _ptr(expert_counts), ws.data_ptr(),
+                                    _ptr(topk_w), _ptr(row_w), _ptr(expert_counts), _wsptr(ws),
                                     ws.numel(), _stream(stream)), "moe_ep_dispatch_prep")
 
 
@@ -361,7 +371,7 @@ def moe_ep_dispatch_p2p(layer: Layer, x, topk_w, perm_slot, expert_offsets, dst_
     _ptr_table(dst_w, n_ranks, "dst_w")
     _check(LIB.moe_ep_dispatch_p2p(ctypes.byref(L.desc()), _ptr(x), _ptr(topk_w), _ptr(perm_slot),
                                    _ptr(expert_offsets), _ptr(dst_base), n_ranks, _ptr(dst_x),
-                                   _ptr(dst_w), dst_rows, ws.data_ptr(), ws.numel(),
+                                   _ptr(dst_w), dst_rows, _wsptr(ws), ws.numel(),
                                    _stream(stream)), "moe_ep_dispatch_p2p")
 
 
@@ -378,7 +388,7 @@ def moe_ep_return_p2p(layer: Layer, y_in, rows_in: int, run_start, src_base, n_r
     _expect(src_base, "src_base", (L.E,), torch.int32)
     _ptr_table(dst_y, n_ranks, "dst_y")
     _check(LIB.moe_ep_return_p2p(ctypes.byref(L.desc()), _ptr(y_in), rows_in, _ptr(run_start),
-                                 _ptr(src_base), n_ranks, _ptr(dst_y), dst_rows, ws.data_ptr(),
+                                 _ptr(src_base), n_ranks, _ptr(dst_y), dst_rows, _wsptr(ws),
                                  ws.numel(), _stream(stream)), "moe_ep_return_p2p")
 
 
@@ -389,7 +399,7 @@ def moe_combine(layer: Layer, y_routed, y_shared, inv_perm, out, ws, stream=None
     _expect(inv_perm, "inv_perm", (L.T * L.k,), torch.int32)
     _expect(out, "out", (L.T, L.H), L.dtype)
     _check(LIB.moe_combine(ctypes.byref(L.desc()), _ptr(y_routed), _ptr(y_shared), _ptr(inv_perm),
-                           _ptr(out), ws.data_ptr(), ws.numel(), _stream(stream)), "moe_combine")
+                           _ptr(out), _wsptr(ws), ws.numel(), _stream(stream)), "moe_combine")
 
 
 def moe_forward(layer: Layer, x, w_router, corr_bias, w_gate_up, w_down, ws_gate_up, ws_down,
@@ -411,7 +421,7 @@ def moe_forward(layer: Layer, x, w_router, corr_bias, w_gate_up, w_down, ws_gate
     _check(LIB.moe_forward(ctypes.byref(L.desc()), _ptr(x), _ptr(w_router), _ptr(corr_bias),
                            _ptr(w_gate_up), _ptr(w_down), _ptr(ws_gate_up), _ptr(ws_down),
                            _ptr(padding_mask), _ptr(out), _ptr(topk_w), _ptr(topk_idx),
-                           _ptr(shared_gamma), ws.data_ptr(), ws.numel(), _stream(stream)),
+                           _ptr(shared_gamma), _wsptr(ws), ws.numel(), _stream(stream)),
            "moe_forward")
 
 
@@ -454,7 +464,7 @@ def moe_forward_prenorm(layer: Layer, x, norm_weight, norm_eps, w_router, corr_b
     _check(LIB.moe_forward_prenorm(ctypes.byref(L.desc()), _ptr(x), _ptr(norm_weight), norm_eps,
                                    _ptr(w_router), _ptr(corr_bias), _ptr(w_gate_up), _ptr(w_down),
                                    _ptr(ws_gate_up), _ptr(ws_down), _ptr(padding_mask), _ptr(out),
-                                   _ptr(topk_w), _ptr(topk_idx), _ptr(shared_gamma), ws.data_ptr(),
+                                   _ptr(topk_w), _ptr(topk_idx), _ptr(shared_gamma), _wsptr(ws),
                                    ws.numel(), _stream(stream)), "moe_forward_prenorm")
 
 
@@ -467,7 +477,7 @@ def moe_dense_mlp_prenorm(layer: "DenseLayer", x, norm_weight, norm_eps, w_gate_
     _expect(w_down, "w_down", (L.H, L.I), L.down_dtype)
     _expect(out, "out", (L.T, L.H), L.dtype)
     _check(LIB.moe_dense_mlp_prenorm(ctypes.byref(L.desc()), _ptr(x), _ptr(norm_weight), norm_eps,
-                                     _ptr(w_gate_up), _ptr(w_down), _ptr(out), ws.data_ptr(),
+                                     _ptr(w_gate_up), _ptr(w_down), _ptr(out), _wsptr(ws),
                                      ws.numel(), _stream(stream)), "moe_dense_mlp_prenorm")
 
 
@@ -482,7 +492,7 @@ def dense_prenorm_kernel_count(layer: "DenseLayer") -> int:
 def selftest_wait_timeout(ws: torch.Tensor, limit_ms: int = 1000, stream=None) -> None:
     """Launch the stall-detection self-test (see the header); the next
     read_device_status() raises MoEError with MOE_ERR_TIMEOUT."""
-    _check(LIB.moe_selftest_wait_timeout(ws.data_ptr(), ws.numel(), limit_ms, _stream(stream)),
+    _check(LIB.moe_selftest_wait_timeout(_wsptr(ws), ws.numel(), limit_ms, _stream(stream)),
            "moe_selftest_wait_timeout")
 
 
@@ -500,7 +510,7 @@ def dense_workspace_size(layer: DenseLayer) -> int:
 def new_dense_workspace(layer: DenseLayer, device=None, stream=None) -> torch.Tensor:
     """Allocate (with torch) and initialise a workspace for the dense ``layer``."""
     ws = torch.empty(dense_workspace_size(layer), dtype=torch.uint8, device=device or "cuda")
-    _check(LIB.moe_workspace_init(ws.data_ptr(), ws.numel(), _stream(stream)), "moe_workspace_init")
+    _check(LIB.moe_workspace_init(_wsptr(ws), ws.numel(), _stream(stream)), "moe_workspace_init")
     return ws
 
 
@@ -511,7 +521,7 @@ def moe_dense_mlp(layer: DenseLayer, x, w_gate_up, w_down, out, ws, stream=None)
     _expect(w_down, "w_down", (L.H, L.I), L.down_dtype)
     _expect(out, "out", (L.T, L.H), L.dtype)
     _check(LIB.moe_dense_mlp(ctypes.byref(L.desc()), _ptr(x), _ptr(w_gate_up), _ptr(w_down),
-                             _ptr(out), ws.data_ptr(), ws.numel(), _stream(stream)),
+                             _ptr(out), _wsptr(ws), ws.numel(), _stream(stream)),
            "moe_dense_mlp")
 
 
