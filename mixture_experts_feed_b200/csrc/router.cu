@@ -15,8 +15,9 @@
 //                         split order, one thread per logit
 //   router_topk_kernel    one warp per token: selection score
 //                         sigmoid(z) + bias over the routed rows, k rounds of
-//                         a warp-shuffle argmax (ties to the lower expert id),
-//                         then the weights.  The softmax over
+//                         a warp-wide argmax (two warp reduction
+//                         instructions a round: the largest score, then the
+//                         lowest expert id holding it), then the weights.  The softmax over
 //                         log-sigmoid(z) of [selected ++ shared] equals
 //                         sigmoid(z_i) / sum sigmoid(z), which is what the
 //                         kernel evaluates, times route_scale*global_scale.
@@ -188,40 +189,42 @@ __global__ void __launch_bounds__(TK_WARPS * 32)
     return v;
   };
 
-  float sel[PL];
+  // Selection scores as order-preserving unsigned keys (a larger score has a
+  // larger key; -0 is taken as +0, a NaN score ranks with -inf, and a row
+  // past E gets key 0, below every score), so that a warp-wide maximum is one
+  // reduction instruction.
+  uint32_t key[PL];
 #pragma unroll
   for (int i = 0; i < PL; ++i) {
     const int e = lane + 32 * i;
-    const float v = e < E ? sigmoidf_(logit(e)) + bias[e] : -INFINITY;
-    sel[i] = isnan(v) ? -INFINITY : v;   // a NaN score ranks last, never breaks the argmax
+    if (e < E) {
+      float v = sigmoidf_(logit(e)) + bias[e];
+      if (isnan(v)) v = -INFINITY;   // a NaN score ranks last, never breaks the argmax
+      if (v == 0.0f) v = 0.0f;
+      const uint32_t u = __float_as_uint(v);
+      key[i] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    } else {
+      key[i] = 0u;
+    }
   }
+  // k rounds: each lane offers its best remaining score (strict '>' keeps
+  // the lowest id among its equal scores), the warp takes the largest, and
+  // among the lanes offering it the lowest expert id.
   uint32_t taken = 0;
   for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
+    uint32_t bk = 0u, bi = 0xffffffffu;
 #pragma unroll
     for (int i = 0; i < PL; ++i) {
-      const int e = lane + 32 * i;
-      const bool avail = e < E && !((taken >> i) & 1u);
-      // strict '>' keeps the lowest id among this lane's equal scores
-      if (avail && (bi == 0x7fffffff || sel[i] > bv)) {
-        bv = sel[i];
-        bi = e;
+      if (!((taken >> i) & 1u) && key[i] > bk) {
+        bk = key[i];
+        bi = static_cast<uint32_t>(lane + 32 * i);
       }
     }
-#pragma unroll
-    for (int d = 16; d > 0; d >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, d);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, d);
-      if (ov > bv || (ov == bv && oi < bi)) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    bi = __shfl_sync(0xffffffffu, bi, 0);
-    if (bi >= E) bi = 0;   // unreachable for k <= E; keeps every index in range
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (lane == 0) s_chosen[warp][j] = bi;
+    const uint32_t top = __reduce_max_sync(0xffffffffu, bk);
+    uint32_t win = __reduce_min_sync(0xffffffffu, bk == top ? bi : 0xffffffffu);
+    if (win >= static_cast<uint32_t>(E)) win = 0;   // unreachable for k <= E; keeps every index in range
+    if ((win & 31u) == static_cast<uint32_t>(lane)) taken |= 1u << (win >> 5);
+    if (lane == 0) s_chosen[warp][j] = static_cast<int>(win);
   }
   __syncwarp();
   float sg = 0.0f;

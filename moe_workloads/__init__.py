@@ -109,6 +109,10 @@ PROFILE_WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
     # the weight-streaming expert GEMMs
     Workload("adhoc-decode-T32-H6144-E16k8S1-I2048-bf16", 32, 6144, 16, 8, 1, 2048,
              "bf16", 2.5, 1.0, seed=3),
+    # the bench workload's routing (T=8192, E=128, k=8, S=1: the same top-k
+    # and the same router K split) over a narrow layer, for the router kernels
+    Workload("adhoc-T8192-H512-E128k8S1-I64-bf16", 8192, 512, 128, 8, 1, 64,
+             "bf16", 2.5, 1.0, seed=3),
 ]}
 
 
