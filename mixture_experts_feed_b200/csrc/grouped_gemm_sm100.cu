@@ -113,7 +113,13 @@ template <int MODE, bool PAIR_> struct Tile {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
   static constexpr int NARROW_STAGES = (!PAIR && MODE != kRouter) ? RING_BYTES / (A_BYTES + B_BYTES / 2) : STAGES;
-  static constexpr int MAX_STAGES = NARROW_STAGES > STAGES ? NARROW_STAGES : STAGES;
+  // Single-CTA expert launches whose tiles hold at most 32 rows (few
+  // tokens) keep 32-row A tiles, so that more stages of weights fit the
+  // ring: up to RING_BYTES / (4 KB + B_BYTES / 2) with narrow n-tiles.
+  static constexpr bool SHORT_OK = !PAIR && MODE != kRouter;
+  static constexpr int SHORT_A_BYTES = 32 * BK * 2;
+  static constexpr int MAX_STAGES = SHORT_OK ? RING_BYTES / (SHORT_A_BYTES + B_BYTES / 2)
+                                             : (NARROW_STAGES > STAGES ? NARROW_STAGES : STAGES);
   static constexpr int TILE_M = PAIR ? 2 * BM : BM;         // rows per tile
   // accumulators: two (the epilogue of one tile overlaps the next tile's
   // MMAs); the router's 160-column accumulation chains keep three, so that
@@ -150,6 +156,8 @@ struct alignas(64) GemmParams {
   int64_t split_stride;       // kRouter: elements between partial outputs
   int* tile_counter;          // tiles drawn from this counter (zero at launch), or null: the
                               // fixed order (tile unit, unit + units, ...)
+  int a_rows;                 // single-CTA expert launches: A rows a stage holds, 128, or 32
+                              // when no tile has more rows (the A maps' boxes are that high)
 };
 
 // Per epilogue warp, a 32 x 32 fp32 staging tile (row stride 36 floats:
@@ -265,12 +273,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // may use narrower tiles (more tiles for layers with few rows)
   const int bn = (PAIR || MODE == kRouter) ? BN : p.bn;
   // the stage ring: narrow single-CTA tiles (bn <= 128) take half the B bytes
-  // a stage and run NARROW_STAGES stages
+  // a stage, and 32-row A tiles a quarter of the A bytes; the ring then
+  // holds more stages.  With 32-row A tiles the M=128 MMA also reads the 96
+  // rows after them (the start of the stage's own B rows, loaded with them):
+  // those accumulator rows lie past every group and are never stored.
   const bool narrow = TL::NARROW_STAGES != TL::STAGES && bn <= 128;
-  const int stages = narrow ? TL::NARROW_STAGES : TL::STAGES;
-  const int stage_bytes = narrow ? A_BYTES + TL::B_BYTES / 2 : TL::STAGE_BYTES;
-  auto stage_a = [&](int st) { return ring + st * stage_bytes; };            // A tile of a stage
-  auto stage_b = [&](int st) { return ring + st * stage_bytes + A_BYTES; };  // its B rows
+  const int a_stage_bytes = (TL::SHORT_OK && p.a_rows == 32) ? TL::SHORT_A_BYTES : A_BYTES;
+  const int stage_bytes = a_stage_bytes + (narrow ? TL::B_BYTES / 2 : TL::B_BYTES);
+  const int stages = min(STAGES, TL::RING_BYTES / stage_bytes);
+  auto stage_a = [&](int st) { return ring + st * stage_bytes; };                  // A tile of a stage
+  auto stage_b = [&](int st) { return ring + st * stage_bytes + a_stage_bytes; };  // its B rows
   const int n_tiles = (p.N + bn - 1) / bn * ksplit;
   const int k_blocks = p.K / BK;                               // per weight part
   const int k_total = MODE == kRouter ? 3 * k_blocks : k_blocks;
@@ -446,7 +458,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int first = tile_row0 + static_cast<int>(rank) * BM + 4 * lane;   // row inside the group
       const bool lane_gathers = gather && first < gi.rows;
       const int a_bytes = gather ? (PAIR ? gathered_bytes(0) + gathered_bytes(1) : gathered_bytes(0))
-                                 : (PAIR ? 2 : 1) * A_BYTES;
+                                 : (PAIR ? 2 * A_BYTES : a_stage_bytes);
       if (gather) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -963,10 +975,13 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   // read; they are encoded over the shared operands so that every map is valid.
   const bool routed = L.E > 0 && Rk > 0;
   const bool gather = routed && x_perm == nullptr;
+  // With T <= 32 no group has more rows than T (a token takes an expert at
+  // most once), so the single-CTA launches keep 32-row A tiles
+  const int a_rows = L.T <= 32 ? 32 : BM;
   GemmParams g{};
   bool ok = (gather ? encode_a(&g.tmA[0], x, L.T, L.H, 1)
-                    : encode_a(&g.tmA[0], routed ? x_perm : x, routed ? Rk : L.T, L.H)) &&
-            encode_a(&g.tmA[1], x, L.T, L.H);
+                    : encode_a(&g.tmA[0], routed ? x_perm : x, routed ? Rk : L.T, L.H, a_rows)) &&
+            encode_a(&g.tmA[1], x, L.T, L.H, a_rows);
   if (ok && L.E > 0) ok = encode_b(&g.tmB[0], w_gate_up, L.E, 2 * L.I, L.H, BROWS);
   if (ok && L.S > 0) ok = encode_b(&g.tmB[1], ws_gate_up, L.S, 2 * L.I, L.H, BROWS);
   if (L.E == 0) g.tmB[0] = g.tmB[1];
@@ -984,6 +999,7 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   g.bn = tiling.gate_up_bn;
   g.gather_k = gather ? L.k : 0;
   g.f16 = L.down_f16 ? 1 : 0;   // h in fp16 for fp16 down projections
+  g.a_rows = a_rows;
   cudaError_t e = cudaSuccess;
   if (!do_gate_up) {
     // the activated rows are already in h
@@ -995,7 +1011,7 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
     const int ks = tiling.gate_up_ksplit;
     if (L.E != 0 || L.S != 1 || pairs || tiling.gate_up_part == nullptr) return cudaErrorInvalidValue;
     GemmParams q{};
-    ok = encode_a(&q.tmA[0], x, L.T, L.H) &&
+    ok = encode_a(&q.tmA[0], x, L.T, L.H, a_rows) &&
          encode_b(&q.tmB[0], ws_gate_up, 1, 2 * L.I, L.H, BROWS) &&
          encode_y(&q.tmY[0], tiling.gate_up_part, L.T * static_cast<int64_t>(ks), 2 * L.I);
     if (!ok) { *map_error = true; return cudaErrorInvalidValue; }
@@ -1010,6 +1026,7 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
     q.ksplit = ks;
     q.split_stride = L.T * static_cast<int64_t>(2 * L.I);
     q.bn = 256;
+    q.a_rows = a_rows;
     e = launch_mode<kDown, false>(q, num_sms, stream);
     if (e == cudaSuccess)
       e = launch_swiglu_partials(tiling.gate_up_part, ks, L.T, L.I, L.global_scale, L.down_f16,
@@ -1025,7 +1042,7 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   // ---------------- down: h [rows, I] x [H, I]^T -> y [rows, H] (fp32)
   GemmParams d{};
   const bool f16 = L.down_f16;   // h and the down weights in fp16
-  ok = encode_a(&d.tmA[0], h, Rh, L.I, BM, f16);
+  ok = encode_a(&d.tmA[0], h, Rh, L.I, a_rows, f16);
   if (ok && L.E > 0) ok = encode_b(&d.tmB[0], w_down, L.E, L.H, L.I, BROWS, f16);
   d.tmA[1] = d.tmA[0];
   if (ok && L.S > 0) ok = encode_b(&d.tmB[1], ws_down, L.S, L.H, L.I, BROWS, f16);
@@ -1053,6 +1070,7 @@ cudaError_t launch_expert_ffn_bf16(const Layer& L, const void* x, const void* x_
   d.bn = 256;
   d.f16 = f16 ? 1 : 0;
   d.y_f16 = y_f16 ? 1 : 0;
+  d.a_rows = a_rows;
   e = pairs ? launch_mode<kDown, true>(d, num_sms, stream) : cudaSuccess;
   if (e == cudaSuccess && singles) e = launch_mode<kDown, false>(d, num_sms, stream);
   return e;
