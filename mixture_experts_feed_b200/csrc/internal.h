@@ -48,6 +48,10 @@ cudaError_t launch_permute(const Layer& L, const int32_t* topk_idx, const uint8_
 // chunk == nullptr selects the workspace-free path (one block per expert).
 int64_t permute_chunk_slots(int64_t slots);
 int64_t permute_chunks(int64_t slots);
+// With a workspace and at most this many slots one kernel counts, scans and
+// scatters; the kernels launch_permute launches, the row gather included.
+constexpr int64_t kOneChunkSlots = 256;
+int permute_kernel_count(int64_t slots, bool workspace);
 
 // The workspace's status region: its first 256 bytes.  Byte 0 holds the
 // sticky device status word; bytes kTileCounterOffset .. +7 hold the tile

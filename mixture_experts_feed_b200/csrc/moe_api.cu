@@ -656,12 +656,14 @@ int32_t moe_forward_kernel_count(const moe_layer_desc_t* desc) {
   if (check_desc(desc, &L) != MOE_OK || L.T == 0) return 0;
   // router: (bf16: split + tensor-core logits | fp32: logits) + top-k (plus
   // a partial-logit sum when K is split 4 or more ways); permute: chunk
-  // counts, chunk scan, scatter, row gather; experts: gate_up + down (bf16
+  // counts, chunk scan, scatter (one kernel for at most 256 slots), row
+  // gather; experts: gate_up + down (bf16
   // with T > 128: CTA-pair launch + single-CTA launch each; bf16 with shared
   // experts: their gate_up on the side stream too, their down in the routed
   // experts' down launches); combine.
   const int experts = L.dtype == MOE_BF16 ? (L.T > 128 ? 4 : 2) + (L.S > 0 ? 1 : 0) : 2;
-  return (L.dtype == MOE_BF16 ? 2 : 1) + router_topk_launches(router_ksplit(L)) + 4 + experts + 1;
+  return (L.dtype == MOE_BF16 ? 2 : 1) + router_topk_launches(router_ksplit(L)) +
+         permute_kernel_count(L.T * L.k, true) + experts + 1;
 }
 
 moe_status_t moe_dense_workspace_size(const moe_dense_desc_t* desc, size_t* bytes) {

@@ -15,6 +15,9 @@
 //                     among earlier slots of its expert is its rank in its
 //                     warp's match group plus the earlier warps' and
 //                     iterations' counts
+//   perm_one_chunk    at most 256 slots (few tokens): the three steps above
+//                     for the one chunk in a single block of 256 threads
+//                     (a slot a thread), with the same order
 // Without one (moe_permute_noalloc): perm_count (totals only), perm_scan,
 // and perm_compact: one block per expert walks the tokens in order.
 //   gather_rows   x_perm[r] = x[perm_slot[r] / k], one warp per row,
@@ -244,6 +247,78 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// At most 256 slots: counts, offsets and the stable scatter in one block
+// (thread i holds slot i), in the order of the chunked kernels: a slot's row
+// is its expert's first row plus the earlier warps' slots of that expert
+// plus its rank in its warp's match group.
+__global__ void __launch_bounds__(256)
+    perm_one_chunk_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ pad,
+                          int64_t slots, int k, int E, int32_t* __restrict__ offsets,
+                          int32_t* __restrict__ perm_slot, int32_t* __restrict__ inv_perm,
+                          int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ int s_mem[];
+  int* s_cnt = s_mem;             // [8 warps][E]
+  int* s_base = s_mem + 8 * E;    // [E]: the counts, then each expert's first row
+  __shared__ int s_warp[8];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < 9 * E; i += blockDim.x) s_mem[i] = 0;
+  __syncthreads();
+  int e = -1;   // this thread's slot's expert, or -1
+  if (tid < slots) {
+    const bool padded = pad != nullptr && pad[tid / k] != 0;
+    const int v = idx[tid];
+    if (padded) {
+      inv_perm[tid] = -1;
+    } else if (v < 0 || v >= E) {
+      record_status(status, DEV_BAD_EXPERT_ID);
+      inv_perm[tid] = -1;
+    } else {
+      e = v;
+    }
+  }
+  if (e >= 0) atomicAdd(&s_base[e], 1);
+  __syncthreads();
+  // exclusive scan of the counts: thread t takes experts [t * per, t * per + per)
+  const int per = (E + 255) / 256;   // at most 4 (E <= 1024)
+  int c[4];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int ee = tid * per + i;
+    c[i] = (i < per && ee < E) ? s_base[ee] : 0;
+    sum += c[i];
+  }
+  int total = 0;
+  int run = block_excl_scan_256(sum, s_warp, total);   // its barriers order the reads above
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int ee = tid * per + i;
+    if (i < per && ee < E) {
+      s_base[ee] = run;
+      offsets[ee] = run;
+    }
+    run += c[i];
+  }
+  if (tid == 0) offsets[E] = total;
+  const uint32_t grp = __match_any_sync(0xffffffffu, e);
+  const int rank = __popc(grp & ((1u << lane) - 1u));
+  if (e >= 0 && rank == 0) s_cnt[warp * E + e] = __popc(grp);
+  __syncthreads();
+  if (e >= 0) {
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += s_cnt[w * E + e];
+    const int64_t pos = static_cast<int64_t>(s_base[e]) + before + rank;
+    if (pos >= 0 && pos < slots) {
+      perm_slot[pos] = tid;
+      inv_perm[tid] = static_cast<int32_t>(pos);
+    } else {
+      record_status(status, DEV_BAD_ROW);
+    }
+  }
+}
+
 constexpr int COMPACT_THREADS = 1024;
 
 __global__ void __launch_bounds__(COMPACT_THREADS)
@@ -350,14 +425,26 @@ int64_t permute_chunks(int64_t slots) {
   return slots == 0 ? 0 : ceil_div(slots, permute_chunk_slots(slots));
 }
 
+int permute_kernel_count(int64_t slots, bool workspace) {
+  return workspace && slots <= kOneChunkSlots ? 2 : 4;   // with the row gather
+}
+
 cudaError_t launch_permute(const Layer& L, const int32_t* topk_idx, const uint8_t* padding_mask,
                            const void* x, int32_t* offsets, int32_t* perm_slot, int32_t* inv_perm,
                            void* x_perm, int32_t* counts, int32_t* chunk, int32_t* status,
                            int num_sms, cudaStream_t stream) {
-  cudaError_t err = cudaMemsetAsync(counts, 0, sizeof(int32_t) * L.E, stream);
-  if (err != cudaSuccess) return err;
   const int64_t slots = L.T * L.k;
-  if (chunk != nullptr) {
+  cudaError_t err = cudaSuccess;
+  if (chunk != nullptr && slots <= kOneChunkSlots) {
+    err = launch_chained(perm_one_chunk_kernel, 1, 256, sizeof(int) * 9 * L.E, stream, topk_idx,
+                         padding_mask, slots, L.k, L.E, offsets, perm_slot, inv_perm, status);
+  } else {
+    err = cudaMemsetAsync(counts, 0, sizeof(int32_t) * L.E, stream);
+  }
+  if (err != cudaSuccess) return err;
+  if (chunk != nullptr && slots <= kOneChunkSlots) {
+    // counted, scanned and scattered above
+  } else if (chunk != nullptr) {
     const int64_t cs = permute_chunk_slots(slots);
     const int nc = static_cast<int>(permute_chunks(slots));
     err = launch_chained(perm_chunk_count_kernel, nc, 256, sizeof(int) * L.E, stream, topk_idx,
