@@ -159,6 +159,24 @@ def test_padding_mask():
     assert torch.equal(f["out"], r["out"])
 
 
+@pytest.mark.parametrize("T", [32, 33], ids=["256-slots-one-block", "264-slots-chunked"])
+def test_few_slot_permutation_with_padding(T):
+    """T * k = 256 slots take the one-block permutation, 264 the chunked
+    kernels: with a padding mask and E = 16 (many rows an expert, so the
+    stable order within an expert matters) both are bit-exact against the
+    oracle, and the layer meets the bar."""
+    w, inputs = small_case(T, 256, 16, 8, 1, 128, seed=43)
+    g = torch.Generator().manual_seed(44)
+    pm = torch.rand(w.T, generator=g) < 0.3
+    L = moe.Layer.from_workload(w)
+    r = run_chain(L, to_device(inputs), padding_mask=pm)
+    assert int(r["offsets"][-1]) == int((~pm).sum()) * w.k
+    assert bool((r["inv_perm"].view(w.T, w.k)[pm] == -1).all())
+    check_all(w, inputs, r, padding_mask=pm)
+    f = run_forward(L, to_device(inputs), padding_mask=pm)
+    assert torch.equal(f["out"], r["out"])
+
+
 @pytest.mark.parametrize("route_scale,global_scale", [(8.0, 0.5), (1.0, 2.0)])
 def test_route_and_global_scales(route_scale, global_scale):
     """Other scales than the workloads' 2.5 x 1: the weights of every token
