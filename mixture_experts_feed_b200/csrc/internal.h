@@ -32,7 +32,7 @@ cudaError_t launch_router_split(const Layer& L, const float* w_router, void* w_p
 cudaError_t launch_router_logits(const Layer& L, const void* x, const float* w_router,
                                  float* logits, int ld, cudaStream_t stream);
 // kernels launch_router_topk launches for this K-split count (1 or 2)
-int router_topk_launches(int ksplit);
+int router_topk_launches(int ksplit, int64_t T);
 cudaError_t launch_router_topk(const Layer& L, const float* logits, int ld, int ksplit,
                                const float* corr_bias,
                                float* topk_w, int32_t* topk_idx, float* shared_gamma,

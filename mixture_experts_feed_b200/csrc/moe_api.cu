@@ -662,7 +662,7 @@ int32_t moe_forward_kernel_count(const moe_layer_desc_t* desc) {
   // experts: their gate_up on the side stream too, their down in the routed
   // experts' down launches); combine.
   const int experts = L.dtype == MOE_BF16 ? (L.T > 128 ? 4 : 2) + (L.S > 0 ? 1 : 0) : 2;
-  return (L.dtype == MOE_BF16 ? 2 : 1) + router_topk_launches(router_ksplit(L)) +
+  return (L.dtype == MOE_BF16 ? 2 : 1) + router_topk_launches(router_ksplit(L), L.T) +
          permute_kernel_count(L.T * L.k, true) + experts + 1;
 }
 

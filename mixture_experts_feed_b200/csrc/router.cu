@@ -11,7 +11,7 @@
 //                         fp32 FFMA, tiled 64 tokens x 64 rows x 32 K.
 //   Both give fp32 logits for all E routed + S shared rows of the gate bank
 //   (the gate runs in fp32: gate_precision=torch.float32).
-//   router_sum_splits_kernel  (many K splits only) partial logits summed in
+//   router_sum_splits_kernel  (many K splits, few tokens) partial logits summed in
 //                         split order, one thread per logit
 //   router_topk_kernel    one warp per token: selection score
 //                         sigmoid(z) + bias over the routed rows, k rounds of
@@ -143,8 +143,11 @@ __global__ void __launch_bounds__(RL_THREADS)
 __device__ __forceinline__ float sigmoidf_(float v) { return 1.0f / (1.0f + expf(-v)); }
 
 constexpr int TK_WARPS = 8;
-// From this many K splits on, a separate kernel sums the partial logits first.
+// From this many K splits on, and below this many tokens (a top-k grid of
+// few warps, each of which would read every split of its logits), a
+// separate kernel sums the partial logits first.
 constexpr int kSumSplitsFrom = 4;
+constexpr int64_t kSumSplitsBelowT = 2048;
 
 // PL: routed scores held per lane (E <= 32 * PL).
 // Sum the K-split partial logits into split 0, in split order, one thread
@@ -263,12 +266,14 @@ cudaError_t launch_router_logits(const Layer& L, const void* x, const float* w_r
                         static_cast<const float*>(x), w_router, logits, L.T, L.H, NE, ld);
 }
 
-int router_topk_launches(int ksplit) { return ksplit >= kSumSplitsFrom ? 2 : 1; }
+int router_topk_launches(int ksplit, int64_t T) {
+  return ksplit >= kSumSplitsFrom && T < kSumSplitsBelowT ? 2 : 1;
+}
 
 cudaError_t launch_router_topk(const Layer& L, const float* logits, int ld, int ksplit,
                                const float* corr_bias, float* topk_w, int32_t* topk_idx,
                                float* shared_gamma, cudaStream_t stream) {
-  if (router_topk_launches(ksplit) == 2) {
+  if (router_topk_launches(ksplit, L.T) == 2) {
     const int NE = L.E + L.S;
     const int64_t n = L.T * static_cast<int64_t>(NE);
     const unsigned sgrid = static_cast<unsigned>(std::min<int64_t>(ceil_div(n, 256), 148 * 8));

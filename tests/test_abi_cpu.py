@@ -60,12 +60,13 @@ def test_workspace_size_covers_intermediates(w):
     # down joins the routed experts' down launches)
     experts = ((4 if w.T > 128 else 2) + (1 if w.S else 0)) if w.dtype == "bf16" else 2
     # tensor-core router: K split across ~148 CTAs when T is small; from 4
-    # splits on a separate kernel sums the partial logits before the top-k
+    # splits on, below 2048 tokens, a separate kernel sums the partial logits
+    # before the top-k
     ksplit = 1
     if w.dtype == "bf16":
         tiles = -(-w.T // 128) * -(-(w.E + w.S) // 160)
         ksplit = max(1, min(32, 148 // tiles))
-    router = (2 if w.dtype == "bf16" else 1) + (2 if ksplit >= 4 else 1)
+    router = (2 if w.dtype == "bf16" else 1) + (2 if ksplit >= 4 and w.T < 2048 else 1)
     # permute: chunk counts, chunk scan, scatter, row gather (at most 256
     # slots: one kernel for the first three)
     permute = 2 if w.T * w.k <= 256 else 4
