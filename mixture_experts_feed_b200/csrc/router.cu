@@ -11,8 +11,9 @@
 //                         fp32 FFMA, tiled 64 tokens x 64 rows x 32 K.
 //   Both give fp32 logits for all E routed + S shared rows of the gate bank
 //   (the gate runs in fp32: gate_precision=torch.float32).
-//   router_sum_splits_kernel  (many K splits, few tokens) partial logits summed in
-//                         split order, one thread per logit
+//   router_sum_splits_kernel  (many K splits, few tokens) partial logits summed
+//                         by eight threads a logit: eighths of the splits in
+//                         order, then a fixed tree
 //   router_topk_kernel    one warp per token: selection score
 //                         sigmoid(z) + bias over the routed rows, k rounds of
 //                         a warp-wide argmax (two warp reduction
@@ -149,28 +150,40 @@ constexpr int TK_WARPS = 8;
 constexpr int kSumSplitsFrom = 4;
 constexpr int64_t kSumSplitsBelowT = 2048;
 
-// PL: routed scores held per lane (E <= 32 * PL).
-// Sum the K-split partial logits into split 0, in split order, one thread
-// per logit over the whole grid (the same additions, in the same order, as
-// the top-k kernel makes when it reads the partials itself).  Used when the
-// split count is large (few tokens): there the top-k kernel has few warps.
+// Sum the K-split partial logits into split 0 (many splits, few tokens).
+// Eight consecutive lanes of a warp hold one logit: lane q adds the splits
+// [ks * q / 8, ks * (q + 1) / 8) in order, then the eight sums combine in a
+// fixed tree (neighbours, then pairs, then fours), which every one of the
+// eight lanes computes alike; lane 0 of the eight stores it.  Short chains
+// over 8x the threads: the launch is latency-bound.
 __global__ void router_sum_splits_kernel(float* __restrict__ z, int ld, int ksplit, int64_t T,
                                          int NE) {
   pdl_wait();
   pdl_trigger();
   const int64_t split = T * static_cast<int64_t>(ld);
-  const int64_t n = T * static_cast<int64_t>(NE);
+  const int64_t total = T * static_cast<int64_t>(NE) * 8;   // eight threads a logit
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
-    const int64_t t = i / NE;
-    const int e = static_cast<int>(i - t * NE);
-    float* zt = z + t * ld + e;
-    float v = zt[0];
-    for (int s2 = 1; s2 < ksplit; ++s2) v += zt[s2 * split];
-    zt[0] = v;
+  const int lane = threadIdx.x & 31, q = lane & 7;
+  // whole warps iterate together (the shuffles below take all 32 lanes)
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31);
+       base < total; base += stride) {
+    const int64_t i = (base + lane) >> 3;                   // this lane's logit
+    const bool live = base + lane < total;
+    float* zt = z;
+    float v = 0.0f;
+    if (live) {
+      const int64_t t = i / NE;
+      zt = z + t * ld + (i - t * NE);
+      for (int s2 = ksplit * q / 8; s2 < ksplit * (q + 1) / 8; ++s2) v += zt[s2 * split];
+    }
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    if (live && q == 0) zt[0] = v;
   }
 }
 
+// PL: routed scores held per lane (E <= 32 * PL).
 template <int PL>
 __global__ void __launch_bounds__(TK_WARPS * 32)
     router_topk_kernel(const float* __restrict__ z, int ld, int ksplit,
@@ -275,7 +288,7 @@ cudaError_t launch_router_topk(const Layer& L, const float* logits, int ld, int 
                                float* shared_gamma, cudaStream_t stream) {
   if (router_topk_launches(ksplit, L.T) == 2) {
     const int NE = L.E + L.S;
-    const int64_t n = L.T * static_cast<int64_t>(NE);
+    const int64_t n = L.T * static_cast<int64_t>(NE) * 8;   // eight threads a logit
     const unsigned sgrid = static_cast<unsigned>(std::min<int64_t>(ceil_div(n, 256), 148 * 8));
     const cudaError_t e = launch_chained(router_sum_splits_kernel, sgrid, 256, 0, stream,
                                          const_cast<float*>(logits), ld, ksplit, L.T, NE);
